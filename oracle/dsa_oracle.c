@@ -1,0 +1,292 @@
+/*
+ * dsa_oracle.c -- float64 CPU oracle for the DSA sparse-attention step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or constant with the CUDA library; the two only read the same
+ * seeded input bytes.
+ *
+ * What it computes, step by step, in the order the pages give them:
+ *
+ *  1. Lightning Indexer relevance scoring with head-weight weighting.
+ *     "Day0 Adaptation and Performance Optimization for Novel Long-Sequence
+ *     Reasoning Models", section 1 (Sparse Index Branch) and section 3 (the
+ *     index stage fuses relevance scoring, head-weight weighting and Top-K);
+ *     "Day0 Adaptation and Sparse Attention Optimization for Long-Sequence LLM
+ *     Inference", section 4 (index generation = scoring, multi-head weight
+ *     aggregation, Top-K).  The pages give no formula; the gate used here is
+ *     the ReLU form of the Lightning Indexer:
+ *         score(t, s) = sum_h w[t,h] * max(0, sum_d q[t,h,d] * k[s,d])
+ *     for every position s the query token t can see (0..pos(t), causal).
+ *     fp8 keys: k[s,d] = e4m3(code[s,d]) * scale[s, d/64] (one fp32 scale per
+ *     64 contiguous elements of a key; "Day0 Adaptation and Performance
+ *     Optimization ...", section 4, every N elements share a scaling factor).
+ *
+ *  2. Top-K selection.  "Large Model Inference Acceleration: Day-0
+ *     Adaptation ...", section 1.1 (a Top-K pass picks the most important
+ *     positions).  Done here as a FULL SORT of the visible positions by
+ *     (score descending, position ascending) -- the lower position wins a
+ *     tie -- keeping the first min(K, visible).  The kept set is written in
+ *     ascending position order and padded with -1.
+ *
+ *  3. Sparse Flash Attention over the selected rows of the MLA latent cache.
+ *     "Day0 Adaptation and Sparse Attention Optimization ...", section 4
+ *     (the sparse read stage gathers the selected KV entries and computes
+ *     attention); "Optimizing and Deploying Ultra-Long Sequence Inference
+ *     Architectures", section I.  Each cache row is [512 latent | 64 RoPE];
+ *     the key is the whole 576-wide row, the value is the 512-wide latent:
+ *         l_j  = sm_scale * sum_{d<576} q[t,g,d] * kv[s_j,d]
+ *         p_j  = exp(l_j - max l) / sum_i exp(l_i - max l)
+ *         o    = sum_j p_j * kv[s_j, 0:512],   lse = max l + ln sum_i exp(l_i - max l)
+ *     Rows with index -1 are skipped.
+ *
+ * All arithmetic is IEEE float64, no fused multiply-add contraction
+ * (built with -ffp-contract=off), summation in index order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_BLOCK 64
+#define ORACLE_DQK 576
+#define ORACLE_DV 512
+
+/* bf16 bits -> double: the bf16 value is the top half of a float32. */
+static double bf16_to_f64(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* OCP e4m3fn code -> double.  Sign bit, 4 exponent bits (bias 7), 3 mantissa
+ * bits; exponent 0 is subnormal (2^-6 * m/8); S.1111.111 is NaN (returned as
+ * NaN; the generator never produces it). */
+double oracle_e4m3_to_f64(uint8_t c) {
+    int s = (c >> 7) & 1, e = (c >> 3) & 0xF, m = c & 7;
+    double v;
+    if (e == 0xF && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+typedef struct {
+    int32_t B, T, H_I, D_I, K;
+    int32_t key_fp8;                 /* 0: bf16 keys, 1: e4m3 codes + scales */
+    const int32_t* seq_lens;         /* [B] */
+    const int32_t* cu_q;             /* [B+1] */
+    const int32_t* block_table;      /* [B, max_blocks] */
+    int32_t max_blocks;
+    const uint16_t* q_idx;           /* [T, H_I, D_I] bf16 bits */
+    const float* w;                  /* [T, H_I] */
+    const void* k_idx;               /* [nblk, 64, D_I] bf16 bits or u8 codes */
+    const float* k_scale;            /* [nblk, 64, D_I/64] or NULL */
+} oracle_indexer_args;
+
+/* Sequence and absolute position of query token t. */
+static void token_place(const int32_t* cu_q, const int32_t* seq_lens, int B, int t,
+                        int* b_out, int64_t* pos_out) {
+    int b = 0;
+    while (b + 1 < B + 1 && cu_q[b + 1] <= t) b++;
+    int nq = cu_q[b + 1] - cu_q[b];
+    *b_out = b;
+    *pos_out = (int64_t)seq_lens[b] - nq + (t - cu_q[b]);
+}
+
+static int64_t phys_row(const oracle_indexer_args* a, int b, int64_t pos) {
+    int64_t blk = a->block_table[(int64_t)b * a->max_blocks + pos / ORACLE_BLOCK];
+    return blk * ORACLE_BLOCK + pos % ORACLE_BLOCK;
+}
+
+/* Key element d of logical position pos of sequence b, as a double. */
+static double key_elem(const oracle_indexer_args* a, int64_t row, int d) {
+    if (!a->key_fp8) {
+        const uint16_t* k = (const uint16_t*)a->k_idx;
+        return bf16_to_f64(k[row * a->D_I + d]);
+    } else {
+        const uint8_t* k = (const uint8_t*)a->k_idx;
+        double sc = (double)a->k_scale[row * (a->D_I / 64) + d / 64];
+        return oracle_e4m3_to_f64(k[row * a->D_I + d]) * sc;
+    }
+}
+
+/* Step 1 for one token: scores of positions 0..pos into out[0..pos]. */
+static void score_token(const oracle_indexer_args* a, int t, double* out, int64_t* npos_out) {
+    int b;
+    int64_t pos;
+    token_place(a->cu_q, a->seq_lens, a->B, t, &b, &pos);
+    int H = a->H_I, D = a->D_I;
+    double* q = (double*)malloc(sizeof(double) * (size_t)H * D);
+    double* k = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int i = 0; i < H * D; i++) q[i] = bf16_to_f64(a->q_idx[(int64_t)t * H * D + i]);
+    for (int64_t s = 0; s <= pos; s++) {
+        int64_t row = phys_row(a, b, s);
+        for (int d = 0; d < D; d++) k[d] = key_elem(a, row, d);
+        double acc = 0.0;
+        for (int h = 0; h < H; h++) {
+            double dot = 0.0;
+            for (int d = 0; d < D; d++) dot += q[h * D + d] * k[d];
+            double relu = dot > 0.0 ? dot : 0.0;
+            acc += (double)a->w[(int64_t)t * H + h] * relu;
+        }
+        out[s] = acc;
+    }
+    *npos_out = pos + 1;
+    free(q);
+    free(k);
+}
+
+typedef struct { double score; int64_t pos; } scored_pos;
+
+/* Order: score descending, then position ascending (lower position wins). */
+static int cmp_rank(const void* x, const void* y) {
+    const scored_pos* a = (const scored_pos*)x;
+    const scored_pos* b = (const scored_pos*)y;
+    if (a->score > b->score) return -1;
+    if (a->score < b->score) return 1;
+    return (a->pos > b->pos) - (a->pos < b->pos);
+}
+
+static int cmp_i64(const void* x, const void* y) {
+    int64_t a = *(const int64_t*)x, b = *(const int64_t*)y;
+    return (a > b) - (a < b);
+}
+
+/*
+ * Steps 1+2 for the tokens listed in `tokens` (n_tokens entries).
+ * out_idx   [n_tokens, K] int32: selected positions ascending, -1 padded.
+ * out_score [n_tokens, K] double: score of each selected position (NaN pad).
+ * out_kth   [n_tokens] double: the K-th largest visible score (smallest kept
+ *           score), or -inf when fewer than K positions are visible.
+ * out_all   optional [n_tokens, all_stride] double: every visible score.
+ */
+int oracle_indexer_topk(const oracle_indexer_args* a, const int32_t* tokens, int n_tokens,
+                        int32_t* out_idx, double* out_score, double* out_kth,
+                        double* out_all, int64_t all_stride) {
+    int rc = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n_tokens; i++) {
+        int t = tokens[i];
+        int b;
+        int64_t pos;
+        token_place(a->cu_q, a->seq_lens, a->B, t, &b, &pos);
+        int64_t nvis = pos + 1;
+        double* sc = (double*)malloc(sizeof(double) * (size_t)nvis);
+        scored_pos* sp = (scored_pos*)malloc(sizeof(scored_pos) * (size_t)nvis);
+        int64_t* keep = (int64_t*)malloc(sizeof(int64_t) * (size_t)(a->K > 0 ? a->K : 1));
+        if (!sc || !sp || !keep) { rc = -1; free(sc); free(sp); free(keep); continue; }
+        score_token(a, t, sc, &nvis);
+        if (out_all) memcpy(out_all + (int64_t)i * all_stride, sc, sizeof(double) * (size_t)nvis);
+        for (int64_t s = 0; s < nvis; s++) { sp[s].score = sc[s]; sp[s].pos = s; }
+        qsort(sp, (size_t)nvis, sizeof(scored_pos), cmp_rank);
+        int64_t nk = nvis < a->K ? nvis : a->K;
+        for (int64_t j = 0; j < nk; j++) keep[j] = sp[j].pos;
+        out_kth[i] = (nvis >= a->K && a->K > 0) ? sp[a->K - 1].score : -INFINITY;
+        qsort(keep, (size_t)nk, sizeof(int64_t), cmp_i64);
+        for (int64_t j = 0; j < a->K; j++) {
+            int64_t o = (int64_t)i * a->K + j;
+            out_idx[o] = j < nk ? (int32_t)keep[j] : -1;
+            out_score[o] = j < nk ? sc[keep[j]] : NAN;
+        }
+        free(sc);
+        free(sp);
+        free(keep);
+    }
+    return rc;
+}
+
+/* Step 1 alone: the score of each (token, position) pair listed. */
+int oracle_indexer_score_pairs(const oracle_indexer_args* a, const int32_t* tokens,
+                               const int64_t* positions, int64_t n_pairs, double* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n_pairs; i++) {
+        int b;
+        int64_t pos;
+        int t = tokens[i];
+        token_place(a->cu_q, a->seq_lens, a->B, t, &b, &pos);
+        int64_t s = positions[i];
+        if (s < 0 || s > pos) { out[i] = NAN; continue; }
+        int64_t row = phys_row(a, b, s);
+        double acc = 0.0;
+        for (int h = 0; h < a->H_I; h++) {
+            double dot = 0.0;
+            for (int d = 0; d < a->D_I; d++)
+                dot += bf16_to_f64(a->q_idx[((int64_t)t * a->H_I + h) * a->D_I + d]) * key_elem(a, row, d);
+            acc += (double)a->w[(int64_t)t * a->H_I + h] * (dot > 0.0 ? dot : 0.0);
+        }
+        out[i] = acc;
+    }
+    return 0;
+}
+
+typedef struct {
+    int32_t B, T, H, K;
+    double sm_scale;
+    const int32_t* seq_lens;
+    const int32_t* cu_q;
+    const int32_t* block_table;
+    int32_t max_blocks;
+    const uint16_t* q;               /* [T, H, 576] bf16 bits */
+    const uint16_t* kv;              /* [nblk, 64, 576] bf16 bits */
+    const int32_t* idx;              /* [T, K] logical positions, -1 = skip */
+} oracle_attn_args;
+
+/*
+ * Step 3 for the tokens listed: out_o [n_tokens, H, 512] double,
+ * out_lse [n_tokens, H] double (-inf when no row is selected; o is then 0).
+ */
+int oracle_sparse_attn(const oracle_attn_args* a, const int32_t* tokens, int n_tokens,
+                       double* out_o, double* out_lse) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n_tokens; i++) {
+        int t = tokens[i];
+        int b = 0;
+        while (b + 1 < a->B + 1 && a->cu_q[b + 1] <= t) b++;
+        const int32_t* sel = a->idx + (int64_t)t * a->K;
+        double* logit = (double*)malloc(sizeof(double) * (size_t)a->K);
+        int64_t* rows = (int64_t*)malloc(sizeof(int64_t) * (size_t)a->K);
+        int n = 0;
+        for (int j = 0; j < a->K; j++) {
+            if (sel[j] < 0) continue;
+            int64_t p = sel[j];
+            rows[n++] = (int64_t)a->block_table[(int64_t)b * a->max_blocks + p / ORACLE_BLOCK] * ORACLE_BLOCK
+                        + p % ORACLE_BLOCK;
+        }
+        for (int g = 0; g < a->H; g++) {
+            const uint16_t* qg = a->q + ((int64_t)t * a->H + g) * ORACLE_DQK;
+            double* o = out_o + ((int64_t)i * a->H + g) * ORACLE_DV;
+            for (int d = 0; d < ORACLE_DV; d++) o[d] = 0.0;
+            if (n == 0) { out_lse[(int64_t)i * a->H + g] = -INFINITY; continue; }
+            double m = -INFINITY;
+            for (int j = 0; j < n; j++) {
+                const uint16_t* kr = a->kv + rows[j] * ORACLE_DQK;
+                double dot = 0.0;
+                for (int d = 0; d < ORACLE_DQK; d++) dot += bf16_to_f64(qg[d]) * bf16_to_f64(kr[d]);
+                logit[j] = a->sm_scale * dot;
+                if (logit[j] > m) m = logit[j];
+            }
+            double den = 0.0;
+            for (int j = 0; j < n; j++) den += exp(logit[j] - m);
+            for (int j = 0; j < n; j++) {
+                double p = exp(logit[j] - m) / den;
+                const uint16_t* kr = a->kv + rows[j] * ORACLE_DQK;
+                for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d]);
+            }
+            out_lse[(int64_t)i * a->H + g] = m + log(den);
+        }
+        free(logit);
+        free(rows);
+    }
+    return 0;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

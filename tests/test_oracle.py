@@ -1,0 +1,268 @@
+"""Pins for the float64 oracle, checked against things other than itself.
+
+* hand-worked cases from tests/golden/hand_cases.json (derived by hand);
+* special cases that reduce to library routines: with one head and w=1 the
+  indexer is ReLU(q.k) ranked by numpy.lexsort; with K >= context the sparse
+  attention is dense causal softmax attention computed by torch in float64;
+* the e4m3 decode of all 256 codes against torch.float8_e4m3fn;
+* invariants: page permutation, positive rescaling of w, convex outputs,
+  a dominant logit;
+* the planted million-token workload: its Top-K must be the planted set;
+* exactness: integer-valued indexer inputs give scores equal to an
+  integer-arithmetic evaluation.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from indexer_top_sparse_lightning_b200 import workloads as W
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")))
+
+
+def manual_workload(q_idx_f, w, keys_f, *, K, key_dtype="bf16", k_codes=None, k_scale=None,
+                    q_mla=None, kv=None, H=1, sm_scale=1.0):
+    """One sequence, one query token at the last position; identity paging."""
+    q_idx_f = np.asarray(q_idx_f, np.float32)
+    H_I, D_I = q_idx_f.shape
+    L = len(keys_f) if keys_f is not None else k_codes.shape[0]
+    nblk = (L + W.BLOCK - 1) // W.BLOCK
+    rows = nblk * W.BLOCK
+    if key_dtype == "bf16":
+        kk = np.zeros((rows, D_I), np.float32)
+        kk[:L] = np.asarray(keys_f, np.float32)
+        k_idx = W.to_bf16_bits(kk).reshape(nblk, W.BLOCK, D_I)
+        ks = None
+    else:
+        cc = np.zeros((rows, D_I), np.uint8)
+        cc[:L] = k_codes
+        k_idx = cc.reshape(nblk, W.BLOCK, D_I)
+        ss = np.ones((rows, D_I // 64), np.float32)
+        ss[:L] = k_scale
+        ks = ss.reshape(nblk, W.BLOCK, D_I // 64)
+    if kv is None:
+        kv = np.zeros((nblk, W.BLOCK, W.D_QK), np.uint16)
+        q_mla = np.zeros((1, H, W.D_QK), np.uint16)
+    return W.Workload(name="manual", B=1, T=1, H_I=H_I, D_I=D_I, H=H, K=K, key_dtype=key_dtype,
+                      seq_lens=np.array([L], np.int32), cu_q=np.array([0, 1], np.int32),
+                      block_table=np.arange(nblk, dtype=np.int32)[None, :], num_blocks=nblk,
+                      q_idx=W.to_bf16_bits(q_idx_f)[None], w=np.asarray(w, np.float32)[None],
+                      k_idx=k_idx, k_scale=ks, q=q_mla, kv=kv, sm_scale=sm_scale)
+
+
+# ----------------------------------------------------------------------------- hand cases
+
+def test_hand_indexer_relu_gate_weights_and_tie():
+    g = GOLD["indexer_relu_tie"]
+    for k_str, want in g["topk"].items():
+        wl = manual_workload(g["q"], g["w"], g["keys"], K=int(k_str))
+        r = oracle.indexer_topk(wl, want_all_scores=True)
+        assert r["idx"][0].tolist() == want
+        np.testing.assert_array_equal(r["all"][0, :3], np.array(g["scores"]))
+
+
+def test_hand_fp8_scale_groups():
+    g = GOLD["fp8_scale_groups"]
+    q = np.zeros((1, 128), np.float32)
+    q[0, 0] = 1.0
+    q[0, 64] = 1.0
+    codes = np.zeros((1, 128), np.uint8)
+    codes[0, 0] = g["code0"]
+    codes[0, 64] = g["code64"]
+    wl = manual_workload(q, [1.0], None, K=1, key_dtype="fp8", k_codes=codes,
+                         k_scale=np.array([g["scales"]], np.float32))
+    r = oracle.indexer_topk(wl, want_all_scores=True)
+    assert r["all"][0, 0] == g["score"]
+
+
+def test_hand_softmax_two_rows():
+    g = GOLD["softmax_two_rows"]
+    q = np.zeros((1, 1, W.D_QK), np.float32)
+    q[0, 0, 512] = 1.0
+    kvf = np.zeros((1, W.BLOCK, W.D_QK), np.float32)
+    kvf[0, 0, 512] = 2.0
+    kvf[0, 0, 0] = 1.0
+    kvf[0, 1, 1] = 1.0
+    wl = manual_workload(np.zeros((1, 64)), [0.0], np.zeros((2, 64)), K=2, H=1,
+                         q_mla=W.to_bf16_bits(q), kv=W.to_bf16_bits(kvf), sm_scale=math.log(3.0) / 2)
+    o, lse = oracle.sparse_attn(wl, np.array([[0, 1]], np.int32))
+    assert abs(o[0, 0, 0] - g["o0"]) < 1e-15
+    assert abs(o[0, 0, 1] - g["o1"]) < 1e-15
+    assert np.all(o[0, 0, 2:] == 0.0)
+    assert abs(lse[0, 0] - g["lse"]) < 1e-14
+
+
+# ----------------------------------------------------------------------------- library routines
+
+def test_e4m3_decode_all_codes_vs_torch():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_to_f64(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert set(np.nonzero(nan)[0].tolist()) == {0x7F, 0xFF}
+    assert np.array_equal(np.isnan(got), nan)
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+
+
+def test_single_head_unit_weight_is_relu_dot_lexsort():
+    rng = np.random.default_rng(7)
+    L, D = 700, 128
+    q = rng.standard_normal((1, D)).astype(np.float32)
+    keys = rng.standard_normal((L, D)).astype(np.float32)
+    wl = W.make_workload("x", seq_lens=[L], nq=1, H_I=1, D_I=D, H=1, K=100, seed=3, with_kv=False)
+    # overwrite with our own draws so the reference below sees the same bf16 values
+    wl.q_idx = W.to_bf16_bits(q)[None]
+    wl.w = np.ones((1, 1), np.float32)
+    kb = W.to_bf16_bits(keys)
+    phys = np.zeros((wl.num_blocks * W.BLOCK, D), np.uint16)
+    pos = np.arange(L)
+    prow = wl.block_table[0, pos // W.BLOCK].astype(np.int64) * W.BLOCK + pos % W.BLOCK
+    phys[prow] = kb
+    wl.k_idx = phys.reshape(wl.num_blocks, W.BLOCK, D)
+    qd = W.bf16_bits_to_f32(wl.q_idx[0, 0]).astype(np.float64)
+    kd = W.bf16_bits_to_f32(kb).astype(np.float64)
+    s = np.maximum(kd @ qd, 0.0)
+    order = np.lexsort((pos, -s))          # score descending, then position ascending
+    for K in (1, 37, 100, 699, 700, 701):
+        wl.K = K
+        r = oracle.indexer_topk(wl)
+        want = np.sort(order[:min(K, L)])
+        got = r["idx"][0]
+        assert np.array_equal(got[:len(want)], want)
+        assert np.all(got[len(want):] == -1)
+
+
+def _dense_causal_reference(wl):
+    """torch float64 dense attention over all visible rows of each token."""
+    seq, pos = wl.token_seq(), wl.token_pos()
+    out_o = []
+    out_l = []
+    for t in range(wl.T):
+        b = int(seq[t])
+        p = np.arange(pos[t] + 1)
+        rows = wl.block_table[b, p // W.BLOCK].astype(np.int64) * W.BLOCK + p % W.BLOCK
+        kv = torch.from_numpy(W.bf16_bits_to_f32(wl.kv.reshape(-1, W.D_QK)[rows]).astype(np.float64))
+        q = torch.from_numpy(W.bf16_bits_to_f32(wl.q[t]).astype(np.float64))
+        logits = (q @ kv.T) * wl.sm_scale
+        out_o.append((torch.softmax(logits, dim=-1) @ kv[:, :512]).numpy())
+        out_l.append(torch.logsumexp(logits, dim=-1).numpy())
+    return np.stack(out_o), np.stack(out_l)
+
+
+def test_k_at_least_context_equals_dense_causal_attention():
+    wl = W.make_workload("dense", seq_lens=[70, 130, 5], nq=[3, 2, 1], H_I=4, D_I=64, H=8, K=160,
+                         seed=11)
+    r = oracle.indexer_topk(wl)
+    pos = wl.token_pos()
+    for t in range(wl.T):      # every visible position is selected
+        n = int(pos[t]) + 1
+        assert r["idx"][t, :n].tolist() == list(range(n))
+        assert np.all(r["idx"][t, n:] == -1)
+    o, lse = oracle.sparse_attn(wl, r["idx"])
+    ro, rl = _dense_causal_reference(wl)
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- invariants
+
+def test_page_permutation_invariance():
+    a = W.make_workload("p", seq_lens=[300, 1000], nq=[1, 2], H_I=8, D_I=128, H=4, K=64, seed=5,
+                        shuffle=False)
+    b = W.make_workload("p", seq_lens=[300, 1000], nq=[1, 2], H_I=8, D_I=128, H=4, K=64, seed=5,
+                        shuffle=False)
+    # move every physical page of b to a permuted slot, same logical content
+    rng = np.random.default_rng(0)
+    perm = rng.permutation(b.num_blocks)
+    for arr_name in ("k_idx", "kv"):
+        src = getattr(a, arr_name)
+        dst = np.empty_like(src)
+        dst[perm] = src
+        setattr(b, arr_name, dst)
+    tbl = b.block_table.copy()
+    tbl[tbl >= 0] = perm[tbl[tbl >= 0]]
+    b.block_table = tbl
+    ra, rb = oracle.indexer_topk(a), oracle.indexer_topk(b)
+    np.testing.assert_array_equal(ra["idx"], rb["idx"])
+    np.testing.assert_array_equal(ra["score"], rb["score"])
+    oa, la = oracle.sparse_attn(a, ra["idx"])
+    ob, lb = oracle.sparse_attn(b, rb["idx"])
+    np.testing.assert_array_equal(oa, ob)
+    np.testing.assert_array_equal(la, lb)
+
+
+def test_positive_weight_scaling_keeps_topk():
+    wl = W.make_workload("s", seq_lens=[2000], nq=2, H_I=16, D_I=128, H=1, K=300, seed=9,
+                         with_kv=False)
+    r1 = oracle.indexer_topk(wl)
+    wl.w = (wl.w * np.float32(4.0)).astype(np.float32)      # power of two: exact rescale
+    r2 = oracle.indexer_topk(wl)
+    np.testing.assert_array_equal(r1["idx"], r2["idx"])
+    np.testing.assert_array_equal(r1["score"] * 4.0, r2["score"])
+
+
+def test_attention_output_is_convex_combination_and_dominant_logit():
+    wl = W.make_workload("c", seq_lens=[200], nq=1, H_I=4, D_I=64, H=4, K=50, seed=21)
+    r = oracle.indexer_topk(wl)
+    # identical rows -> output equals that row's latent
+    kvf = W.bf16_bits_to_f32(wl.kv.reshape(-1, W.D_QK)).reshape(wl.kv.shape)
+    kvf[:] = kvf[0, 0]
+    wl.kv = W.to_bf16_bits(kvf)
+    o, _ = oracle.sparse_attn(wl, r["idx"])
+    np.testing.assert_allclose(o[0], np.broadcast_to(kvf[0, 0, :512], o[0].shape), atol=1e-12)
+    # one dominant logit -> output is (almost exactly) that row
+    wl2 = W.make_workload("c", seq_lens=[200], nq=1, H_I=4, D_I=64, H=4, K=50, seed=21)
+    idx = r["idx"]
+    target = int(idx[0, 7])
+    kvf = W.bf16_bits_to_f32(wl2.kv.reshape(-1, W.D_QK)).copy()
+    row = int(wl2.block_table[0, target // W.BLOCK]) * W.BLOCK + target % W.BLOCK
+    qf = W.bf16_bits_to_f32(wl2.q[0])
+    kvf[row, 512:] = 0.0
+    kvf[row, 512] = 256.0
+    qf = qf.copy()
+    qf[:, 512] = 64.0
+    wl2.kv = W.to_bf16_bits(kvf).reshape(wl2.kv.shape)
+    wl2.q = W.to_bf16_bits(qf)[None]
+    o2, _ = oracle.sparse_attn(wl2, idx)
+    np.testing.assert_allclose(o2[0], np.broadcast_to(kvf[row, :512], o2[0].shape), atol=1e-9)
+
+
+def test_integer_inputs_scores_are_exact():
+    wl = W.preset("tiny", with_kv=False)
+    r = oracle.indexer_topk(wl, want_all_scores=True)
+    qi = W.bf16_bits_to_f32(wl.q_idx[0]).astype(np.int64)             # [8, 64]
+    pos = np.arange(wl.seq_lens[0])
+    rows = wl.block_table[0, pos // W.BLOCK].astype(np.int64) * W.BLOCK + pos % W.BLOCK
+    ki = W.bf16_bits_to_f32(wl.k_idx.reshape(-1, wl.D_I)[rows]).astype(np.int64)
+    dots = np.maximum(ki @ qi.T, 0)                                   # exact integers
+    w256 = np.round(wl.w[0].astype(np.float64) * 256).astype(np.int64)
+    assert np.all(w256.astype(np.float64) / 256 == wl.w[0])
+    exact = (dots * w256[None, :]).sum(axis=1)                        # score * 256, exact
+    np.testing.assert_array_equal(r["all"][0] * 256.0, exact.astype(np.float64))
+
+
+def test_tie_heavy_integer_workload_breaks_ties_by_position():
+    # unit head weights: scores are small integers, so the K-th score is shared by many
+    # positions and the lower-position rule decides the boundary
+    wl = W.make_workload("ties", seq_lens=[3000], nq=1, H_I=8, D_I=64, H=1, K=256,
+                         int_inputs=True, w_dist="ones", seed=1, with_kv=False)
+    r = oracle.indexer_topk(wl, want_all_scores=True)
+    s = r["all"][0]
+    kth = r["kth"][0]
+    tied = np.nonzero(s == kth)[0]
+    above = np.nonzero(s > kth)[0]
+    assert len(tied) > 1 and len(above) < wl.K < len(above) + len(tied)
+    want = np.sort(np.concatenate([above, tied[:wl.K - len(above)]]))
+    np.testing.assert_array_equal(r["idx"][0], want)
+
+
+@pytest.mark.slow
+def test_million_token_planted_set_is_the_topk():
+    wl = W.preset("1m", with_kv=False)
+    r = oracle.indexer_topk(wl)
+    np.testing.assert_array_equal(r["idx"][0], wl.planted.astype(np.int32))

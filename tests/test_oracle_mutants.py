@@ -1,0 +1,59 @@
+"""Plant plausible mistakes in a COPY of the oracle source and check that the
+pins of test_oracle.py catch every one of them (the oracle itself is never
+edited; each mutant is compiled into a temporary library)."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "dsa_oracle.c")
+
+# (name, text in the oracle, mistaken replacement)
+MUTANTS = [
+    ("no_relu_gate", "double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;"),
+    ("tie_break_reversed", "return (a->pos > b->pos) - (a->pos < b->pos);",
+     "return (a->pos < b->pos) - (a->pos > b->pos);"),
+    ("head_weight_transposed", "acc += (double)a->w[(int64_t)t * H + h] * relu;",
+     "acc += (double)a->w[(int64_t)t * H + (H - 1 - h)] * relu;"),
+    ("scale_group_swapped", "double sc = (double)a->k_scale[row * (a->D_I / 64) + d / 64];",
+     "double sc = (double)a->k_scale[row * (a->D_I / 64) + (a->D_I / 64 - 1 - d / 64)];"),
+    ("key_without_rope", "for (int d = 0; d < ORACLE_DQK; d++) dot += bf16_to_f64(qg[d])",
+     "for (int d = 0; d < ORACLE_DV; d++) dot += bf16_to_f64(qg[d])"),
+    ("lse_without_log", "out_lse[(int64_t)i * a->H + g] = m + log(den);",
+     "out_lse[(int64_t)i * a->H + g] = m + den;"),
+    ("causal_off_by_one", "for (int64_t s = 0; s <= pos; s++) {", "for (int64_t s = 0; s < pos; s++) {"),
+    ("pad_with_zero", "out_idx[o] = j < nk ? (int32_t)keep[j] : -1;",
+     "out_idx[o] = j < nk ? (int32_t)keep[j] : 0;"),
+    ("e4m3_bias_8", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("softmax_value_from_rope", "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d]);",
+     "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d + 64]);"),
+]
+
+PINS = [pins.test_hand_indexer_relu_gate_weights_and_tie, pins.test_hand_fp8_scale_groups,
+        pins.test_hand_softmax_two_rows, pins.test_e4m3_decode_all_codes_vs_torch,
+        pins.test_single_head_unit_weight_is_relu_dot_lexsort,
+        pins.test_k_at_least_context_equals_dense_causal_attention]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mutant_c = tmp_path / "mutant.c"
+    mutant_c.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O1", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
+                           "-o", str(so), str(mutant_c), "-lm"])
+    caught = []
+    with oracle.swapped_library(str(so)):
+        for pin in PINS:
+            try:
+                pin()
+            except AssertionError:
+                caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
