@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Decode-step throughput of the DSA sparse-attention step on B200.
+
+One step = the whole hot path on one batch: fused Lightning Indexer + Top-K
+over every cached position, then Sparse Flash Attention over the selected
+rows of the MLA latent cache.  The default workload is the 32-sequence
+batched decode at 32K context (64 indexer heads x 128, bf16 keys, K = 2048,
+128 MLA heads x (512 + 64)), with caches resident in HBM.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Under torchrun each rank runs its own replica of the batch (weak scaling, no
+data-path collective); the step time is the maximum over ranks.  Prints one
+JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/sec (indexer+TopK+SFA) at 32K ctx; achieved HBM GB/s vs 8 TB/s"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="batch32", choices=["batch32", "tiny", "prefill16k", "ragged", "1m"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "indexer_top_sparse_lightning_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
+    if absent or taken on different kernel sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        d = json.load(open(p))
+        e = d[kernel]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def describe(wl):
+    return (f"{wl.name}: B={wl.B}, tokens={wl.T}, ctx max {int(wl.seq_lens.max())}, indexer {wl.H_I}x{wl.D_I} "
+            f"{wl.key_dtype} keys, K={wl.K}, MLA {wl.H} heads x (512+64) bf16, page 64, "
+            f"{'permuted' if wl.name != 'prefill16k' else 'contiguous'} block tables")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        win = [p for (t, p) in self.samples if t0 <= t <= t1]
+        if not win:
+            return None
+        sm = [float(p[0]) for p in win if p[0].replace(".", "").isdigit()]
+        mx = [float(p[1]) for p in win if p[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for p in win for n, v in zip(names, p[4:8]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(win)}
+
+
+def cpu_baseline(wl, tokens):
+    import numpy as np
+    import oracle
+    tokens = np.asarray(tokens)
+    t0 = time.perf_counter()
+    r = oracle.indexer_topk(wl, tokens)
+    idx = np.full((wl.T, wl.K), -1, dtype=np.int32)
+    idx[tokens] = r["idx"]
+    oracle.sparse_attn(wl, idx, tokens)
+    dt = time.perf_counter() - t0
+    return len(tokens) / dt, dt
+
+
+def run_reference(args, rank):
+    """The oracle timed on the host cores: each step = a bounded sample of the workload."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from indexer_top_sparse_lightning_b200 import workloads as W
+    wl = W.preset(args.workload)
+    n = min(8, wl.T)
+    sample = np.linspace(0, wl.T - 1, n).astype(np.int64)
+    for _ in range(args.warmup):
+        cpu_baseline(wl, sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cpu_baseline(wl, sample)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    cores = oracle.num_threads()
+    samp = f"{n} of the {wl.T} query tokens per step (indexer over all visible positions, full sort, attention)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": describe(wl), "global_batch": wl.T, "seq_len": int(wl.seq_lens.max()),
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": samp},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import indexer_top_sparse_lightning_b200 as dsa
+    from indexer_top_sparse_lightning_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dsa.load_library()
+    wl = W.preset(args.workload)
+    d = W.to_device(wl, dev)
+    batch = dsa.Batch(d["seq_lens"], d["cu_q"], d["block_table"], wl.num_blocks, int(wl.seq_lens.max()),
+                      int(wl.nq.max()))
+    ws = dsa.Workspace(dev)
+    T, K = wl.T, wl.K
+    out_idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    out = torch.empty((T, wl.H, 512), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    ev_i0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_i1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def step(i=None):
+        if i is not None:
+            ev_i0[i].record(stream)
+        dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], K, k_scale=d["k_scale"], out_idx=out_idx,
+                         want_score=False, workspace=ws)
+        if i is not None:
+            ev_i1[i].record(stream)
+        dsa.sparse_mla_attn(batch, d["q"], d["kv"], out_idx, wl.sm_scale, out=out, want_lse=False, workspace=ws)
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    t_warm = time.time()
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if dsa.get_status(ws) != 0:
+        raise RuntimeError("device reported an error during warm-up")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t_start = time.time()
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_end = time.time()
+    if world > 1:
+        dist.barrier()
+    ms_total = e0.elapsed_time(e1)
+    idx_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev_i0, ev_i1))
+    # keep the GPU busy long enough for the clock sampler if the timed region was short
+    soak_end = t_end
+    if t_end - t_start < 1.0:
+        while time.time() - t_start < 1.2:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+        soak_end = time.time()
+    status = dsa.get_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    t = torch.tensor([ms_total, idx_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, idx_ms = float(t[0]), float(t[1])
+    ms_step = ms_total / args.steps
+
+    # ------------------------------------------------------------ end to end through the public API
+    pin = lambda x: x.cpu().pin_memory()
+    host_in = {k: pin(d[k]) for k in ("q_idx", "w", "q", "seq_lens", "cu_q", "block_table")}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    host_idx = torch.empty(out_idx.shape, dtype=out_idx.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * host_out.element_size() + host_idx.numel() * host_idx.element_size()
+
+    def e2e_step():
+        for k, v in host_in.items():
+            d[k].copy_(v, non_blocking=True)
+        dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], K, wl.sm_scale,
+                       k_scale=d["k_scale"], out_idx=out_idx, out=out, workspace=ws)
+        host_out.copy_(out, non_blocking=True)
+        host_idx.copy_(out_idx, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t[0]) / args.e2e_steps
+    sampler.stop()
+
+    launches = dsa.decode_launch_count(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], K, wl.sm_scale,
+                                       k_scale=d["k_scale"])
+    if rank != 0:
+        return
+    key_bytes = wl.key_bytes()
+    kv_bytes = wl.kv_bytes()
+    step_bytes = key_bytes + kv_bytes
+    peak, peak_kind = peaks()
+    idx_gbs = key_bytes / (idx_ms * 1e-3) / 1e9
+    step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
+    tokens_total = T * world
+    clocks = sampler.summary(t_start, t_end) or sampler.summary(t_warm, soak_end)
+    window = "timed region" if sampler.summary(t_start, t_end) else "warm-up + timed + soak of the same step"
+    line = {
+        "metric": METRIC, "value": tokens_total / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(wl), "global_batch": tokens_total, "seq_len": int(wl.seq_lens.max()),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: {step_bytes / 1e6:.1f} MB read per step vs "
+                         f"{L2_BYTES / 1e6:.0f} MB L2, no flush"},
+        "hbm": {"bytes_per_step": step_bytes, "indexer_key_bytes": key_bytes, "gathered_kv_bytes": kv_bytes,
+                "step_gbs": step_gbs, "frac_of_8tbs": step_gbs / SPEC_HBM_GBS,
+                "frac_of_measured": step_gbs / peak},
+        "roofline": {"kernel": "indexer_topk_kernel", "bound": "hbm", "achieved": idx_gbs, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": idx_gbs / peak,
+                     "traffic": ncu_traffic("indexer_topk_kernel"), "ms_per_launch": idx_ms,
+                     "algorithmic_bytes_per_launch": key_bytes},
+        "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches * args.steps,
+        "clocks": dict(clocks or {}, window=window),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        value, dt = cpu_baseline(wl, np.arange(wl.T) if wl.T <= 64 else np.linspace(0, wl.T - 1, 32).astype(np.int64))
+        n = wl.T if wl.T <= 64 else 32
+        line["cpu_baseline"] = {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"{n} query tokens ({'one full step' if n == wl.T else 'evenly spaced'}), "
+                                          f"{dt:.1f} s: scores over every visible position, full sort, attention"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

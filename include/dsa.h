@@ -1,0 +1,184 @@
+/*
+ * dsa.h -- C ABI of the DSA sparse-attention step for NVIDIA B200 (sm_100a).
+ *
+ * The step has two parts, as the pages describe it:
+ *
+ *  1. Index stage ("Day0 Adaptation and Performance Optimization for Novel
+ *     Long-Sequence Reasoning Models", section 3; "Large Model Inference
+ *     Acceleration: Day-0 Adaptation and Performance Optimization for New
+ *     Architectures", section 1.1 "Indexer Fusion: Three Kernels into One"):
+ *     relevance scoring of every cached position, head-weight weighting and
+ *     Top-K selection in ONE kernel that reads the paged indexer-key cache in
+ *     place and writes only the final index list.  The score is the Lightning
+ *     Indexer form with a ReLU gate:
+ *         score(t, s) = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])
+ *     Ties are broken by position (the lower position wins).
+ *
+ *  2. Sparse read stage ("Day0 Adaptation and Sparse Attention Optimization
+ *     for Long-Sequence LLM Inference", section 4): Sparse Flash Attention
+ *     gathers only the selected rows of the MLA latent cache (512 latent +
+ *     64 RoPE, shared by all query heads) and computes softmax attention over
+ *     them: logits = sm_scale * q . row[0:576], output = softmax . row[0:512].
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers unless stated; the caller owns
+ *    every buffer (inputs, outputs and the workspace).  The library never
+ *    allocates or frees memory and never synchronizes the stream, except
+ *    dsa_get_status(), which synchronizes by design.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t, passed as
+ *    void*; NULL = legacy default stream).  Pointers must stay valid until
+ *    that work completes.
+ *  - Host-side validation failures return before anything is launched.
+ *    Launch failures return DSA_ERR_CUDA.  Errors found by the kernels
+ *    (out-of-range block ids, a co-scheduling wait that timed out) are
+ *    recorded in a status word inside the workspace and read with
+ *    dsa_get_status().
+ *  - Layouts are dense, row-major, with the innermost dimension last.
+ *    Query tokens are sequence-major: tokens cu_q[b] .. cu_q[b+1]-1 belong to
+ *    sequence b and sit at positions seq_lens[b]-nq_b .. seq_lens[b]-1; token
+ *    j of a sequence sees positions 0..its own position (causal).
+ *  - Paged caches: page size 64 tokens.  block_table[b, i] is the physical
+ *    page holding positions 64*i .. 64*i+63 of sequence b.  The indexer-key
+ *    cache and the latent cache share the table.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,    /* a pointer, size or shape failed validation       */
+    DSA_ERR_UNSUPPORTED = 2,    /* valid request outside what the kernels implement */
+    DSA_ERR_WORKSPACE = 3,      /* workspace NULL, too small or misaligned          */
+    DSA_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed              */
+    DSA_ERR_TIMEOUT = 5,        /* device: a bounded wait expired (kernel returned) */
+    DSA_ERR_DEVICE_BOUNDS = 6,  /* device: block id or index out of range (skipped) */
+    DSA_ERR_CAPACITY = 7        /* device: a key chunk exceeded on-chip capacity    */
+} dsa_status;
+
+typedef enum {
+    DSA_KEY_BF16 = 0,           /* indexer keys: bf16 [num_blocks, 64, D_I]                       */
+    DSA_KEY_FP8_E4M3 = 1        /* indexer keys: e4m3fn codes [num_blocks, 64, D_I] (uint8) plus  */
+                                /* fp32 scales [num_blocks, 64, D_I/64], one per 64 elements      */
+} dsa_key_dtype;
+
+/* Batch and paging description shared by all entry points. */
+typedef struct {
+    int32_t batch;              /* B sequences                                            */
+    int32_t num_tokens;         /* T query tokens in total                                */
+    const int32_t* seq_lens;    /* device [B]: cached length INCLUDING this step's tokens */
+    const int32_t* cu_q;        /* device [B+1]: query-token offsets, cu_q[0] = 0         */
+    const int32_t* block_table; /* device [B, max_blocks_per_seq]                         */
+    int32_t max_blocks_per_seq;
+    int32_t num_blocks;         /* physical pages in each cache (bounds checks)           */
+    int32_t max_seq_len;        /* host-side upper bound on every seq_lens[b]             */
+    int32_t max_q_per_seq;      /* host-side upper bound on cu_q[b+1] - cu_q[b]           */
+} dsa_batch;
+
+/* Indexer inputs (Lightning Indexer + Top-K). */
+typedef struct {
+    const void* q_idx;          /* device [T, H_I, D_I] bf16                                   */
+    const float* w;             /* device [T, H_I] fp32 head weights (any sign)                */
+    const void* k_cache;        /* device indexer-key cache, layout per key_dtype              */
+    const float* k_scale;       /* device [num_blocks, 64, D_I/64] (fp8 keys), NULL for bf16   */
+    int32_t key_dtype;          /* dsa_key_dtype                                               */
+    int32_t H_I;                /* indexer heads: 8, 16, 32 or 64                              */
+    int32_t D_I;                /* indexer dim: 64 or 128                                      */
+    int32_t K;                  /* Top-K, 1..2048                                              */
+} dsa_indexer_inputs;
+
+/* Sparse MLA attention inputs. */
+typedef struct {
+    const void* q;              /* device [T, H, 576] bf16 (512 latent + 64 RoPE)   */
+    const void* kv_cache;       /* device [num_blocks, 64, 576] bf16                */
+    int32_t H;                  /* query heads, 1..128                              */
+    float sm_scale;             /* softmax scale applied to q . row[0:576]          */
+} dsa_attn_inputs;
+
+/*
+ * Bytes of workspace needed by indexer_topk, sparse_mla_attn and dsa_decode
+ * for this batch shape (the maximum of the three; dsa_decode additionally
+ * needs nothing else).  The workspace must be 256-byte aligned and
+ * ZERO-FILLED before its first use; every call that completes without a
+ * device error leaves it zero-filled again, so it can be reused by later
+ * calls on the same stream.  After a device error (dsa_get_status != OK)
+ * zero-fill it again.  Calls sharing one workspace must not overlap in time.
+ * Returns 0 if the shape is invalid.
+ */
+DSA_API size_t dsa_workspace_size(const dsa_batch* batch, const dsa_indexer_inputs* ix,
+                          const dsa_attn_inputs* at);
+
+/*
+ * Fused Lightning Indexer + Top-K.
+ * out_idx   device [T, K] int32: the selected positions of each token in
+ *           ascending order, -1 padded when fewer than K positions are
+ *           visible (then every visible position is selected).
+ * out_score device [T, K] fp32 score of each selected position (-inf on
+ *           padding) or NULL.
+ * Score rows are never written to global memory.
+ */
+DSA_API dsa_status indexer_topk(const dsa_batch* batch, const dsa_indexer_inputs* ix,
+                        int32_t* out_idx, float* out_score,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Sparse Flash Attention over the rows listed in idx (device [T, K] int32
+ * logical positions; negative entries are skipped).
+ * out device [T, H, 512] bf16; lse device [T, H] fp32 natural-log
+ * log-sum-exp of the scaled logits (-inf if a token selects nothing) or NULL.
+ */
+DSA_API dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs* at,
+                           const int32_t* idx, int32_t K,
+                           void* out, float* lse,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The whole decode step: indexer_topk then sparse_mla_attn on one stream,
+ * without a host synchronization in between.  out_idx [T, K] is required
+ * (it carries the index list between the stages); out_score and lse may be
+ * NULL.
+ */
+DSA_API dsa_status dsa_decode(const dsa_batch* batch, const dsa_indexer_inputs* ix,
+                      const dsa_attn_inputs* at,
+                      int32_t* out_idx, float* out_score, void* out, float* lse,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronizes `stream`, reads the device status word kept in `workspace`
+ * (DSA_OK if no kernel reported an error since the last read) into
+ * *device_status and clears it.  Returns DSA_ERR_CUDA if the stream itself
+ * failed.
+ */
+DSA_API dsa_status dsa_get_status(void* workspace, void* stream, int32_t* device_status);
+
+/*
+ * Number of kernel launches dsa_decode enqueues for this shape (indexer
+ * launches + attention launches), or -1 if the shape is invalid.  Useful for
+ * sizing CUDA graphs and for launch accounting; performs no launch.
+ */
+DSA_API int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexer_inputs* ix,
+                                        const dsa_attn_inputs* at);
+
+/* Static description of a status code. */
+DSA_API const char* dsa_status_str(int32_t status);
+
+/* Library version string. */
+DSA_API const char* dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,83 @@
+// common.h -- parameter blocks and shared-memory layouts shared by the host
+// launcher (api.cu) and the kernels.  No arithmetic of the method lives here.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+namespace dsa {
+
+constexpr int kPage = 64;             // tokens per cache page
+constexpr int kTileKeys = 128;        // keys per indexer MMA tile (two pages)
+constexpr int kMaxTopK = 2048;
+constexpr int kDqk = 576;             // latent 512 + RoPE 64
+constexpr int kDv = 512;
+constexpr int kEpiThreads = 128;      // four epilogue warps, one TMEM lane each
+
+// Device status word values (mirrors dsa_status).
+enum : uint32_t {
+    kStOk = 0, kStTimeout = 5, kStBounds = 6, kStCapacity = 7
+};
+
+// Workspace header (first 256 bytes).
+struct WsHeader {
+    uint32_t status;
+    uint32_t pad[63];
+};
+
+// ------------------------------------------------------------------ indexer
+// Work decomposition:
+//  mode 0 (decode): one group per sequence of the launch range [b_begin,
+//    b_end); each group gets g_b CTAs, each CTA scores a contiguous chunk of
+//    key tiles, and the group agrees on its Top-K through global histograms.
+//  mode 1 (independent): every query token is its own group with one CTA;
+//    CTAs loop over tokens in zig-zag order (head-tail pairing).
+struct IndexerParams {
+    const int32_t* seq_lens;
+    const int32_t* cu_q;
+    const int32_t* block_table;
+    const float* w;
+    const float* k_scale;
+    int32_t* out_idx;
+    float* out_score;
+    uint32_t* status;
+    uint8_t* group_ws;        // mode 0: per-group sync + histograms + counts
+    int64_t group_ws_stride;  // bytes per group
+    int32_t B, T, max_blocks, num_blocks;
+    int32_t b_begin, b_end;   // mode 0 launch range
+    int32_t t_begin, t_end;   // mode 1 token range
+    int32_t mode;
+    int32_t K;
+    int32_t score_cap;        // fp32 score slots per CTA (all tokens of a group)
+};
+
+// Group workspace layout (mode 0), per group:
+//   [0,128)   sync {count, gen}
+//   hist[3][NQ][2048] u32
+//   cnt[max_ctas][NQ][2] u32
+__host__ __device__ constexpr int64_t group_ws_bytes(int nq, int max_ctas) {
+    return 128 + 3LL * nq * 2048 * 4 + (int64_t)max_ctas * nq * 2 * 4;
+}
+
+template <int DI, bool FP8>
+struct KeyTileBytes {
+    static constexpr int value = kTileKeys * DI * (FP8 ? 1 : 2);
+};
+
+// ------------------------------------------------------------------ sparse attention
+struct SfaParams {
+    const int32_t* seq_lens;
+    const int32_t* cu_q;
+    const int32_t* block_table;
+    const uint16_t* kv;       // [num_blocks*64, 576] bf16 bits
+    const int32_t* idx;       // [T, K]
+    uint16_t* out;            // [T, H, 512] bf16 bits
+    float* lse;               // [T, H] or null
+    float* part_o;            // split partials: [T, S, 128 chunks of 4 dims, 128 heads, 4]
+    float* part_ml;           // [T, S, 2, 128] (m in log2 domain, l)
+    uint32_t* status;
+    int32_t B, T, H, K, max_blocks, num_blocks;
+    int32_t n_splits, rows_per_split;
+    float scale_log2;         // sm_scale * log2(e)
+};
+
+}  // namespace dsa

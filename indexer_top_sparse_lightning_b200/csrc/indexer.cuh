@@ -1,0 +1,796 @@
+// indexer.cuh -- fused Lightning Indexer + Top-K kernel for sm_100a.
+//
+// One kernel performs the whole index stage the pages describe as a single
+// fused operator ("Large Model Inference Acceleration: Day-0 Adaptation and
+// Performance Optimization for New Architectures", section 1.1 "Indexer
+// Fusion: Three Kernels into One"; "Day0 Adaptation and Sparse Attention
+// Optimization for Long-Sequence LLM Inference", section 4): it reads the
+// paged indexer-key cache in place, scores every visible position, applies
+// the head weights, selects the Top-K and writes only the index list.
+//
+//   score(t, s) = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])
+//
+// Roles inside a CTA (warp specialised, mbarrier pipelines):
+//   warps 0-3  epilogue: TMEM -> registers, ReLU, head-weighted sum in fp32,
+//              scores into shared memory, then the radix Top-K select
+//   warp 4     TMA producer: walks the block table, loads 128-key tiles
+//              (two 64-token pages) with cp.async.bulk.tensor into a
+//              128-byte-swizzled ring of shared-memory stages
+//   warp 5     TMEM allocator and tcgen05.mma issuer:
+//              D[key, (token,head)] = K_tile[128 x D_I] . Q^T, fp32 in TMEM,
+//              double-buffered so the epilogue of tile i overlaps the MMA of
+//              tile i+1
+//   warps 6-9  (fp8 keys only) widen e4m3 codes to bf16 in shared memory;
+//              the per-64-element scales are applied in the fp32 epilogue
+//
+// Top-K: scores never leave shared memory.  A CTA, or a group of CTAs that
+// share one sequence, finds the exact K-th largest order-preserving key with
+// three radix passes (11/11/10 bits); the CTAs of a group add their
+// histograms into a small global histogram and meet at a bounded group
+// barrier.  Elements above the threshold are taken; elements equal to it are
+// taken lowest position first.  Indices are emitted in ascending position
+// order with warp ballots and prefix counts (no atomics on the output).
+#pragma once
+#include "common.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+__host__ __device__ constexpr int pow2_at_least(int v) {
+    int p = 32;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+template <bool FP8, int HI, int DI, int NQ>
+struct IdxCfg {
+    static constexpr int KB = DI / 64;                        // 64-wide K blocks
+    static constexpr int N = (NQ * HI < 16) ? 16 : NQ * HI;   // MMA N (token-major heads)
+    static constexpr int ACC = FP8 ? KB : 1;                  // fp8: one accumulator per scale group
+    static constexpr int COLS_BUF = N * ACC;
+    static constexpr int TMEM_COLS = pow2_at_least(2 * COLS_BUF);
+    static constexpr int NSTAGE = FP8 ? 4 : (NQ == 1 ? 4 : 3);
+    static constexpr int STAGE_BYTES = kTileKeys * DI * (FP8 ? 1 : 2);
+    static constexpr int NCONV = FP8 ? 2 : 0;                 // widened-operand buffers
+    static constexpr int NCV = FP8 ? 2 : 1;                   // (modulus for the ring index)
+    static constexpr int CONV_BYTES = kTileKeys * DI * 2;
+    static constexpr int Q_BYTES = N * DI * 2;
+    static constexpr int Q_TX = NQ * HI * DI * 2;             // bytes one Q load brings in
+    static constexpr bool Q_PAD = NQ * HI < N;                // rows [NQ*HI, N) stay zero
+    static constexpr int HIST_WORDS = NQ * 2048;
+    static constexpr int W_FLOATS = NQ * HI;
+    static constexpr int THREADS = FP8 ? 320 : 192;
+    static constexpr int PRODUCER_WARP = 4;
+    static constexpr int MMA_WARP = 5;
+    static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, false, false);
+
+    static constexpr int OFF_STAGE = 0;
+    static constexpr int OFF_CONV = OFF_STAGE + NSTAGE * STAGE_BYTES;
+    static constexpr int OFF_Q = OFF_CONV + NCONV * CONV_BYTES;
+    static constexpr int OFF_HIST = OFF_Q + Q_BYTES;
+    static constexpr int OFF_W = OFF_HIST + HIST_WORDS * 4;
+    static constexpr int OFF_MISC = OFF_W + ((W_FLOATS * 4 + 127) / 128) * 128;
+    static constexpr int MISC_BYTES = 1024;
+    static constexpr int OFF_SCORE = OFF_MISC + MISC_BYTES;
+    // dynamic shared memory = 1024 (alignment slack) + OFF_SCORE + score_cap * 4
+    static constexpr int FIXED_SMEM = 1024 + OFF_SCORE;
+};
+
+struct IdxMisc {
+    uint64_t full[8];
+    uint64_t empty[8];
+    uint64_t conv_full[2];
+    uint64_t conv_empty[2];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t q_full;
+    uint64_t q_empty;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    // mode-0 assignment of this CTA
+    int g_valid, g_b, g_rank, g_size, g_tile_begin, g_tile_count, g_group;
+    uint32_t scan[8];
+    uint32_t wcnt[4][4][2];   // [token][warp][gt, eq]
+    uint32_t wallow[4][4];    // [token][warp] tied elements the warp may take
+    uint32_t sel_bin[4];
+    uint32_t sel_kk[4];
+    uint32_t sel_take[4];
+    uint32_t sel_base[4];
+};
+
+// One unit of work: a group of query tokens of one sequence and a chunk of
+// its key tiles.
+struct IdxItem {
+    int b, t0, nq, rank, G, group;
+    int tile_begin, tile_count;
+    int64_t L;
+    int64_t pos[4];
+};
+
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) {
+    atomicCAS(status, 0u, code);
+}
+
+template <int NQ>
+__device__ __forceinline__ bool get_item(const IndexerParams& p, const IdxMisc* m, int k, IdxItem& it) {
+    if (p.mode == 0) {
+        if (k != 0 || !m->g_valid) return false;
+        it.b = m->g_b;
+        it.rank = m->g_rank;
+        it.G = m->g_size;
+        it.group = m->g_group;
+        it.tile_begin = m->g_tile_begin;
+        it.tile_count = m->g_tile_count;
+        it.t0 = __ldg(p.cu_q + it.b);
+        it.nq = __ldg(p.cu_q + it.b + 1) - it.t0;
+        it.L = __ldg(p.seq_lens + it.b);
+        for (int j = 0; j < NQ; ++j) it.pos[j] = it.L - it.nq + j;
+        return true;
+    }
+    // mode 1: zig-zag over tokens -- even rounds ascend, odd rounds descend
+    const int C = gridDim.x;
+    const int local = (k & 1) ? (k * C + (C - 1 - (int)blockIdx.x)) : (k * C + (int)blockIdx.x);
+    const int t = p.t_begin + local;
+    if (local < 0 || t >= p.t_end) return false;
+    // sequence of token t
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (__ldg(p.cu_q + mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    it.b = lo;
+    it.t0 = t;
+    it.nq = 1;
+    it.rank = 0;
+    it.G = 1;
+    it.group = 0;
+    it.L = __ldg(p.seq_lens + lo);
+    const int nqb = __ldg(p.cu_q + lo + 1) - __ldg(p.cu_q + lo);
+    it.pos[0] = it.L - nqb + (t - __ldg(p.cu_q + lo));
+    if (it.L > (int64_t)p.max_blocks * kPage || it.pos[0] < 0 || it.pos[0] >= p.score_cap) {
+        // inconsistent lengths: report and give this token an empty key range
+        set_status(p.status, kStBounds);
+        it.L = 0;
+        it.pos[0] = -1;
+    }
+    for (int j = 1; j < NQ; ++j) it.pos[j] = -1;
+    it.tile_begin = 0;
+    it.tile_count = (int)((it.pos[0] + kTileKeys) / kTileKeys);
+    return true;
+}
+
+// Mode-0 partition: every CTA computes the same split of CTAs over the
+// sequences [b_begin, b_end), proportional to their key tiles.
+__device__ void assign_groups(const IndexerParams& p, IdxMisc* m, int nq_max, int score_cap) {
+    const int Bp = p.b_end - p.b_begin;
+    const int C = gridDim.x;
+    int64_t total = 0;
+    for (int b = p.b_begin; b < p.b_end; ++b) total += (__ldg(p.seq_lens + b) + kTileKeys - 1) / kTileKeys;
+    m->g_valid = 0;
+    if (total <= 0 || C < Bp) return;
+    int acc = 0;
+    for (int b = p.b_begin; b < p.b_end; ++b) {
+        const int64_t L = __ldg(p.seq_lens + b);
+        const int tiles = (int)((L + kTileKeys - 1) / kTileKeys);
+        int g = 1 + (int)(((int64_t)(C - Bp) * tiles) / total);
+        if (g > tiles) g = tiles;
+        if (g < 1) g = 1;
+        if ((int)blockIdx.x >= acc && (int)blockIdx.x < acc + g) {
+            const int r = (int)blockIdx.x - acc;
+            const int base = tiles / g, rem = tiles % g;
+            const int t0 = __ldg(p.cu_q + b);
+            const int nq = __ldg(p.cu_q + b + 1) - t0;
+            const int max_chunk = (base + (rem ? 1 : 0)) * kTileKeys;
+            if (nq < 1 || nq > nq_max || nq > L || t0 < 0 || t0 + nq > p.T || L > (int64_t)p.max_blocks * kPage) {
+                set_status(p.status, kStBounds);
+                return;
+            }
+            if ((int64_t)max_chunk * nq > score_cap) {
+                set_status(p.status, kStCapacity);
+                return;
+            }
+            m->g_valid = 1;
+            m->g_b = b;
+            m->g_rank = r;
+            m->g_size = g;
+            m->g_group = b - p.b_begin;
+            m->g_tile_begin = r * base + (r < rem ? r : rem);
+            m->g_tile_count = base + (r < rem ? 1 : 0);
+            return;
+        }
+        acc += g;
+    }
+}
+
+// Bounded barrier among the CTAs of one group (called by the 128 epilogue
+// threads).  Sense-reversing: the last arriver resets the count and bumps
+// the generation.
+__device__ bool group_sync(uint32_t* sync, int G, uint32_t* status, volatile int* abort) {
+    named_bar_sync(1, kEpiThreads);
+    if (threadIdx.x == 0 && !*abort) {
+        uint32_t* count = sync;
+        uint32_t* gen = sync + 1;
+        const uint32_t g0 = ld_acquire_gpu(gen);
+        const uint32_t old = atom_add_acq_rel_gpu(count, 1u);
+        if (old == (uint32_t)G - 1u) {
+            *reinterpret_cast<volatile uint32_t*>(count) = 0u;
+            st_release_gpu(gen, g0 + 1u);
+        } else {
+            const uint64_t t0 = globaltimer();
+            while (ld_acquire_gpu(gen) == g0) {
+                if (globaltimer() - t0 > kWaitTimeoutNs) {
+                    set_status(status, kStTimeout);
+                    *abort = 1;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+    }
+    named_bar_sync(1, kEpiThreads);
+    return !*abort;
+}
+
+// Exclusive prefix over the 128 epilogue threads; *total receives the sum.
+__device__ __forceinline__ uint32_t epi_exclusive_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    named_bar_sync(1, kEpiThreads);
+    uint32_t before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t s = scratch[w];
+        if (w < warp) before += s;
+        all += s;
+    }
+    named_bar_sync(1, kEpiThreads);
+    *total = all;
+    return before + x - v;
+}
+
+// Radix step: given the histogram of the current digit (nb bins, highest bin
+// first is most significant), find the bin holding the kk-th largest element.
+__device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t kk, uint32_t* scratch,
+                                         uint32_t* out_bin, uint32_t* out_kk) {
+    const int per = nb / kEpiThreads;
+    const int t = threadIdx.x;
+    const int hi_bin = nb - 1 - t * per;
+    uint32_t s = 0;
+    for (int i = 0; i < per; ++i) s += hist[hi_bin - i];
+    uint32_t total;
+    const uint32_t before = epi_exclusive_scan(s, scratch, &total);
+    if (before < kk && kk <= before + s) {
+        uint32_t c = before;
+        for (int i = 0; i < per; ++i) {
+            const uint32_t h = hist[hi_bin - i];
+            if (c + h >= kk) {
+                *out_bin = (uint32_t)(hi_bin - i);
+                *out_kk = kk - c;
+                break;
+            }
+            c += h;
+        }
+    }
+    named_bar_sync(1, kEpiThreads);
+}
+
+template <bool FP8, int HI, int DI, int NQ>
+__global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
+    indexer_topk_kernel(const __grid_constant__ IndexerParams p, const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k) {
+    using Cfg = IdxCfg<FP8, HI, DI, NQ>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* s_stage = smem + Cfg::OFF_STAGE;
+    uint8_t* s_conv = smem + Cfg::OFF_CONV;
+    uint8_t* s_q = smem + Cfg::OFF_Q;
+    uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_HIST);
+    float* s_w = reinterpret_cast<float*>(smem + Cfg::OFF_W);
+    IdxMisc* m = reinterpret_cast<IdxMisc*>(smem + Cfg::OFF_MISC);
+    float* s_score = reinterpret_cast<float*>(smem + Cfg::OFF_SCORE);
+    volatile int* abort = &m->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < Cfg::NSTAGE; ++i) {
+            mbar_init(&m->full[i], 1);
+            mbar_init(&m->empty[i], FP8 ? kEpiThreads : 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&m->conv_full[i], kEpiThreads);
+            mbar_init(&m->conv_empty[i], 1);
+            mbar_init(&m->tfull[i], 1);
+            mbar_init(&m->tempty[i], kEpiThreads);
+        }
+        mbar_init(&m->q_full, 1);
+        mbar_init(&m->q_empty, 1);
+        mbar_init(&m->drain, 1);
+        m->abort = 0;
+        fence_mbar_init();
+        if (p.mode == 0) assign_groups(p, m, NQ, p.score_cap);
+    }
+    if (warp == Cfg::MMA_WARP) {
+        tmem_alloc(&m->tmem_base, Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == Cfg::PRODUCER_WARP && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+    }
+    if (Cfg::Q_PAD) {
+        // MMA rows beyond the real heads read zeros (the Q loads never touch them)
+        for (int i = threadIdx.x; i < Cfg::Q_BYTES / 16; i += blockDim.x)
+            reinterpret_cast<uint4*>(s_q)[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = m->tmem_base;
+
+    if (warp == Cfg::PRODUCER_WARP) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            uint32_t it = 0;
+            IdxItem item;
+            for (int k = 0; get_item<NQ>(p, m, k, item); ++k) {
+                if (!mbar_wait(&m->q_empty, (k & 1) ^ 1, abort)) break;
+                mbar_arrive_expect_tx(&m->q_full, Cfg::Q_TX);
+                for (int kb = 0; kb < Cfg::KB; ++kb)
+                    tma_load_3d(s_q + kb * Cfg::N * 128, &tm_q, &m->q_full, kb * 64, 0, item.t0);
+                const int64_t npages = (item.L + kPage - 1) / kPage;
+                bool ok = true;
+                for (int li = 0; li < item.tile_count; ++li, ++it) {
+                    const int s = it % Cfg::NSTAGE;
+                    if (!mbar_wait(&m->empty[s], ((it / Cfg::NSTAGE) & 1) ^ 1, abort)) { ok = false; break; }
+                    const int tile = item.tile_begin + li;
+                    int blk[2];
+                    int nvalid = 0;
+                    for (int pp = 0; pp < 2; ++pp) {
+                        const int64_t pg = (int64_t)tile * 2 + pp;
+                        blk[pp] = -2;
+                        if (pg < npages) {
+                            int bid = __ldg(p.block_table + (int64_t)item.b * p.max_blocks + pg);
+                            if (bid < 0 || bid >= p.num_blocks) {
+                                set_status(p.status, kStBounds);
+                                bid = -1;   // out-of-range coordinate: TMA fills zeros
+                            }
+                            blk[pp] = bid;
+                            ++nvalid;
+                        }
+                    }
+                    uint8_t* st = s_stage + s * Cfg::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&m->full[s], nvalid * kPage * DI * (FP8 ? 1 : 2));
+                    for (int pp = 0; pp < 2; ++pp) {
+                        if (blk[pp] == -2) continue;
+                        if (FP8) {
+                            tma_load_2d_hint(st + pp * kPage * DI, &tm_k, &m->full[s], 0, blk[pp] * kPage, pol);
+                        } else {
+                            for (int kb = 0; kb < Cfg::KB; ++kb)
+                                tma_load_2d_hint(st + kb * (kTileKeys * 128) + pp * (kPage * 128), &tm_k,
+                                                 &m->full[s], kb * 64, blk[pp] * kPage, pol);
+                        }
+                    }
+                }
+                if (!ok) break;
+            }
+            // drain: no TMA write may still be in flight when the CTA exits
+            const uint32_t first = it > (uint32_t)Cfg::NSTAGE ? it - Cfg::NSTAGE : 0u;
+            volatile int no_abort = 0;
+            for (uint32_t d = first; d < it; ++d)
+                mbar_wait(&m->full[d % Cfg::NSTAGE], (d / Cfg::NSTAGE) & 1, &no_abort);
+        }
+    } else if (warp == Cfg::MMA_WARP) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0;
+            IdxItem item;
+            bool ok = true;
+            for (int k = 0; ok && get_item<NQ>(p, m, k, item); ++k) {
+                if (!mbar_wait(&m->q_full, k & 1, abort)) break;
+                tc_fence_after();
+                for (int li = 0; li < item.tile_count; ++li, ++it) {
+                    const int buf = it & 1;
+                    const uint8_t* a_base;
+                    if (FP8) {
+                        const int cb = it % Cfg::NCV;
+                        if (!mbar_wait(&m->conv_full[cb], (it / Cfg::NCV) & 1, abort)) { ok = false; break; }
+                        a_base = s_conv + cb * Cfg::CONV_BYTES;
+                    } else {
+                        const int s = it % Cfg::NSTAGE;
+                        if (!mbar_wait(&m->full[s], (it / Cfg::NSTAGE) & 1, abort)) { ok = false; break; }
+                        a_base = s_stage + s * Cfg::STAGE_BYTES;
+                    }
+                    if (!mbar_wait(&m->tempty[buf], ((it >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(a_base);
+                    const uint32_t b_addr = smem_u32(s_q);
+#pragma unroll
+                    for (int kb = 0; kb < Cfg::KB; ++kb) {
+#pragma unroll
+                        for (int k16 = 0; k16 < 4; ++k16) {
+                            const uint64_t ad = sdesc_sw128(a_addr + kb * (kTileKeys * 128) + k16 * 32, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(b_addr + kb * (Cfg::N * 128) + k16 * 32, 16, 1024);
+                            const uint32_t d = tmem_base + buf * Cfg::COLS_BUF + (FP8 ? kb * Cfg::N : 0);
+                            const uint32_t acc = FP8 ? (k16 > 0) : (kb > 0 || k16 > 0);
+                            umma_bf16(d, ad, bd, Cfg::IDESC, acc);
+                        }
+                    }
+                    if (FP8) umma_commit(&m->conv_empty[it % Cfg::NCV]);
+                    else umma_commit(&m->empty[it % Cfg::NSTAGE]);
+                    umma_commit(&m->tfull[buf]);
+                }
+                umma_commit(&m->q_empty);
+            }
+            // drain: every issued MMA completes before TMEM is released
+            umma_commit(&m->drain);
+            volatile int no_abort = 0;
+            mbar_wait(&m->drain, 0, &no_abort);
+        }
+    } else if (FP8 && warp >= 6) {
+        // ---------------------------------------------------------------- fp8 -> bf16 widening
+        const int ct = threadIdx.x - 192;
+        uint32_t it = 0;
+        IdxItem item;
+        bool ok = true;
+        constexpr int CH = DI / 16;   // 16-byte chunks of codes per key
+        for (int k = 0; ok && get_item<NQ>(p, m, k, item); ++k) {
+            for (int li = 0; li < item.tile_count; ++li, ++it) {
+                const int s = it % Cfg::NSTAGE;
+                const int cb = it % Cfg::NCV;
+                if (!mbar_wait(&m->full[s], (it / Cfg::NSTAGE) & 1, abort)) { ok = false; break; }
+                if (!mbar_wait(&m->conv_empty[cb], ((it / Cfg::NCV) & 1) ^ 1, abort)) { ok = false; break; }
+                const uint8_t* raw = s_stage + s * Cfg::STAGE_BYTES;
+                uint8_t* dst = s_conv + cb * Cfg::CONV_BYTES;
+#pragma unroll 4
+                for (int u = ct; u < kTileKeys * CH; u += kEpiThreads) {
+                    const int r = u / CH, c = u % CH;
+                    const uint4 v = *reinterpret_cast<const uint4*>(raw + r * DI + c * 16);
+                    uint32_t outw[8];
+                    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        uint32_t h01, h23;
+                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"((uint16_t)(in[e] & 0xFFFFu)));
+                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"((uint16_t)(in[e] >> 16)));
+                        const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+                        const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+                        const __nv_bfloat162 b01 = __float22bfloat162_rn(f01);
+                        const __nv_bfloat162 b23 = __float22bfloat162_rn(f23);
+                        outw[2 * e] = *reinterpret_cast<const uint32_t*>(&b01);
+                        outw[2 * e + 1] = *reinterpret_cast<const uint32_t*>(&b23);
+                    }
+                    const int kb = c >> 2;
+                    const int q0 = (c & 3) * 2;
+                    uint8_t* row = dst + kb * (kTileKeys * 128) + r * 128;
+                    *reinterpret_cast<uint4*>(row + ((q0 ^ (r & 7)) << 4)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+                    *reinterpret_cast<uint4*>(row + (((q0 + 1) ^ (r & 7)) << 4)) =
+                        make_uint4(outw[4], outw[5], outw[6], outw[7]);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&m->conv_full[cb]);
+                mbar_arrive(&m->empty[s]);
+            }
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- epilogue + select
+        const int row = threadIdx.x;            // TMEM lane == key row in the tile
+        uint32_t it = 0;
+        IdxItem item;
+        bool ok = true;
+        for (int k = 0; ok && get_item<NQ>(p, m, k, item); ++k) {
+            for (int i = threadIdx.x; i < NQ * HI; i += kEpiThreads) {
+                const int j = i / HI;
+                s_w[i] = (j < item.nq) ? __ldg(p.w + (int64_t)(item.t0 + j) * HI + (i % HI)) : 0.0f;
+            }
+            for (int i = threadIdx.x; i < Cfg::HIST_WORDS; i += kEpiThreads) s_hist[i] = 0u;
+            named_bar_sync(1, kEpiThreads);
+            const int stride = item.tile_count * kTileKeys;   // score slots per token
+            const int64_t chunk0 = (int64_t)item.tile_begin * kTileKeys;
+            const int64_t npages = (item.L + kPage - 1) / kPage;
+            for (int li = 0; li < item.tile_count; ++li, ++it) {
+                const int buf = it & 1;
+                const int64_t pos = chunk0 + (int64_t)li * kTileKeys + row;
+                float sc[2] = {1.0f, 1.0f};
+                if (FP8) {
+                    const int64_t pg = pos / kPage;
+                    if (pg < npages) {
+                        const int bid = __ldg(p.block_table + (int64_t)item.b * p.max_blocks + pg);
+                        if (bid >= 0 && bid < p.num_blocks) {
+                            const float* sp = p.k_scale + ((int64_t)bid * kPage + pos % kPage) * Cfg::KB;
+                            sc[0] = __ldg(sp);
+                            if (Cfg::KB > 1) sc[1] = __ldg(sp + 1);
+                        }
+                    }
+                }
+                if (!mbar_wait(&m->tfull[buf], (it >> 1) & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * Cfg::COLS_BUF;
+                float score[NQ];
+#pragma unroll
+                for (int j = 0; j < NQ; ++j) {
+                    float acc = 0.0f;
+                    if (j < item.nq) {
+                        constexpr int CW = HI < 32 ? HI : 32;
+#pragma unroll
+                        for (int c0 = 0; c0 < HI; c0 += CW) {
+                            uint32_t a0[32], a1[32];
+                            const uint32_t col = j * HI + c0;
+                            if constexpr (CW == 32) {
+                                tmem_ld32(tb + col, a0);
+                                if (FP8 && Cfg::KB > 1) tmem_ld32(tb + Cfg::N + col, a1);
+                            } else if constexpr (CW == 16) {
+                                tmem_ld16(tb + col, *reinterpret_cast<uint32_t(*)[16]>(a0));
+                                if (FP8 && Cfg::KB > 1) tmem_ld16(tb + Cfg::N + col, *reinterpret_cast<uint32_t(*)[16]>(a1));
+                            } else {
+                                tmem_ld8(tb + col, *reinterpret_cast<uint32_t(*)[8]>(a0));
+                                if (FP8 && Cfg::KB > 1) tmem_ld8(tb + Cfg::N + col, *reinterpret_cast<uint32_t(*)[8]>(a1));
+                            }
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int h = 0; h < CW; ++h) {
+                                float x = __uint_as_float(a0[h]);
+                                if (FP8) {
+                                    x = x * sc[0];
+                                    if (Cfg::KB > 1) x = fmaf(__uint_as_float(a1[h]), sc[1], x);
+                                }
+                                acc = fmaf(s_w[j * HI + c0 + h], fmaxf(x, 0.0f), acc);
+                            }
+                        }
+                    }
+                    score[j] = acc;
+                }
+                tc_fence_before();
+                mbar_arrive(&m->tempty[buf]);
+#pragma unroll
+                for (int j = 0; j < NQ; ++j) {
+                    if (j < item.nq) {
+                        const float f = score[j] == 0.0f ? 0.0f : score[j];
+                        s_score[j * stride + li * kTileKeys + row] = f;
+                        if (pos <= item.pos[j]) atomicAdd(&s_hist[j * 2048 + (order_key(f) >> 21)], 1u);
+                    }
+                }
+            }
+            if (!ok) break;
+            named_bar_sync(1, kEpiThreads);
+
+            // ------------------------------------------------------------ Top-K select
+            uint32_t* gsync = nullptr;
+            uint32_t* ghist = nullptr;
+            uint32_t* gcnt = nullptr;
+            if (item.G > 1) {
+                uint8_t* gw = p.group_ws + (int64_t)item.group * p.group_ws_stride;
+                gsync = reinterpret_cast<uint32_t*>(gw);
+                ghist = reinterpret_cast<uint32_t*>(gw + 128);
+                gcnt = ghist + 3 * NQ * 2048;
+            }
+            int nloc[NQ];
+            bool active[NQ];
+            bool any_active = false;
+#pragma unroll
+            for (int j = 0; j < NQ; ++j) {
+                const int64_t vis = item.pos[j] + 1;      // group-wide visible positions
+                int64_t n = vis - chunk0;
+                n = n < 0 ? 0 : (n > stride ? stride : n);
+                nloc[j] = (j < item.nq) ? (int)n : 0;
+                active[j] = (j < item.nq) && vis > p.K;
+                any_active |= active[j];
+            }
+            // take-all tokens: every visible position, in place
+#pragma unroll
+            for (int j = 0; j < NQ; ++j) {
+                if (j >= item.nq || active[j]) continue;
+                const int64_t tok = item.t0 + j;
+                int32_t* oi = p.out_idx + tok * p.K;
+                float* os = p.out_score ? p.out_score + tok * p.K : nullptr;
+                for (int i = threadIdx.x; i < nloc[j]; i += kEpiThreads) {
+                    oi[chunk0 + i] = (int32_t)(chunk0 + i);
+                    if (os) os[chunk0 + i] = s_score[j * stride + i];
+                }
+                if (item.rank == 0) {
+                    for (int64_t i = item.pos[j] + 1 + threadIdx.x; i < p.K; i += kEpiThreads) {
+                        oi[i] = -1;
+                        if (os) os[i] = -__int_as_float(0x7f800000);
+                    }
+                }
+            }
+            if (any_active) {
+                uint32_t prefix[NQ], kk[NQ];
+#pragma unroll
+                for (int j = 0; j < NQ; ++j) { prefix[j] = 0; kk[j] = (uint32_t)p.K; }
+                for (int pass = 0; pass < 3 && ok; ++pass) {
+                    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+                    const int nb = pass == 2 ? 1024 : 2048;
+                    if (pass > 0) {
+                        for (int i = threadIdx.x; i < Cfg::HIST_WORDS; i += kEpiThreads) s_hist[i] = 0u;
+                        named_bar_sync(1, kEpiThreads);
+                        const uint32_t pmask = 0xFFFFFFFFu << (shift + (pass == 1 ? 11 : 10));
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) {
+                            if (!active[j]) continue;
+                            const float* sj = s_score + j * stride;
+                            for (int i = threadIdx.x; i < nloc[j]; i += kEpiThreads) {
+                                const uint32_t key = order_key(sj[i]);
+                                if ((key & pmask) == prefix[j])
+                                    atomicAdd(&s_hist[j * 2048 + ((key >> shift) & (nb - 1))], 1u);
+                            }
+                        }
+                        named_bar_sync(1, kEpiThreads);
+                    }
+                    if (item.G > 1) {
+                        uint32_t* gh = ghist + pass * NQ * 2048;
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) {
+                            if (!active[j]) continue;
+                            for (int i = threadIdx.x; i < nb; i += kEpiThreads) {
+                                const uint32_t v = s_hist[j * 2048 + i];
+                                if (v) atomicAdd(gh + j * 2048 + i, v);
+                            }
+                        }
+                        if (!group_sync(gsync, item.G, p.status, abort)) { ok = false; break; }
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) {
+                            if (!active[j]) continue;
+                            for (int i = threadIdx.x; i < nb; i += kEpiThreads)
+                                s_hist[j * 2048 + i] = __ldcg(gh + j * 2048 + i);
+                        }
+                        // the histogram of the previous pass has been read by every CTA
+                        if (item.rank == 0 && pass > 0) {
+                            uint32_t* prev = ghist + (pass - 1) * NQ * 2048;
+                            for (int i = threadIdx.x; i < NQ * 2048; i += kEpiThreads) prev[i] = 0u;
+                        }
+                        named_bar_sync(1, kEpiThreads);
+                    }
+#pragma unroll
+                    for (int j = 0; j < NQ; ++j) {
+                        if (!active[j]) continue;
+                        find_bin(s_hist + j * 2048, nb, kk[j], m->scan, &m->sel_bin[j], &m->sel_kk[j]);
+                        prefix[j] |= m->sel_bin[j] << shift;
+                        kk[j] = m->sel_kk[j];
+                    }
+                }
+                if (!ok) break;
+                // counts above / equal to the threshold, per warp (warp w owns a
+                // contiguous quarter of the chunk, so warp order is position order)
+                uint32_t wgt[NQ], weq[NQ];
+#pragma unroll
+                for (int j = 0; j < NQ; ++j) {
+                    wgt[j] = weq[j] = 0;
+                    if (!active[j]) continue;
+                    const int qlen = ((nloc[j] + 4 * 32 - 1) / (4 * 32)) * 32;
+                    const int beg = warp * qlen, end = min(nloc[j], beg + qlen);
+                    const float* sj = s_score + j * stride;
+                    for (int i0 = beg; i0 < end; i0 += 32) {
+                        const int i = i0 + lane;
+                        const bool in = i < end;
+                        const uint32_t key = in ? order_key(sj[i]) : 0u;
+                        wgt[j] += __popc(__ballot_sync(0xffffffffu, in && key > prefix[j]));
+                        weq[j] += __popc(__ballot_sync(0xffffffffu, in && key == prefix[j]));
+                    }
+                    if (lane == 0) {
+                        m->wcnt[j][warp][0] = wgt[j];
+                        m->wcnt[j][warp][1] = weq[j];
+                    }
+                }
+                named_bar_sync(1, kEpiThreads);
+                uint32_t cgt[NQ], ceq[NQ], gt_before[NQ], eq_before[NQ];
+#pragma unroll
+                for (int j = 0; j < NQ; ++j) {
+                    cgt[j] = ceq[j] = gt_before[j] = eq_before[j] = 0;
+                    for (int w = 0; w < 4; ++w) {
+                        const uint32_t g = m->wcnt[j][w][0], e = m->wcnt[j][w][1];
+                        if (w < warp) { gt_before[j] += g; eq_before[j] += e; }
+                        cgt[j] += g;
+                        ceq[j] += e;
+                    }
+                }
+                uint32_t take[NQ], base[NQ];
+#pragma unroll
+                for (int j = 0; j < NQ; ++j) { take[j] = min(kk[j], ceq[j]); base[j] = 0; }
+                if (item.G > 1) {
+                    // split the tied elements (lowest positions first, i.e. lower
+                    // ranks first) and the output offsets across the group
+                    if (threadIdx.x == 0) {
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) {
+                            if (!active[j]) continue;
+                            __stcg(gcnt + (item.rank * NQ + j) * 2, cgt[j]);
+                            __stcg(gcnt + (item.rank * NQ + j) * 2 + 1, ceq[j]);
+                        }
+                    }
+                    if (!group_sync(gsync, item.G, p.status, abort)) break;
+                    if (threadIdx.x == 0) {
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) {
+                            if (!active[j]) continue;
+                            uint32_t eqb = 0, ob = 0;
+                            for (int r = 0; r < item.rank; ++r) {
+                                const uint32_t g_gt = __ldcg(gcnt + (r * NQ + j) * 2);
+                                const uint32_t g_eq = __ldcg(gcnt + (r * NQ + j) * 2 + 1);
+                                ob += g_gt + (kk[j] > eqb ? min(kk[j] - eqb, g_eq) : 0u);
+                                eqb += g_eq;
+                            }
+                            m->sel_take[j] = kk[j] > eqb ? min(kk[j] - eqb, ceq[j]) : 0u;
+                            m->sel_base[j] = ob;
+                        }
+                    }
+                    if (item.rank == 0) {
+                        // every CTA of the group has read the last pass's histogram
+                        uint32_t* last = ghist + 2 * NQ * 2048;
+                        for (int i = threadIdx.x; i < NQ * 2048; i += kEpiThreads) last[i] = 0u;
+                    }
+                    named_bar_sync(1, kEpiThreads);
+#pragma unroll
+                    for (int j = 0; j < NQ; ++j) {
+                        take[j] = m->sel_take[j];
+                        base[j] = m->sel_base[j];
+                    }
+                }
+                // this warp's share of the tied elements
+                uint32_t allow[NQ];
+#pragma unroll
+                for (int j = 0; j < NQ; ++j) {
+                    allow[j] = take[j] > eq_before[j] ? min(take[j] - eq_before[j], weq[j]) : 0u;
+                    if (lane == 0) m->wallow[j][warp] = allow[j];
+                }
+                named_bar_sync(1, kEpiThreads);
+                const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+                for (int j = 0; j < NQ; ++j) {
+                    if (!active[j]) continue;
+                    uint32_t out = base[j] + gt_before[j];
+                    for (int w = 0; w < warp; ++w) out += m->wallow[j][w];
+                    const int qlen = ((nloc[j] + 4 * 32 - 1) / (4 * 32)) * 32;
+                    const int beg = warp * qlen, end = min(nloc[j], beg + qlen);
+                    const float* sj = s_score + j * stride;
+                    const int64_t tok = item.t0 + j;
+                    int32_t* oi = p.out_idx + tok * p.K;
+                    float* os = p.out_score ? p.out_score + tok * p.K : nullptr;
+                    uint32_t eq_seen = 0;
+                    for (int i0 = beg; i0 < end; i0 += 32) {
+                        const int i = i0 + lane;
+                        const bool in = i < end;
+                        const float f = in ? sj[i] : 0.0f;
+                        const uint32_t key = in ? order_key(f) : 0u;
+                        const bool is_gt = in && key > prefix[j];
+                        const bool is_eq = in && key == prefix[j];
+                        const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+                        const bool sel = is_gt || (is_eq && eq_seen + __popc(eqm & lt_mask) < allow[j]);
+                        const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+                        if (sel) {
+                            const uint32_t o = out + __popc(selm & lt_mask);
+                            if (o < (uint32_t)p.K) {
+                                oi[o] = (int32_t)(chunk0 + i);
+                                if (os) os[o] = f;
+                            }
+                        }
+                        out += __popc(selm);
+                        eq_seen += __popc(eqm);
+                    }
+                }
+                named_bar_sync(1, kEpiThreads);
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == Cfg::MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && m->abort) set_status(p.status, kStTimeout);
+}
+
+}  // namespace dsa

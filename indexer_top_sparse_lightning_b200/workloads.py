@@ -44,9 +44,9 @@ D_QK = D_LATENT + D_ROPE
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """float32 -> bf16 bit patterns, round to nearest even (finite inputs)."""
-    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    b = b + (((b >> 16) & 1) + 0x7FFF)
-    return (b >> 16).astype(np.uint16)
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    # no uint32 overflow for finite inputs (largest is 0xFF7FFFFF + 0x8000)
+    return ((b + ((b >> 16) & 1) + np.uint32(0x7FFF)) >> 16).astype(np.uint16)
 
 
 def bf16_bits_to_f32(u: np.ndarray) -> np.ndarray:
@@ -122,14 +122,31 @@ def _rng(seed: int, stream: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, stream])))
 
 
-def _normal_bf16(rng: np.random.Generator, shape, chunk_rows: int = 1 << 14) -> np.ndarray:
-    """N(0,1) draws rounded to bf16 bits, generated in row chunks to bound memory."""
+def _normal_bf16(seed: int, stream: int, shape, chunk_elems: int = 1 << 22) -> np.ndarray:
+    """N(0,1) draws rounded to bf16 bits.  Row chunk c draws from its own
+    stream (seed, stream, c), so the result does not depend on how many
+    threads fill the chunks."""
+    import concurrent.futures
+    import os
     shape = tuple(int(s) for s in shape)
     out = np.empty(shape, dtype=np.uint16)
     flat = out.reshape(shape[0], -1)
-    for r0 in range(0, shape[0], chunk_rows):
-        r1 = min(shape[0], r0 + chunk_rows)
-        flat[r0:r1] = to_bf16_bits(rng.standard_normal((r1 - r0, flat.shape[1]), dtype=np.float32))
+    rows = max(1, chunk_elems // max(1, flat.shape[1]))
+    starts = list(range(0, shape[0], rows))
+
+    def fill(ci):
+        r0 = starts[ci]
+        r1 = min(shape[0], r0 + rows)
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, stream, ci])))
+        flat[r0:r1] = to_bf16_bits(g.standard_normal((r1 - r0, flat.shape[1]), dtype=np.float32))
+
+    workers = min(16, os.cpu_count() or 1, len(starts))
+    if workers <= 1:
+        for ci in range(len(starts)):
+            fill(ci)
+    else:
+        with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+            list(ex.map(fill, range(len(starts))))
     return out
 
 
@@ -178,11 +195,10 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
 
     table, num_blocks = _paging(_rng(seed, 1), seq_lens, shuffle)
 
-    r = _rng(seed, 2)
     if int_inputs:
-        q_idx = to_bf16_bits(r.integers(-4, 5, size=(T, H_I, D_I)).astype(np.float32))
+        q_idx = to_bf16_bits(_rng(seed, 2).integers(-4, 5, size=(T, H_I, D_I)).astype(np.float32))
     else:
-        q_idx = _normal_bf16(r, (T, H_I, D_I))
+        q_idx = _normal_bf16(seed, 2, (T, H_I, D_I))
 
     r = _rng(seed, 3)
     u = r.random((T, H_I), dtype=np.float64)
@@ -203,7 +219,7 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
             k_f = r.integers(-4, 5, size=(n_keys, D_I)).astype(np.float32)
             k_idx = to_bf16_bits(k_f).reshape(num_blocks, BLOCK, D_I)
         else:
-            k_idx = _normal_bf16(r, (num_blocks, BLOCK, D_I))
+            k_idx = _normal_bf16(seed, 4, (num_blocks, BLOCK, D_I))
         k_scale = None
     else:
         k_f = r.standard_normal((n_keys, D_I), dtype=np.float32)
@@ -224,8 +240,8 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
         k_scale = scale.reshape(num_blocks, BLOCK, D_I // 64)
 
     if with_kv:
-        q = _normal_bf16(_rng(seed, 6), (T, H, D_QK))
-        kv = _normal_bf16(_rng(seed, 7), (num_blocks, BLOCK, D_QK))
+        q = _normal_bf16(seed, 6, (T, H, D_QK))
+        kv = _normal_bf16(seed, 7, (num_blocks, BLOCK, D_QK))
     else:
         q = np.zeros((T, H, D_QK), dtype=np.uint16)
         kv = np.zeros((0, BLOCK, D_QK), dtype=np.uint16)
@@ -261,3 +277,28 @@ def preset(name: str, with_kv: bool = True) -> Workload:
     if name == "ragged":
         kw["seq_lens"] = _rng(kw["seed"], 0).integers(16384, 131072 + 1, size=8).astype(np.int32)
     return make_workload(name, with_kv=with_kv, **kw)
+
+
+def to_device(wl: Workload, device="cuda", with_kv: bool = True) -> dict:
+    """Copy a workload's arrays to torch tensors on `device` (bf16 bits are
+    reinterpreted as torch.bfloat16, e4m3 codes stay uint8)."""
+    import torch
+
+    def t(a, dtype=None):
+        x = torch.from_numpy(np.ascontiguousarray(a))
+        if dtype is not None:
+            x = x.view(dtype)
+        return x.to(device)
+
+    d = dict(seq_lens=t(wl.seq_lens), cu_q=t(wl.cu_q), block_table=t(wl.block_table),
+             q_idx=t(wl.q_idx, torch.bfloat16), w=t(wl.w))
+    if wl.key_dtype == "bf16":
+        d["k_cache"] = t(wl.k_idx, torch.bfloat16)
+        d["k_scale"] = None
+    else:
+        d["k_cache"] = t(wl.k_idx)
+        d["k_scale"] = t(wl.k_scale)
+    if with_kv:
+        d["q"] = t(wl.q, torch.bfloat16)
+        d["kv"] = t(wl.kv, torch.bfloat16)
+    return d

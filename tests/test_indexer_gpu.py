@@ -1,0 +1,149 @@
+"""Fused Lightning Indexer + Top-K on the GPU against the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import indexer_top_sparse_lightning_b200 as dsa
+from indexer_top_sparse_lightning_b200 import workloads as W
+from tests.gpu_helpers import assert_topk, device_batch, run_indexer
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_preset_is_bit_exact():
+    # batch 1, 4096 context, 8 heads x d=64, integer q/k, K=256: fp32 scores are exact
+    wl = W.preset("tiny", with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
+
+
+def test_tie_heavy_single_cta_is_bit_exact():
+    wl = W.make_workload("ties", seq_lens=[3000], nq=1, H_I=8, D_I=64, H=1, K=256, int_inputs=True,
+                         w_dist="ones", seed=1, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
+
+
+def test_tie_heavy_groups_split_ties_by_position():
+    # long sequences are split over many CTAs: tied scores at the threshold span CTAs
+    wl = W.make_workload("ties2", seq_lens=[20000, 9000, 130], nq=[1, 2, 1], H_I=8, D_I=64, H=1, K=1024,
+                         int_inputs=True, w_dist="ones", seed=2, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
+
+
+@pytest.mark.parametrize("H_I,D_I", [(64, 128), (32, 64), (16, 128), (8, 128)])
+def test_bf16_decode_ragged_tails(H_I, D_I):
+    wl = W.make_workload("small", seq_lens=[1000, 5000, 9999], nq=1, H_I=H_I, D_I=D_I, H=1, K=512, seed=3,
+                         with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+def test_bf16_two_token_verify():
+    wl = W.make_workload("verify", seq_lens=[3000, 7001, 2], nq=2, H_I=64, D_I=128, H=1, K=1024, seed=4,
+                         with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+@pytest.mark.parametrize("nq", [1, 2])
+def test_fp8_keys(nq):
+    wl = W.make_workload("fp8", seq_lens=[4000, 9000, 700], nq=nq, H_I=64, D_I=128, H=1, K=512,
+                         key_dtype="fp8", seed=5, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+def test_contexts_around_k():
+    # fewer visible than K: every visible position, -1 padded; around the boundary
+    lens = [1, 63, 64, 65, 127, 128, 129, 2047, 2048, 2049, 4100]
+    wl = W.make_workload("edge", seq_lens=lens, nq=1, H_I=64, D_I=128, H=1, K=2048, seed=6, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+def test_many_sequences_more_than_ctas():
+    # more sequences than SMs: the launcher splits the batch over several launches
+    rng = np.random.default_rng(0)
+    lens = rng.integers(1, 3000, size=300)
+    wl = W.make_workload("many", seq_lens=lens, nq=1, H_I=16, D_I=64, H=1, K=256, seed=7, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+def test_causal_prefill_chunk():
+    # many query tokens of one sequence: one CTA per token, zig-zag order
+    wl = W.make_workload("prefill", seq_lens=[3000], nq=3000, H_I=16, D_I=64, H=1, K=512, seed=8,
+                         with_kv=False, shuffle=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+def test_prefill_after_cached_prefix():
+    # a chunk of 700 new tokens on top of 5000 cached ones, paged and shuffled
+    wl = W.make_workload("chunk", seq_lens=[5700], nq=700, H_I=32, D_I=128, H=1, K=1024, seed=9,
+                         with_kv=False)
+    idx, score = run_indexer(wl)
+    tok = np.concatenate([np.arange(0, 700, 37), [699]])
+    assert_topk(wl, tok, idx[tok], score[tok], exact=False)
+
+
+def test_score_output_is_optional():
+    wl = W.preset("tiny", with_kv=False)
+    idx, score = run_indexer(wl, want_score=False)
+    assert score is None
+    assert_topk(wl, np.arange(wl.T), idx, None, exact=True)
+
+
+def test_repeated_calls_reuse_workspace():
+    wl = W.make_workload("rep", seq_lens=[9000, 8000], nq=1, H_I=64, D_I=128, H=1, K=512, seed=10,
+                         with_kv=False)
+    d = W.to_device(wl, with_kv=False)
+    first = run_indexer(wl, d)[0]
+    for _ in range(3):
+        np.testing.assert_array_equal(run_indexer(wl, d)[0], first)
+
+
+def test_out_of_range_block_id_is_reported_not_fatal():
+    wl = W.make_workload("bad", seq_lens=[3000], nq=1, H_I=64, D_I=128, H=1, K=256, seed=11, with_kv=False)
+    d = W.to_device(wl, with_kv=False)
+    d["block_table"][0, 5] = wl.num_blocks + 7          # caught by the kernel's own range check
+    dsa.indexer_topk(device_batch(wl, d), d["q_idx"], d["w"], d["k_cache"], wl.K)
+    assert dsa.get_status() == 6                         # DSA_ERR_DEVICE_BOUNDS
+    assert dsa.get_status() == 0                         # read-and-clear
+    idx, _ = run_indexer(wl)                             # the context stays usable
+    assert idx.shape == (1, 256)
+
+
+# ---------------------------------------------------------------- full-size workloads (sampled)
+
+@pytest.mark.slow
+def test_batch32_full_size_sampled():
+    wl = W.preset("batch32", with_kv=False)
+    idx, score = run_indexer(wl)
+    tok = np.array([0, 13, 31])
+    assert_topk(wl, tok, idx[tok], score[tok], exact=False)
+
+
+@pytest.mark.slow
+def test_prefill16k_full_size_sampled():
+    wl = W.preset("prefill16k", with_kv=False)
+    idx, score = run_indexer(wl)
+    tok = np.array([0, 1, 2046, 2047, 2048, 9000, 16383])
+    assert_topk(wl, tok, idx[tok], score[tok], exact=False)
+
+
+@pytest.mark.slow
+def test_ragged_fp8_full_size_sampled():
+    wl = W.preset("ragged", with_kv=False)
+    idx, score = run_indexer(wl)
+    tok = np.array([0, 1, 7, 14, 15])
+    assert_topk(wl, tok, idx[tok], score[tok], exact=False)
+
+
+@pytest.mark.slow
+def test_million_token_planted_set():
+    wl = W.preset("1m", with_kv=False)
+    idx, score = run_indexer(wl)
+    np.testing.assert_array_equal(idx[0], wl.planted.astype(np.int32))

@@ -1,0 +1,64 @@
+"""Sparse Flash Attention on the GPU against the float64 oracle on the same index lists."""
+import numpy as np
+import pytest
+
+import oracle
+from indexer_top_sparse_lightning_b200 import workloads as W
+from tests.gpu_helpers import assert_attention, run_attention
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_idx(wl):
+    return oracle.indexer_topk(wl)["idx"]
+
+
+@pytest.mark.parametrize("K", [512, 300])
+def test_split_rows_multi_sequence(K):
+    # few tokens -> several row splits per token -> partials merged by the combine kernel
+    wl = W.make_workload("s", seq_lens=[100, 3000, 9000], nq=[1, 2, 1], H_I=8, D_I=64, H=128, K=K, seed=21)
+    idx = _oracle_idx(wl)
+    o, lse = run_attention(wl, idx)
+    assert_attention(wl, idx, np.arange(wl.T), o, lse)
+
+
+def test_sixteen_heads_tiny_preset():
+    wl = W.preset("tiny")
+    idx = _oracle_idx(wl)
+    o, lse = run_attention(wl, idx)
+    assert_attention(wl, idx, np.arange(wl.T), o, lse)
+
+
+def test_single_split_many_tokens():
+    # enough tokens that every (token) pair of CTAs takes all its rows: no partials
+    rng = np.random.default_rng(3)
+    lens = rng.integers(50, 900, size=80)
+    wl = W.make_workload("many", seq_lens=lens, nq=1, H_I=8, D_I=64, H=128, K=256, seed=22)
+    idx = _oracle_idx(wl)
+    o, lse = run_attention(wl, idx)
+    assert_attention(wl, idx, np.arange(wl.T), o, lse)
+
+
+def test_unsorted_lists_with_holes():
+    # any order, -1 holes anywhere; an all-hole token yields zeros and lse = -inf
+    wl = W.make_workload("holes", seq_lens=[5000, 2000, 64], nq=1, H_I=8, D_I=64, H=64, K=200, seed=23)
+    rng = np.random.default_rng(4)
+    pos = wl.token_pos()
+    idx = np.stack([rng.choice(int(p) + 1, size=200, replace=int(p) + 1 < 200) for p in pos]).astype(np.int32)
+    idx[0, rng.choice(200, 50, replace=False)] = -1
+    idx[2, :] = -1
+    o, lse = run_attention(wl, idx)
+    assert_attention(wl, idx, np.arange(wl.T), o, lse)
+    assert np.all(o[2] == 0) and np.all(np.isneginf(lse[2]))
+
+
+def test_peaked_logits_rescale_path():
+    # large logits: the running max jumps by far more than 2^8 between row blocks
+    wl = W.make_workload("peak", seq_lens=[3000], nq=1, H_I=8, D_I=64, H=128, K=1024, seed=24)
+    kvf = W.bf16_bits_to_f32(wl.kv).copy()
+    kvf *= 3.0
+    wl.kv = W.to_bf16_bits(kvf)
+    wl.sm_scale = 0.3
+    idx = _oracle_idx(wl)
+    o, lse = run_attention(wl, idx)
+    assert_attention(wl, idx, np.arange(wl.T), o, lse)
