@@ -108,13 +108,18 @@ typedef struct {
 } dsa_attn_inputs;
 
 /*
- * Bytes of workspace needed by indexer_topk, sparse_mla_attn and dsa_decode
- * for this batch shape (the maximum of the three; dsa_decode additionally
- * needs nothing else).  The workspace must be 256-byte aligned and
- * ZERO-FILLED before its first use; every call that completes without a
- * device error leaves it zero-filled again, so it can be reused by later
- * calls on the same stream.  After a device error (dsa_get_status != OK)
- * zero-fill it again.  Calls sharing one workspace must not overlap in time.
+ * Bytes of workspace needed for this batch shape by indexer_topk (ix given),
+ * sparse_mla_attn (at given) or both / dsa_decode (both given).  The
+ * layout is [256-byte status header][indexer group region, a fixed size per
+ * device][attention split partials]; one buffer sized with both serves all
+ * three entry points, for any mix of shapes.
+ * The workspace must be 256-byte aligned and ZERO-FILLED before its first
+ * use.  After that the library keeps it consistent by itself (a call that
+ * completes without a device error leaves its histograms zero and its
+ * barrier counters at rest), so it can be reused by later calls on the same
+ * stream; the caller must not modify it.  After a device error
+ * (dsa_get_status != OK) zero-fill it again.  Calls sharing one workspace
+ * must not overlap in time.
  * Returns 0 if the shape is invalid.
  */
 DSA_API size_t dsa_workspace_size(const dsa_batch* batch, const dsa_indexer_inputs* ix,

@@ -17,7 +17,7 @@
 using namespace dsa;
 
 static_assert(sizeof(IdxMisc) <= 1024, "indexer misc block exceeds its slot");
-static_assert(sizeof(SfaMisc) <= 2048, "attention misc block exceeds its slot");
+static_assert(sizeof(SfaMisc) <= SfaCfg::MISC_BYTES, "attention misc block exceeds its slot");
 
 namespace {
 
@@ -143,7 +143,10 @@ bool plan_for(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl) {
     while (bp >= 1 && (bp * mt + (pl.grid - bp) - 1) / (pl.grid - bp > 0 ? pl.grid - bp : 1) > cap_tiles) --bp;
     if (bp < 1) return false;
     pl.seqs_per_launch = (int)bp;
-    pl.group_ws = (size_t)bp * (size_t)group_ws_bytes(NQ, pl.grid);
+    // one stride for every NQ: the barrier words of group g sit at the same
+    // offset whichever kernel used the workspace last (they are not zero
+    // between calls; everything else is)
+    pl.group_ws = (size_t)bp * (size_t)group_ws_bytes(2, pl.grid);
     return true;
 }
 
@@ -194,7 +197,7 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
     p.out_score = out_score;
     p.status = status;
     p.group_ws = group_ws;
-    p.group_ws_stride = group_ws_bytes(NQ, pl.grid);
+    p.group_ws_stride = group_ws_bytes(2, pl.grid);
     p.B = bt->batch;
     p.T = bt->num_tokens;
     p.max_blocks = bt->max_blocks_per_seq;
@@ -302,6 +305,15 @@ AttnPlan plan_attn(const dsa_batch* bt, int K, const DevInfo& di) {
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Workspace layout, the same for every shape on a given device:
+//   [header 256 B][indexer group region, fixed size][attention partials]
+// The indexer region is sized for the largest grouped launch (one group per
+// SM, two tokens per group), so calls of any shape sharing one workspace
+// never write attention partials over the indexer's zero-filled region.
+size_t idx_region_bytes(const DevInfo& di) {
+    return align256((size_t)di.sms * (size_t)group_ws_bytes(2, di.sms));
+}
+
 dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int32_t* idx, int K, void* out,
                        float* lse, uint32_t* status, uint8_t* part, const AttnPlan& ap, cudaStream_t stream) {
     CUtensorMap tm_q;
@@ -367,21 +379,18 @@ size_t dsa_workspace_size(const dsa_batch* batch, const dsa_indexer_inputs* ix, 
     if (check_batch(batch) != DSA_OK) return 0;
     const DevInfo di = dev_info();
     if (di.sms <= 0) return 0;
-    size_t need = kHeaderBytes;
-    size_t ix_bytes = 0, at_bytes = 0;
+    size_t need = kHeaderBytes + idx_region_bytes(di);
     if (ix) {
         if (check_indexer(ix) != DSA_OK) return 0;
         IdxPlan pl;
         LaunchFn fn = nullptr;
         if (plan_indexer(batch, ix, di, pl, fn) != DSA_OK) return 0;
-        ix_bytes = align256(pl.group_ws);
+        if (pl.group_ws > idx_region_bytes(di)) return 0;
     }
     if (at) {
         if (check_attn(at) != DSA_OK) return 0;
-        const int K = ix ? ix->K : kMaxTopK;
-        at_bytes = align256(plan_attn(batch, K, di).part_bytes);
+        need += align256(plan_attn(batch, kMaxTopK, di).part_bytes);
     }
-    need += ix_bytes > at_bytes ? ix_bytes : at_bytes;
     return need;
 }
 
@@ -397,6 +406,7 @@ dsa_status indexer_topk(const dsa_batch* batch, const dsa_indexer_inputs* ix, in
     IdxPlan pl;
     LaunchFn fn = nullptr;
     if ((st = plan_indexer(batch, ix, di, pl, fn)) != DSA_OK) return st;
+    if (pl.group_ws > idx_region_bytes(di)) return DSA_ERR_UNSUPPORTED;
     if (workspace_bytes < kHeaderBytes + pl.group_ws) return DSA_ERR_WORKSPACE;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     return fn(batch, ix, out_idx, out_score, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, pl,
@@ -414,9 +424,10 @@ dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs* at, co
     const DevInfo di = dev_info();
     if (di.sms <= 0 || di.max_smem < SfaCfg::SMEM) return DSA_ERR_CUDA;
     const AttnPlan ap = plan_attn(batch, K, di);
-    if (workspace_bytes < kHeaderBytes + ap.part_bytes) return DSA_ERR_WORKSPACE;
+    const size_t off = kHeaderBytes + idx_region_bytes(di);
+    if (workspace_bytes < off + ap.part_bytes) return DSA_ERR_WORKSPACE;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-    return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, ap,
+    return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + off, ap,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -476,5 +487,13 @@ const char* dsa_status_str(int32_t s) {
 }
 
 const char* dsa_version(void) { return "dsa-b200 0.1.0 (sm_100a)"; }
+
+#ifdef DSA_TRACE
+// Tracing builds only: copy the per-CTA %globaltimer table ([2048][16] u64).
+DSA_API int32_t dsa_trace_read(void* host_dst, size_t bytes) {
+    if (bytes > sizeof(g_dsa_trace)) bytes = sizeof(g_dsa_trace);
+    return cudaMemcpyFromSymbol(host_dst, g_dsa_trace, bytes) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+#endif
 
 }  // extern "C"

@@ -71,7 +71,9 @@ struct IdxCfg {
     static constexpr int OFF_W = OFF_HIST + HIST_WORDS * 4;
     static constexpr int OFF_MISC = OFF_W + ((W_FLOATS * 4 + 127) / 128) * 128;
     static constexpr int MISC_BYTES = 1024;
-    static constexpr int OFF_SCORE = OFF_MISC + MISC_BYTES;
+    static constexpr int MAX_PAGES = 512;                     // page ids of one work item, staged in smem
+    static constexpr int OFF_BLK = OFF_MISC + MISC_BYTES;
+    static constexpr int OFF_SCORE = OFF_BLK + MAX_PAGES * 4;
     // dynamic shared memory = 1024 (alignment slack) + OFF_SCORE + score_cap * 4
     static constexpr int FIXED_SMEM = 1024 + OFF_SCORE;
 };
@@ -336,38 +338,51 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = m->tmem_base;
+    if (threadIdx.x == 0) DSA_TRACE_MARK(0);
 
     if (warp == Cfg::PRODUCER_WARP) {
         // ---------------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            uint32_t it = 0;
-            IdxItem item;
-            for (int k = 0; get_item<NQ>(p, m, k, item); ++k) {
-                if (!mbar_wait(&m->q_empty, (k & 1) ^ 1, abort)) break;
-                mbar_arrive_expect_tx(&m->q_full, Cfg::Q_TX);
-                for (int kb = 0; kb < Cfg::KB; ++kb)
-                    tma_load_3d(s_q + kb * Cfg::N * 128, &tm_q, &m->q_full, kb * 64, 0, item.t0);
-                const int64_t npages = (item.L + kPage - 1) / kPage;
-                bool ok = true;
-                for (int li = 0; li < item.tile_count; ++li, ++it) {
+        int32_t* s_blk = reinterpret_cast<int32_t*>(smem + Cfg::OFF_BLK);
+        const uint64_t pol = policy_evict_first();
+        uint32_t it = 0;
+        IdxItem item;
+        for (int k = 0; get_item<NQ>(p, m, k, item); ++k) {
+            // the page ids of this chunk, staged with one coalesced warp load
+            const int64_t npages = (item.L + kPage - 1) / kPage;
+            const int pg0 = item.tile_begin * 2;
+            int npg = item.tile_count * 2;
+            if (pg0 + npg > npages) npg = (int)(npages - pg0);
+            if (npg > Cfg::MAX_PAGES) {
+                set_status(p.status, kStCapacity);
+                npg = Cfg::MAX_PAGES;
+            }
+            __syncwarp();
+            for (int i = lane; i < npg; i += 32) {
+                int bid = __ldg(p.block_table + (int64_t)item.b * p.max_blocks + pg0 + i);
+                if (bid < 0 || bid >= p.num_blocks) {
+                    set_status(p.status, kStBounds);
+                    bid = -1;   // out-of-range coordinate: TMA fills zeros
+                }
+                s_blk[i] = bid;
+            }
+            __syncwarp();
+            int ok = 1;
+            if (lane == 0) {
+                if (!mbar_wait(&m->q_empty, (k & 1) ^ 1, abort)) ok = 0;
+                if (ok) {
+                    mbar_arrive_expect_tx(&m->q_full, Cfg::Q_TX);
+                    for (int kb = 0; kb < Cfg::KB; ++kb)
+                        tma_load_3d(s_q + kb * Cfg::N * 128, &tm_q, &m->q_full, kb * 64, 0, item.t0);
+                }
+                for (int li = 0; ok && li < item.tile_count; ++li, ++it) {
                     const int s = it % Cfg::NSTAGE;
-                    if (!mbar_wait(&m->empty[s], ((it / Cfg::NSTAGE) & 1) ^ 1, abort)) { ok = false; break; }
-                    const int tile = item.tile_begin + li;
+                    if (!mbar_wait(&m->empty[s], ((it / Cfg::NSTAGE) & 1) ^ 1, abort)) { ok = 0; break; }
                     int blk[2];
                     int nvalid = 0;
                     for (int pp = 0; pp < 2; ++pp) {
-                        const int64_t pg = (int64_t)tile * 2 + pp;
-                        blk[pp] = -2;
-                        if (pg < npages) {
-                            int bid = __ldg(p.block_table + (int64_t)item.b * p.max_blocks + pg);
-                            if (bid < 0 || bid >= p.num_blocks) {
-                                set_status(p.status, kStBounds);
-                                bid = -1;   // out-of-range coordinate: TMA fills zeros
-                            }
-                            blk[pp] = bid;
-                            ++nvalid;
-                        }
+                        const int i = li * 2 + pp;
+                        blk[pp] = i < npg ? s_blk[i] : -2;
+                        nvalid += i < npg;
                     }
                     uint8_t* st = s_stage + s * Cfg::STAGE_BYTES;
                     mbar_arrive_expect_tx(&m->full[s], nvalid * kPage * DI * (FP8 ? 1 : 2));
@@ -382,9 +397,13 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         }
                     }
                 }
-                if (!ok) break;
             }
-            // drain: no TMA write may still be in flight when the CTA exits
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+        }
+        if (lane == 0) DSA_TRACE_MARK(8);
+        // drain: no TMA write may still be in flight when the CTA exits
+        if (lane == 0) {
             const uint32_t first = it > (uint32_t)Cfg::NSTAGE ? it - Cfg::NSTAGE : 0u;
             volatile int no_abort = 0;
             for (uint32_t d = first; d < it; ++d)
@@ -514,6 +533,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                     }
                 }
                 if (!mbar_wait(&m->tfull[buf], (it >> 1) & 1, abort)) { ok = false; break; }
+                if (li == 0 && threadIdx.x == 0) DSA_TRACE_MARK(1);
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * Cfg::COLS_BUF;
                 float score[NQ];
@@ -563,6 +583,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             }
             if (!ok) break;
             named_bar_sync(1, kEpiThreads);
+            if (threadIdx.x == 0) DSA_TRACE_MARK(2);
 
             // ------------------------------------------------------------ Top-K select
             uint32_t* gsync = nullptr;
@@ -658,6 +679,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         prefix[j] |= m->sel_bin[j] << shift;
                         kk[j] = m->sel_kk[j];
                     }
+                    if (threadIdx.x == 0) DSA_TRACE_MARK(3 + pass);
                 }
                 if (!ok) break;
                 // counts above / equal to the threshold, per warp (warp w owns a
@@ -736,6 +758,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         base[j] = m->sel_base[j];
                     }
                 }
+                if (threadIdx.x == 0) DSA_TRACE_MARK(6);
                 // this warp's share of the tied elements
                 uint32_t allow[NQ];
 #pragma unroll
@@ -780,6 +803,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 }
                 named_bar_sync(1, kEpiThreads);
             }
+            if (threadIdx.x == 0) DSA_TRACE_MARK(7);
         }
     }
 
@@ -791,6 +815,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
     if (threadIdx.x == 0 && m->abort) set_status(p.status, kStTimeout);
+    if (threadIdx.x == 0) DSA_TRACE_MARK(9);
 }
 
 }  // namespace dsa

@@ -23,6 +23,21 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
+// ------------------------------------------------------------------ phase tracing (debug builds only)
+// Built with -DDSA_TRACE, kernels record %globaltimer at fixed points of
+// each CTA's life into a device table read back by dsa_trace_read().
+#ifdef DSA_TRACE
+__device__ uint64_t g_dsa_trace[2048][16];
+#define DSA_TRACE_MARK(slot)                                                     \
+    do {                                                                         \
+        if (blockIdx.x < 2048) g_dsa_trace[blockIdx.x][(slot)] = globaltimer(); \
+    } while (0)
+#else
+#define DSA_TRACE_MARK(slot) \
+    do {                     \
+    } while (0)
+#endif
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -53,7 +53,11 @@ struct SfaCfg {
     static constexpr int OFF_P = OFF_KV + NS * STAGE_BYTES;
     static constexpr int OFF_X = OFF_P + P_BYTES;
     static constexpr int OFF_MISC = OFF_X + X_BYTES;
-    static constexpr int SMEM = 1024 + OFF_MISC + 2048;
+    static constexpr int MISC_BYTES = 1024;
+    static constexpr int MAX_ROWS = 2048;               // rows of one split (K <= 2048)
+    static constexpr int OFF_ROWS = OFF_MISC + MISC_BYTES;
+    static constexpr int OFF_VALID = OFF_ROWS + MAX_ROWS * 4;
+    static constexpr int SMEM = 1024 + OFF_VALID + MAX_ROWS / 8;
     static constexpr int THREADS = 288;
     static constexpr int TMEM_COLS = 512;               // O: [0,256), S buffers: [256,320), [320,384)
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, ROWS, false, false);
@@ -72,9 +76,9 @@ struct SfaMisc {
     uint64_t x_full;    // peer's partial logits have landed in my X buffer
     uint64_t x_free;    // peer has consumed the logits I wrote into its X buffer
     uint64_t drain;
+    uint64_t rows_ready;   // physical rows and validity bits of the split are in shared memory
     uint32_t tmem_base;
     int abort;
-    int64_t row_off[SfaCfg::NS][SfaCfg::ROWS];   // byte offset of each gathered row, -1 = skip
 };
 
 __device__ __forceinline__ int token_sequence(const int32_t* cu_q, int B, int t) {
@@ -96,6 +100,8 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     uint8_t* s_p = smem + Cfg::OFF_P;
     float* s_x = reinterpret_cast<float*>(smem + Cfg::OFF_X);
     SfaMisc* m = reinterpret_cast<SfaMisc*>(smem + Cfg::OFF_MISC);
+    int32_t* s_rows = reinterpret_cast<int32_t*>(smem + Cfg::OFF_ROWS);
+    uint32_t* s_valid = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_VALID);
     volatile int* abort = &m->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -125,6 +131,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         mbar_init(&m->x_full, 128);
         mbar_init(&m->x_free, 128);
         mbar_init(&m->drain, 1);
+        mbar_init(&m->rows_ready, 128);
         m->abort = 0;
         fence_mbar_init();
     }
@@ -144,6 +151,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     const uint32_t tmem_base = m->tmem_base;
     const uint32_t tm_o = tmem_base;            // columns [0, 256)
     const uint32_t tm_s = tmem_base + 256;      // two 64-column logit buffers
+    if (threadIdx.x == 0) DSA_TRACE_MARK(0);
 
     if (warp == 8) {
         // ---------------------------------------------------------------- MMA issuer
@@ -210,37 +218,44 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         const int nch = kbq * 8;                    // 16-byte chunks per row held by this CTA
         const int32_t* idx_t = p.idx + (int64_t)t * p.K;
         const uint8_t* kv_bytes = reinterpret_cast<const uint8_t*>(p.kv);
+        // physical row of every selected position of this split, and validity bits, once
+        const int nrows = nblk * Cfg::ROWS;
+        for (int i = pt; i < nrows; i += 128) {
+            const int r = row_begin + i;
+            int32_t row = -1;
+            if (r < row_end) {
+                const int32_t pos = __ldg(idx_t + r);
+                if (pos >= 0) {
+                    if (pos < L && pos / kPage < p.max_blocks) {
+                        const int blk = __ldg(p.block_table + (int64_t)b * p.max_blocks + pos / kPage);
+                        if (blk >= 0 && blk < p.num_blocks)
+                            row = blk * kPage + pos % kPage;
+                        else
+                            atomicCAS(p.status, 0u, (uint32_t)kStBounds);
+                    } else {
+                        atomicCAS(p.status, 0u, (uint32_t)kStBounds);
+                    }
+                }
+            }
+            s_rows[i] = row;
+            const uint32_t bits = __ballot_sync(0xffffffffu, row >= 0);
+            if ((i & 31) == 0) s_valid[i >> 5] = bits;
+        }
+        mbar_arrive(&m->rows_ready);
+        if (pt == 0) DSA_TRACE_MARK(1);
+        named_bar_sync(2, 128);
         for (int jb = 0; jb < nblk; ++jb) {
             const int s = jb % Cfg::NS;
             if (!mbar_wait(&m->kv_empty[s], ((jb / Cfg::NS) & 1) ^ 1, abort)) break;
-            if (pt < Cfg::ROWS) {
-                const int r = row_begin + jb * Cfg::ROWS + pt;
-                int64_t off = -1;
-                if (r < row_end) {
-                    const int32_t pos = __ldg(idx_t + r);
-                    if (pos >= 0) {
-                        if (pos < L && pos / kPage < p.max_blocks) {
-                            const int blk = __ldg(p.block_table + (int64_t)b * p.max_blocks + pos / kPage);
-                            if (blk >= 0 && blk < p.num_blocks)
-                                off = ((int64_t)blk * kPage + pos % kPage) * (kDqk * 2);
-                            else
-                                atomicCAS(p.status, 0u, (uint32_t)kStBounds);
-                        } else {
-                            atomicCAS(p.status, 0u, (uint32_t)kStBounds);
-                        }
-                    }
-                }
-                m->row_off[s][pt] = off;
-            }
-            named_bar_sync(2, 128);
             const uint32_t st = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
+            const int32_t* rows = s_rows + jb * Cfg::ROWS;
             for (int e = pt; e < Cfg::ROWS * nch; e += 128) {
                 const int r = e / nch, ch = e % nch;
                 const int kb = ch >> 3, q = ch & 7;
                 const int byte = crank == 0 ? (kb < 4 ? kb * 128 + q * 16 : 1024 + q * 16) : 512 + kb * 128 + q * 16;
-                const int64_t off = m->row_off[s][r];
-                const void* src = kv_bytes + (off >= 0 ? off + byte : 0);
-                cp_async_16(st + kb * Cfg::KV_KB_BYTES + r * 128 + ((q ^ (r & 7)) << 4), src, off >= 0);
+                const int32_t row = rows[r];
+                const void* src = kv_bytes + (row >= 0 ? (int64_t)row * (kDqk * 2) + byte : 0);
+                cp_async_16(st + kb * Cfg::KV_KB_BYTES + r * 128 + ((q ^ (r & 7)) << 4), src, row >= 0);
             }
             // the barrier receives this thread's arrival once its copies have landed
             cp_async_arrive_noinc(&m->kv_full[s]);
@@ -253,22 +268,14 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         const uint32_t x_full_peer = mapa_shared(smem_u32(&m->x_full), peer);
         const uint32_t x_free_peer = mapa_shared(smem_u32(&m->x_free), peer);
         const uint32_t x_peer_row = mapa_shared(smem_u32(s_x + h * Cfg::ROWS), peer);
-        const int32_t* idx_t = p.idx + (int64_t)t * p.K;
         float mrun = -INFINITY, lrun = 0.0f;
-        bool ok = true;
-        for (int jb = 0; jb < nblk; ++jb) {
+        bool ok = nblk == 0 || mbar_wait(&m->rows_ready, 0, abort);
+        for (int jb = 0; ok && jb < nblk; ++jb) {
             const int sb = jb & 1;
             // validity of the 64 rows of this block (same for every head)
-            uint32_t vmask[2] = {0u, 0u};
-            {
-                const int r0 = row_begin + jb * Cfg::ROWS;
-                for (int i = 0; i < Cfg::ROWS; ++i) {
-                    const int r = r0 + i;
-                    const bool v = r < row_end && __ldg(idx_t + r) >= 0;
-                    vmask[i >> 5] |= (v ? 1u : 0u) << (i & 31);
-                }
-            }
+            const uint32_t vmask[2] = {s_valid[jb * 2], s_valid[jb * 2 + 1]};
             if (!mbar_wait(&m->s_full[sb], (jb >> 1) & 1, abort)) { ok = false; break; }
+            if (jb == 0 && h == 0) DSA_TRACE_MARK(2);
             tc_fence_after();
             uint32_t a[32], c[32];
             tmem_ld32(tm_s + lane_off + sb * Cfg::ROWS, a);
@@ -353,7 +360,9 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             mbar_arrive(&m->p_full);
         }
         // ---------------------------------------------------------------- epilogue
+        if (h == 0) DSA_TRACE_MARK(3);
         if (ok && mbar_wait(&m->o_full, 0, abort)) {
+            if (h == 0) DSA_TRACE_MARK(4);
             tc_fence_after();
             const int dim0 = crank == 0 ? 0 : 256;
             if (p.n_splits == 1) {
@@ -419,6 +428,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
     if (threadIdx.x == 0 && m->abort) atomicCAS(p.status, 0u, (uint32_t)kStTimeout);
+    if (threadIdx.x == 0) DSA_TRACE_MARK(9);
 }
 
 // Merge the row-split partials of each (token, head): weights 2^(m_s - M).

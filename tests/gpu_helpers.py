@@ -38,7 +38,8 @@ def run_indexer(wl, d=None, want_score=True):
     idx, score = dsa.indexer_topk(device_batch(wl, d), d["q_idx"], d["w"], d["k_cache"], wl.K,
                                   k_scale=d["k_scale"], want_score=want_score)
     torch.cuda.synchronize()
-    assert dsa.get_status() == 0
+    st = dsa.get_status()
+    assert st == 0, f"device status {st}: {dsa.status_str(st)}"
     return idx.cpu().numpy(), (score.cpu().numpy() if score is not None else None)
 
 
@@ -81,7 +82,8 @@ def run_attention(wl, idx_np, d=None):
     idx = torch.from_numpy(np.ascontiguousarray(idx_np, dtype=np.int32)).cuda()
     out, lse = dsa.sparse_mla_attn(device_batch(wl, d), d["q"], d["kv"], idx, wl.sm_scale)
     torch.cuda.synchronize()
-    assert dsa.get_status() == 0
+    st = dsa.get_status()
+    assert st == 0, f"device status {st}: {dsa.status_str(st)}"
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
 

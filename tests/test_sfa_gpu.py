@@ -54,11 +54,9 @@ def test_unsorted_lists_with_holes():
 
 def test_peaked_logits_rescale_path():
     # large logits: the running max jumps by far more than 2^8 between row blocks
+    # (logit std ~24 with sm_scale = 1: nearly one-hot rows, repeated max jumps)
     wl = W.make_workload("peak", seq_lens=[3000], nq=1, H_I=8, D_I=64, H=128, K=1024, seed=24)
-    kvf = W.bf16_bits_to_f32(wl.kv).copy()
-    kvf *= 3.0
-    wl.kv = W.to_bf16_bits(kvf)
-    wl.sm_scale = 0.3
+    wl.sm_scale = 1.0
     idx = _oracle_idx(wl)
     o, lse = run_attention(wl, idx)
     assert_attention(wl, idx, np.arange(wl.T), o, lse)
