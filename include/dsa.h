@@ -110,9 +110,10 @@ typedef struct {
 /*
  * Bytes of workspace needed for this batch shape by indexer_topk (ix given),
  * sparse_mla_attn (at given) or both / dsa_decode (both given).  The
- * layout is [256-byte status header][indexer group region, a fixed size per
- * device][attention split partials]; one buffer sized with both serves all
- * three entry points, for any mix of shapes.
+ * layout is [256-byte status word area][1 KB of split arrival counters]
+ * [indexer group region, a fixed size per device][attention split
+ * partials]; one buffer sized with both serves all three entry points, for
+ * any mix of shapes.
  * The workspace must be 256-byte aligned and ZERO-FILLED before its first
  * use.  After that the library keeps it consistent by itself (a call that
  * completes without a device error leaves its histograms zero and its

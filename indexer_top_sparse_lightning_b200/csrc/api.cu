@@ -21,7 +21,10 @@ static_assert(sizeof(SfaMisc) <= SfaCfg::MISC_BYTES, "attention misc block excee
 
 namespace {
 
-constexpr size_t kHeaderBytes = 256;
+constexpr size_t kStatusBytes = 256;
+constexpr int kMaxSplitTokens = 128;      // row splits are only used for fewer tokens than this
+constexpr size_t kCounterBytes = kMaxSplitTokens * 2 * 4;
+constexpr size_t kHeaderBytes = kStatusBytes + kCounterBytes;
 
 // ------------------------------------------------------------------ driver entry point (no libcuda link)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -293,20 +296,21 @@ AttnPlan plan_attn(const dsa_batch* bt, int K, const DevInfo& di) {
     AttnPlan ap;
     const int max_splits = (K + SfaCfg::ROWS - 1) / SfaCfg::ROWS;
     int s = di.sms / (2 * bt->num_tokens);
-    if (s < 1) s = 1;
+    if (s < 1 || bt->num_tokens > kMaxSplitTokens) s = 1;
     if (s > max_splits) s = max_splits;
     const int per = (K + s - 1) / s;
     ap.rows_per_split = ((per + SfaCfg::ROWS - 1) / SfaCfg::ROWS) * SfaCfg::ROWS;
     ap.splits = (K + ap.rows_per_split - 1) / ap.rows_per_split;
     if (ap.splits > 1)
-        ap.part_bytes = (size_t)bt->num_tokens * ap.splits * (128 * kDv * 4 + 256 * 4);
+        ap.part_bytes = (size_t)bt->num_tokens * ap.splits * (128 * kDv * 4 + 2 * 256 * 4);
     return ap;
 }
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace layout, the same for every shape on a given device:
-//   [header 256 B][indexer group region, fixed size][attention partials]
+//   [status 256 B][split arrival counters 1 KB][indexer group region, fixed
+//   size][attention partials]
 // The indexer region is sized for the largest grouped launch (one group per
 // SM, two tokens per group), so calls of any shape sharing one workspace
 // never write attention partials over the indexer's zero-filled region.
@@ -347,6 +351,7 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     if (ap.splits > 1) {
         p.part_o = reinterpret_cast<float*>(part);
         p.part_ml = reinterpret_cast<float*>(part + (size_t)bt->num_tokens * ap.splits * 128 * kDv * 4);
+        p.split_count = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(status) + kStatusBytes);
     }
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof cfg);
@@ -362,10 +367,6 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, &sfa_decode_kernel, p, tm_q) != cudaSuccess) return DSA_ERR_CUDA;
-    if (ap.splits > 1) {
-        sfa_combine_kernel<<<bt->num_tokens * 64, 256, 0, stream>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-    }
     return DSA_OK;
 }
 
@@ -469,7 +470,8 @@ int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexer_inputs
     if (plan_indexer(batch, ix, di, pl, fn) != DSA_OK) return -1;
     const int idx_launches = pl.mode == 1 ? 1 : (batch->batch + pl.seqs_per_launch - 1) / pl.seqs_per_launch;
     const AttnPlan ap = plan_attn(batch, ix->K, di);
-    return idx_launches + 1 + (ap.splits > 1 ? 1 : 0);
+    (void)ap;   // the split merge runs inside the attention kernel
+    return idx_launches + 1;
 }
 
 const char* dsa_status_str(int32_t s) {
@@ -493,6 +495,10 @@ const char* dsa_version(void) { return "dsa-b200 0.1.0 (sm_100a)"; }
 DSA_API int32_t dsa_trace_read(void* host_dst, size_t bytes) {
     if (bytes > sizeof(g_dsa_trace)) bytes = sizeof(g_dsa_trace);
     return cudaMemcpyFromSymbol(host_dst, g_dsa_trace, bytes) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+DSA_API int32_t dsa_trace_blk_read(void* host_dst, size_t bytes) {
+    if (bytes > sizeof(g_dsa_trace_blk)) bytes = sizeof(g_dsa_trace_blk);
+    return cudaMemcpyFromSymbol(host_dst, g_dsa_trace_blk, bytes) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 #endif
 

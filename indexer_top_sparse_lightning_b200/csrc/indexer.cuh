@@ -33,6 +33,7 @@
 #pragma once
 #include "common.h"
 #include "ptx.cuh"
+#include "select.cuh"
 
 namespace dsa {
 
@@ -73,7 +74,8 @@ struct IdxCfg {
     static constexpr int MISC_BYTES = 1024;
     static constexpr int MAX_PAGES = 512;                     // page ids of one work item, staged in smem
     static constexpr int OFF_BLK = OFF_MISC + MISC_BYTES;
-    static constexpr int OFF_SCORE = OFF_BLK + MAX_PAGES * 4;
+    static constexpr int OFF_LIST = OFF_BLK + MAX_PAGES * 4;   // select lists, u16 [NQ][4 warps][cap]
+    static constexpr int OFF_SCORE = OFF_LIST + NQ * 4 * kListCap * 2;
     // dynamic shared memory = 1024 (alignment slack) + OFF_SCORE + score_cap * 4
     static constexpr int FIXED_SMEM = 1024 + OFF_SCORE;
 };
@@ -92,13 +94,7 @@ struct IdxMisc {
     int abort;
     // mode-0 assignment of this CTA
     int g_valid, g_b, g_rank, g_size, g_tile_begin, g_tile_count, g_group;
-    uint32_t scan[8];
-    uint32_t wcnt[4][4][2];   // [token][warp][gt, eq]
-    uint32_t wallow[4][4];    // [token][warp] tied elements the warp may take
-    uint32_t sel_bin[4];
-    uint32_t sel_kk[4];
-    uint32_t sel_take[4];
-    uint32_t sel_base[4];
+    SelectSmem sel;
 };
 
 // One unit of work: a group of query tokens of one sequence and a chunk of
@@ -109,10 +105,6 @@ struct IdxItem {
     int64_t L;
     int64_t pos[4];
 };
-
-__device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) {
-    atomicCAS(status, 0u, code);
-}
 
 template <int NQ>
 __device__ __forceinline__ bool get_item(const IndexerParams& p, const IdxMisc* m, int k, IdxItem& it) {
@@ -205,84 +197,6 @@ __device__ void assign_groups(const IndexerParams& p, IdxMisc* m, int nq_max, in
     }
 }
 
-// Bounded barrier among the CTAs of one group (called by the 128 epilogue
-// threads).  Sense-reversing: the last arriver resets the count and bumps
-// the generation.
-__device__ bool group_sync(uint32_t* sync, int G, uint32_t* status, volatile int* abort) {
-    named_bar_sync(1, kEpiThreads);
-    if (threadIdx.x == 0 && !*abort) {
-        uint32_t* count = sync;
-        uint32_t* gen = sync + 1;
-        const uint32_t g0 = ld_acquire_gpu(gen);
-        const uint32_t old = atom_add_acq_rel_gpu(count, 1u);
-        if (old == (uint32_t)G - 1u) {
-            *reinterpret_cast<volatile uint32_t*>(count) = 0u;
-            st_release_gpu(gen, g0 + 1u);
-        } else {
-            const uint64_t t0 = globaltimer();
-            while (ld_acquire_gpu(gen) == g0) {
-                if (globaltimer() - t0 > kWaitTimeoutNs) {
-                    set_status(status, kStTimeout);
-                    *abort = 1;
-                    break;
-                }
-                __nanosleep(64);
-            }
-        }
-    }
-    named_bar_sync(1, kEpiThreads);
-    return !*abort;
-}
-
-// Exclusive prefix over the 128 epilogue threads; *total receives the sum.
-__device__ __forceinline__ uint32_t epi_exclusive_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) scratch[warp] = x;
-    named_bar_sync(1, kEpiThreads);
-    uint32_t before = 0, all = 0;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        const uint32_t s = scratch[w];
-        if (w < warp) before += s;
-        all += s;
-    }
-    named_bar_sync(1, kEpiThreads);
-    *total = all;
-    return before + x - v;
-}
-
-// Radix step: given the histogram of the current digit (nb bins, highest bin
-// first is most significant), find the bin holding the kk-th largest element.
-__device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t kk, uint32_t* scratch,
-                                         uint32_t* out_bin, uint32_t* out_kk) {
-    const int per = nb / kEpiThreads;
-    const int t = threadIdx.x;
-    const int hi_bin = nb - 1 - t * per;
-    uint32_t s = 0;
-    for (int i = 0; i < per; ++i) s += hist[hi_bin - i];
-    uint32_t total;
-    const uint32_t before = epi_exclusive_scan(s, scratch, &total);
-    if (before < kk && kk <= before + s) {
-        uint32_t c = before;
-        for (int i = 0; i < per; ++i) {
-            const uint32_t h = hist[hi_bin - i];
-            if (c + h >= kk) {
-                *out_bin = (uint32_t)(hi_bin - i);
-                *out_kk = kk - c;
-                break;
-            }
-            c += h;
-        }
-    }
-    named_bar_sync(1, kEpiThreads);
-}
-
 template <bool FP8, int HI, int DI, int NQ>
 __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
     indexer_topk_kernel(const __grid_constant__ IndexerParams p, const __grid_constant__ CUtensorMap tm_q,
@@ -297,6 +211,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
     float* s_w = reinterpret_cast<float*>(smem + Cfg::OFF_W);
     IdxMisc* m = reinterpret_cast<IdxMisc*>(smem + Cfg::OFF_MISC);
     float* s_score = reinterpret_cast<float*>(smem + Cfg::OFF_SCORE);
+    uint16_t* s_list = reinterpret_cast<uint16_t*>(smem + Cfg::OFF_LIST);
     volatile int* abort = &m->abort;
 
     const int warp = threadIdx.x >> 5;
@@ -513,6 +428,16 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 s_w[i] = (j < item.nq) ? __ldg(p.w + (int64_t)(item.t0 + j) * HI + (i % HI)) : 0.0f;
             }
             for (int i = threadIdx.x; i < Cfg::HIST_WORDS; i += kEpiThreads) s_hist[i] = 0u;
+            GroupView gv{nullptr, nullptr, nullptr, item.G, item.rank};
+            uint32_t gen = 0;
+            if (item.G > 1) {
+                uint8_t* gw = p.group_ws + (int64_t)item.group * p.group_ws_stride;
+                gv.sync = reinterpret_cast<uint32_t*>(gw);
+                gv.hist = reinterpret_cast<uint32_t*>(gw + 128);
+                gv.cnt = gv.hist + 3 * NQ * 2048;
+                // the group's barrier generation cannot move before this CTA arrives
+                if (threadIdx.x == 0) gen = ld_acquire_gpu(gv.sync + 1);
+            }
             named_bar_sync(1, kEpiThreads);
             const int stride = item.tile_count * kTileKeys;   // score slots per token
             const int64_t chunk0 = (int64_t)item.tile_begin * kTileKeys;
@@ -577,7 +502,15 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                     if (j < item.nq) {
                         const float f = score[j] == 0.0f ? 0.0f : score[j];
                         s_score[j * stride + li * kTileKeys + row] = f;
-                        if (pos <= item.pos[j]) atomicAdd(&s_hist[j * 2048 + (order_key(f) >> 21)], 1u);
+                        // pass-0 digit histogram; lanes with the same bin add once (scores of a
+                        // tile cluster in few bins, so plain atomics would serialize)
+                        const bool vis = pos <= item.pos[j];
+                        const uint32_t bin = order_key(f) >> 21;
+                        const uint32_t act = __ballot_sync(0xffffffffu, vis);
+                        if (vis) {
+                            const uint32_t peers = __match_any_sync(act, bin);
+                            if ((int)(__ffs(peers) - 1) == lane) atomicAdd(&s_hist[j * 2048 + bin], (uint32_t)__popc(peers));
+                        }
                     }
                 }
             }
@@ -586,15 +519,6 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             if (threadIdx.x == 0) DSA_TRACE_MARK(2);
 
             // ------------------------------------------------------------ Top-K select
-            uint32_t* gsync = nullptr;
-            uint32_t* ghist = nullptr;
-            uint32_t* gcnt = nullptr;
-            if (item.G > 1) {
-                uint8_t* gw = p.group_ws + (int64_t)item.group * p.group_ws_stride;
-                gsync = reinterpret_cast<uint32_t*>(gw);
-                ghist = reinterpret_cast<uint32_t*>(gw + 128);
-                gcnt = ghist + 3 * NQ * 2048;
-            }
             int nloc[NQ];
             bool active[NQ];
             bool any_active = false;
@@ -625,183 +549,11 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                     }
                 }
             }
-            if (any_active) {
-                uint32_t prefix[NQ], kk[NQ];
-#pragma unroll
-                for (int j = 0; j < NQ; ++j) { prefix[j] = 0; kk[j] = (uint32_t)p.K; }
-                for (int pass = 0; pass < 3 && ok; ++pass) {
-                    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-                    const int nb = pass == 2 ? 1024 : 2048;
-                    if (pass > 0) {
-                        for (int i = threadIdx.x; i < Cfg::HIST_WORDS; i += kEpiThreads) s_hist[i] = 0u;
-                        named_bar_sync(1, kEpiThreads);
-                        const uint32_t pmask = 0xFFFFFFFFu << (shift + (pass == 1 ? 11 : 10));
-#pragma unroll
-                        for (int j = 0; j < NQ; ++j) {
-                            if (!active[j]) continue;
-                            const float* sj = s_score + j * stride;
-                            for (int i = threadIdx.x; i < nloc[j]; i += kEpiThreads) {
-                                const uint32_t key = order_key(sj[i]);
-                                if ((key & pmask) == prefix[j])
-                                    atomicAdd(&s_hist[j * 2048 + ((key >> shift) & (nb - 1))], 1u);
-                            }
-                        }
-                        named_bar_sync(1, kEpiThreads);
-                    }
-                    if (item.G > 1) {
-                        uint32_t* gh = ghist + pass * NQ * 2048;
-#pragma unroll
-                        for (int j = 0; j < NQ; ++j) {
-                            if (!active[j]) continue;
-                            for (int i = threadIdx.x; i < nb; i += kEpiThreads) {
-                                const uint32_t v = s_hist[j * 2048 + i];
-                                if (v) atomicAdd(gh + j * 2048 + i, v);
-                            }
-                        }
-                        if (!group_sync(gsync, item.G, p.status, abort)) { ok = false; break; }
-#pragma unroll
-                        for (int j = 0; j < NQ; ++j) {
-                            if (!active[j]) continue;
-                            for (int i = threadIdx.x; i < nb; i += kEpiThreads)
-                                s_hist[j * 2048 + i] = __ldcg(gh + j * 2048 + i);
-                        }
-                        // the histogram of the previous pass has been read by every CTA
-                        if (item.rank == 0 && pass > 0) {
-                            uint32_t* prev = ghist + (pass - 1) * NQ * 2048;
-                            for (int i = threadIdx.x; i < NQ * 2048; i += kEpiThreads) prev[i] = 0u;
-                        }
-                        named_bar_sync(1, kEpiThreads);
-                    }
-#pragma unroll
-                    for (int j = 0; j < NQ; ++j) {
-                        if (!active[j]) continue;
-                        find_bin(s_hist + j * 2048, nb, kk[j], m->scan, &m->sel_bin[j], &m->sel_kk[j]);
-                        prefix[j] |= m->sel_bin[j] << shift;
-                        kk[j] = m->sel_kk[j];
-                    }
-                    if (threadIdx.x == 0) DSA_TRACE_MARK(3 + pass);
-                }
-                if (!ok) break;
-                // counts above / equal to the threshold, per warp (warp w owns a
-                // contiguous quarter of the chunk, so warp order is position order)
-                uint32_t wgt[NQ], weq[NQ];
-#pragma unroll
-                for (int j = 0; j < NQ; ++j) {
-                    wgt[j] = weq[j] = 0;
-                    if (!active[j]) continue;
-                    const int qlen = ((nloc[j] + 4 * 32 - 1) / (4 * 32)) * 32;
-                    const int beg = warp * qlen, end = min(nloc[j], beg + qlen);
-                    const float* sj = s_score + j * stride;
-                    for (int i0 = beg; i0 < end; i0 += 32) {
-                        const int i = i0 + lane;
-                        const bool in = i < end;
-                        const uint32_t key = in ? order_key(sj[i]) : 0u;
-                        wgt[j] += __popc(__ballot_sync(0xffffffffu, in && key > prefix[j]));
-                        weq[j] += __popc(__ballot_sync(0xffffffffu, in && key == prefix[j]));
-                    }
-                    if (lane == 0) {
-                        m->wcnt[j][warp][0] = wgt[j];
-                        m->wcnt[j][warp][1] = weq[j];
-                    }
-                }
-                named_bar_sync(1, kEpiThreads);
-                uint32_t cgt[NQ], ceq[NQ], gt_before[NQ], eq_before[NQ];
-#pragma unroll
-                for (int j = 0; j < NQ; ++j) {
-                    cgt[j] = ceq[j] = gt_before[j] = eq_before[j] = 0;
-                    for (int w = 0; w < 4; ++w) {
-                        const uint32_t g = m->wcnt[j][w][0], e = m->wcnt[j][w][1];
-                        if (w < warp) { gt_before[j] += g; eq_before[j] += e; }
-                        cgt[j] += g;
-                        ceq[j] += e;
-                    }
-                }
-                uint32_t take[NQ], base[NQ];
-#pragma unroll
-                for (int j = 0; j < NQ; ++j) { take[j] = min(kk[j], ceq[j]); base[j] = 0; }
-                if (item.G > 1) {
-                    // split the tied elements (lowest positions first, i.e. lower
-                    // ranks first) and the output offsets across the group
-                    if (threadIdx.x == 0) {
-#pragma unroll
-                        for (int j = 0; j < NQ; ++j) {
-                            if (!active[j]) continue;
-                            __stcg(gcnt + (item.rank * NQ + j) * 2, cgt[j]);
-                            __stcg(gcnt + (item.rank * NQ + j) * 2 + 1, ceq[j]);
-                        }
-                    }
-                    if (!group_sync(gsync, item.G, p.status, abort)) break;
-                    if (threadIdx.x == 0) {
-#pragma unroll
-                        for (int j = 0; j < NQ; ++j) {
-                            if (!active[j]) continue;
-                            uint32_t eqb = 0, ob = 0;
-                            for (int r = 0; r < item.rank; ++r) {
-                                const uint32_t g_gt = __ldcg(gcnt + (r * NQ + j) * 2);
-                                const uint32_t g_eq = __ldcg(gcnt + (r * NQ + j) * 2 + 1);
-                                ob += g_gt + (kk[j] > eqb ? min(kk[j] - eqb, g_eq) : 0u);
-                                eqb += g_eq;
-                            }
-                            m->sel_take[j] = kk[j] > eqb ? min(kk[j] - eqb, ceq[j]) : 0u;
-                            m->sel_base[j] = ob;
-                        }
-                    }
-                    if (item.rank == 0) {
-                        // every CTA of the group has read the last pass's histogram
-                        uint32_t* last = ghist + 2 * NQ * 2048;
-                        for (int i = threadIdx.x; i < NQ * 2048; i += kEpiThreads) last[i] = 0u;
-                    }
-                    named_bar_sync(1, kEpiThreads);
-#pragma unroll
-                    for (int j = 0; j < NQ; ++j) {
-                        take[j] = m->sel_take[j];
-                        base[j] = m->sel_base[j];
-                    }
-                }
-                if (threadIdx.x == 0) DSA_TRACE_MARK(6);
-                // this warp's share of the tied elements
-                uint32_t allow[NQ];
-#pragma unroll
-                for (int j = 0; j < NQ; ++j) {
-                    allow[j] = take[j] > eq_before[j] ? min(take[j] - eq_before[j], weq[j]) : 0u;
-                    if (lane == 0) m->wallow[j][warp] = allow[j];
-                }
-                named_bar_sync(1, kEpiThreads);
-                const uint32_t lt_mask = (1u << lane) - 1u;
-#pragma unroll
-                for (int j = 0; j < NQ; ++j) {
-                    if (!active[j]) continue;
-                    uint32_t out = base[j] + gt_before[j];
-                    for (int w = 0; w < warp; ++w) out += m->wallow[j][w];
-                    const int qlen = ((nloc[j] + 4 * 32 - 1) / (4 * 32)) * 32;
-                    const int beg = warp * qlen, end = min(nloc[j], beg + qlen);
-                    const float* sj = s_score + j * stride;
-                    const int64_t tok = item.t0 + j;
-                    int32_t* oi = p.out_idx + tok * p.K;
-                    float* os = p.out_score ? p.out_score + tok * p.K : nullptr;
-                    uint32_t eq_seen = 0;
-                    for (int i0 = beg; i0 < end; i0 += 32) {
-                        const int i = i0 + lane;
-                        const bool in = i < end;
-                        const float f = in ? sj[i] : 0.0f;
-                        const uint32_t key = in ? order_key(f) : 0u;
-                        const bool is_gt = in && key > prefix[j];
-                        const bool is_eq = in && key == prefix[j];
-                        const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
-                        const bool sel = is_gt || (is_eq && eq_seen + __popc(eqm & lt_mask) < allow[j]);
-                        const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-                        if (sel) {
-                            const uint32_t o = out + __popc(selm & lt_mask);
-                            if (o < (uint32_t)p.K) {
-                                oi[o] = (int32_t)(chunk0 + i);
-                                if (os) os[o] = f;
-                            }
-                        }
-                        out += __popc(selm);
-                        eq_seen += __popc(eqm);
-                    }
-                }
-                named_bar_sync(1, kEpiThreads);
+            if (any_active &&
+                !topk_select<NQ>(p, gv, gen, s_score, stride, nloc, active, chunk0, item.t0, s_hist, s_list, &m->sel,
+                                 abort)) {
+                ok = false;
+                break;
             }
             if (threadIdx.x == 0) DSA_TRACE_MARK(7);
         }

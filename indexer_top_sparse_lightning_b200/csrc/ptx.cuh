@@ -28,13 +28,21 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // each CTA's life into a device table read back by dsa_trace_read().
 #ifdef DSA_TRACE
 __device__ uint64_t g_dsa_trace[2048][16];
+__device__ uint64_t g_dsa_trace_blk[64][16];  // CTA 0 only: per-block events
 #define DSA_TRACE_MARK(slot)                                                     \
     do {                                                                         \
         if (blockIdx.x < 2048) g_dsa_trace[blockIdx.x][(slot)] = globaltimer(); \
     } while (0)
+#define DSA_TRACE_BLK(jb, ev)                                                          \
+    do {                                                                               \
+        if (blockIdx.x == 0 && (jb) < 64) g_dsa_trace_blk[(jb)][(ev)] = globaltimer(); \
+    } while (0)
 #else
 #define DSA_TRACE_MARK(slot) \
     do {                     \
+    } while (0)
+#define DSA_TRACE_BLK(jb, ev) \
+    do {                      \
     } while (0)
 #endif
 

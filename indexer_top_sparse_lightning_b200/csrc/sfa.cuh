@@ -15,23 +15,25 @@
 //   CTA 0 holds elements [0,256) and [512,576) of every row,
 //   CTA 1 holds elements [256,512).
 // Each CTA gathers only its bytes of each selected row (16-byte cp.async
-// vector loads into 128-byte-swizzled shared memory), computes the partial
-// logits S_c = Q_c . K_c^T on tcgen05 (M=128 heads, N=64 rows), and the two
-// partial logit tiles are exchanged through distributed shared memory, so
-// both CTAs hold the same full S (fp32 add is commutative, so both get the
-// same bits) and make the same online-softmax decisions.  Each CTA then
-// accumulates its 256-wide half of O = P . V in tensor memory (M=128, N=256,
-// V read MN-major straight from the gathered rows).  No logit is computed
-// twice and no row byte is fetched twice.
+// vector loads into 128-byte-swizzled shared memory, rows prefetched into L2
+// two blocks ahead), computes the partial logits S_c = Q_c . K_c^T on
+// tcgen05 (M=128 heads, N=64 rows), and the two partial logit tiles are
+// exchanged through distributed shared memory, so both CTAs hold the same
+// full S (fp32 add is commutative, so both get the same bits) and make the
+// same online-softmax decisions.  Each CTA then accumulates its 256-wide half
+// of O = P . V in tensor memory (M=128, N=256, V read MN-major straight from
+// the gathered rows).  No logit is computed twice and no row byte is fetched
+// twice.
 //
-// Gather completion is signalled with cp.async.mbarrier.arrive.noinc, so each
-// stage's barrier fires as soon as its own rows land.
 // Roles per CTA: warps 0-3 softmax (thread h <-> head h <-> TMEM lane h),
-// warps 4-7 row gather, warp 8 TMEM allocation and MMA issue.
-// The running max uses a lazy rescale: O and l are rescaled only when the max
-// grows by more than 2^8, otherwise the old reference max is kept.
-// With several row splits per token, un-normalised partial O and (m, l) go to
-// the workspace and a small combine kernel merges them.
+// warps 4-6 row gather, warp 7 TMEM allocation and MMA issue.  The MMA warp
+// issues whichever of the next logit tile and the pending P.V product is
+// ready first.  The running max uses a lazy rescale: O and l are rescaled
+// only when the max grows by more than 2^8.
+// With several row splits per token, each CTA writes an un-normalised
+// partial O and (m, l); the last CTA of a (token, half) to finish merges the
+// partials of all splits (arrival counted with a global atomic), so no
+// separate combine launch is needed.
 #pragma once
 #include "common.h"
 #include "ptx.cuh"
@@ -40,7 +42,8 @@ namespace dsa {
 
 struct SfaCfg {
     static constexpr int ROWS = 64;                     // selected rows per block
-    static constexpr int NS = 2;                        // gather stages
+    static constexpr int NS = 2;                        // gather stages in shared memory
+    static constexpr int PF = 2;                        // blocks prefetched into L2 ahead of the gather
     static constexpr int KBQ0 = 5, KBQ1 = 4;            // 64-wide K blocks held by CTA 0 / CTA 1
     static constexpr int KBMAX = 5;
     static constexpr int Q_BYTES = KBMAX * 128 * 128;   // [128 heads x 64] per K block
@@ -58,7 +61,8 @@ struct SfaCfg {
     static constexpr int OFF_ROWS = OFF_MISC + MISC_BYTES;
     static constexpr int OFF_VALID = OFF_ROWS + MAX_ROWS * 4;
     static constexpr int SMEM = 1024 + OFF_VALID + MAX_ROWS / 8;
-    static constexpr int THREADS = 288;
+    static constexpr int THREADS = 256;                   // 8 warps: the register file allows 255 per thread
+    static constexpr int GATHER = 96;                   // threads of warps 4-6
     static constexpr int TMEM_COLS = 512;               // O: [0,256), S buffers: [256,320), [320,384)
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, ROWS, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 256, false, true);
@@ -73,12 +77,13 @@ struct SfaMisc {
     uint64_t p_full;
     uint64_t p_empty;
     uint64_t o_full;
-    uint64_t x_full;    // peer's partial logits have landed in my X buffer
-    uint64_t x_free;    // peer has consumed the logits I wrote into its X buffer
+    uint64_t x_full;       // peer's partial logits have landed in my X buffer
+    uint64_t x_free;       // peer has consumed the logits I wrote into its X buffer
     uint64_t drain;
     uint64_t rows_ready;   // physical rows and validity bits of the split are in shared memory
     uint32_t tmem_base;
     int abort;
+    int last;              // this CTA merges the split partials of its (token, half)
 };
 
 __device__ __forceinline__ int token_sequence(const int32_t* cu_q, int B, int t) {
@@ -88,6 +93,15 @@ __device__ __forceinline__ int token_sequence(const int32_t* cu_q, int B, int t)
         if (__ldg(cu_q + mid) <= t) lo = mid; else hi = mid - 1;
     }
     return lo;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
@@ -118,7 +132,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(&m->q_full, 1);
         for (int i = 0; i < Cfg::NS; ++i) {
-            mbar_init(&m->kv_full[i], 128);
+            mbar_init(&m->kv_full[i], Cfg::GATHER);
             mbar_init(&m->kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -131,11 +145,12 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         mbar_init(&m->x_full, 128);
         mbar_init(&m->x_free, 128);
         mbar_init(&m->drain, 1);
-        mbar_init(&m->rows_ready, 128);
+        mbar_init(&m->rows_ready, Cfg::GATHER);
         m->abort = 0;
+        m->last = 0;
         fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == 7) {
         tmem_alloc(&m->tmem_base, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
@@ -153,7 +168,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     const uint32_t tm_s = tmem_base + 256;      // two 64-column logit buffers
     if (threadIdx.x == 0) DSA_TRACE_MARK(0);
 
-    if (warp == 8) {
+    if (warp == 7) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             bool ok = true;
@@ -167,28 +182,34 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             tc_fence_after();
             const uint32_t q_addr = smem_u32(s_q);
             const uint32_t p_addr = smem_u32(s_p);
-            auto issue_qk = [&](int jb) -> bool {
+            // readiness of the two kinds of work, polled without blocking
+            auto qk_ready = [&](int jb) -> bool {
+                return mbar_try_wait(smem_u32(&m->kv_full[jb % Cfg::NS]), (jb / Cfg::NS) & 1) &&
+                       mbar_try_wait(smem_u32(&m->s_empty[jb & 1]), ((jb >> 1) & 1) ^ 1);
+            };
+            auto pv_ready = [&](int jb) -> bool { return mbar_try_wait(smem_u32(&m->p_full), jb & 1); };
+            auto issue_qk = [&](int jb) {
                 const int s = jb % Cfg::NS, sb = jb & 1;
-                if (!mbar_wait(&m->kv_full[s], (jb / Cfg::NS) & 1, abort)) return false;
+                DSA_TRACE_BLK(jb, 6);
                 // rows were written by cp.async (generic proxy); the MMA reads them through the async proxy
                 fence_proxy_async_smem();
-                if (!mbar_wait(&m->s_empty[sb], ((jb >> 1) & 1) ^ 1, abort)) return false;
                 tc_fence_after();
                 const uint32_t kv_addr = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
                 for (int kb = 0; kb < kbq; ++kb)
+#pragma unroll
                     for (int k16 = 0; k16 < 4; ++k16)
                         umma_bf16(tm_s + sb * Cfg::ROWS,
                                   sdesc_sw128(q_addr + kb * 16384 + k16 * 32, 16, 1024),
                                   sdesc_sw128(kv_addr + kb * Cfg::KV_KB_BYTES + k16 * 32, 16, 1024),
                                   Cfg::IDESC_QK, (kb | k16) != 0);
                 umma_commit(&m->s_full[sb]);
-                return true;
             };
-            auto issue_pv = [&](int jb) -> bool {
+            auto issue_pv = [&](int jb) {
                 const int s = jb % Cfg::NS;
-                if (!mbar_wait(&m->p_full, jb & 1, abort)) return false;
+                DSA_TRACE_BLK(jb, 7);
                 tc_fence_after();
                 const uint32_t kv_addr = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
+#pragma unroll
                 for (int k16 = 0; k16 < 4; ++k16)
                     // A = P [128 heads x 64 rows] K-major; B = V [64 rows x 256 dims] MN-major:
                     // 64-dim groups are K blocks (LBO apart), 8-row groups 1024 B apart (SBO).
@@ -197,12 +218,28 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                               Cfg::IDESC_PV, (jb > 0 || k16 > 0));
                 umma_commit(&m->kv_empty[s]);
                 umma_commit(&m->p_empty);
-                return true;
             };
-            if (ok && nblk > 0) ok = issue_qk(0);
-            for (int jb = 0; ok && jb < nblk; ++jb) {
-                if (jb + 1 < nblk && !issue_qk(jb + 1)) { ok = false; break; }
-                if (!issue_pv(jb)) { ok = false; break; }
+            // QK(j) may run up to two blocks ahead of PV(j) (two logit buffers)
+            int next_qk = 0, next_pv = 0;
+            uint64_t t_idle = 0;
+            while (ok && next_pv < nblk) {
+                bool progressed = false;
+                if (next_qk < nblk && next_qk <= next_pv + 1 && qk_ready(next_qk)) {
+                    issue_qk(next_qk++);
+                    progressed = true;
+                } else if (next_pv < next_qk && pv_ready(next_pv)) {
+                    issue_pv(next_pv++);
+                    progressed = true;
+                }
+                if (progressed) {
+                    t_idle = 0;
+                } else if (*abort) {
+                    ok = false;
+                } else {
+                    const uint64_t now = globaltimer();
+                    if (t_idle == 0) t_idle = now;
+                    else if (now - t_idle > kWaitTimeoutNs) ok = false;
+                }
             }
             umma_commit(&m->o_full);
             umma_commit(&m->drain);
@@ -212,50 +249,84 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         }
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- row gather
-        const int pt = threadIdx.x - 128;           // 0..127
+        const int pt = threadIdx.x - 128;           // 0..GATHER-1
         const int b = token_sequence(p.cu_q, p.B, t);
         const int64_t L = __ldg(p.seq_lens + b);
-        const int nch = kbq * 8;                    // 16-byte chunks per row held by this CTA
+        const int gw = pt >> 5;                      // gather warp 0..2
+        const uint32_t lane_q = (uint32_t)(lane & 7);
+        const uint32_t lane_kb_off = (uint32_t)(lane >> 3) * Cfg::KV_KB_BYTES;
+        const int lane_byte = (crank == 0 ? 0 : 512) + lane * 16;
         const int32_t* idx_t = p.idx + (int64_t)t * p.K;
         const uint8_t* kv_bytes = reinterpret_cast<const uint8_t*>(p.kv);
-        // physical row of every selected position of this split, and validity bits, once
+        // physical row of every selected position of this split and its validity bit,
+        // computed once with all loads of a thread in flight together
         const int nrows = nblk * Cfg::ROWS;
-        for (int i = pt; i < nrows; i += 128) {
-            const int r = row_begin + i;
-            int32_t row = -1;
-            if (r < row_end) {
-                const int32_t pos = __ldg(idx_t + r);
-                if (pos >= 0) {
-                    if (pos < L && pos / kPage < p.max_blocks) {
-                        const int blk = __ldg(p.block_table + (int64_t)b * p.max_blocks + pos / kPage);
-                        if (blk >= 0 && blk < p.num_blocks)
-                            row = blk * kPage + pos % kPage;
-                        else
-                            atomicCAS(p.status, 0u, (uint32_t)kStBounds);
-                    } else {
-                        atomicCAS(p.status, 0u, (uint32_t)kStBounds);
-                    }
-                }
+        constexpr int RPT = (Cfg::MAX_ROWS + Cfg::GATHER - 1) / Cfg::GATHER;
+        int32_t pos[RPT], blk[RPT];
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const int i = pt + k * Cfg::GATHER;
+            pos[k] = (i < nrows && row_begin + i < row_end) ? __ldg(idx_t + row_begin + i) : -1;
+        }
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            blk[k] = -1;
+            if (pos[k] >= 0) {
+                if (pos[k] < L && pos[k] / kPage < p.max_blocks)
+                    blk[k] = __ldg(p.block_table + (int64_t)b * p.max_blocks + pos[k] / kPage);
+                else
+                    atomicCAS(p.status, 0u, (uint32_t)kStBounds);
             }
-            s_rows[i] = row;
-            const uint32_t bits = __ballot_sync(0xffffffffu, row >= 0);
-            if ((i & 31) == 0) s_valid[i >> 5] = bits;
+        }
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const int i = pt + k * Cfg::GATHER;
+            if (i < nrows) {                           // uniform per warp (nrows is a multiple of 32)
+                int32_t row = -1;
+                if (blk[k] >= 0 && blk[k] < p.num_blocks) row = blk[k] * kPage + pos[k] % kPage;
+                else if (pos[k] >= 0 && blk[k] != -1) atomicCAS(p.status, 0u, (uint32_t)kStBounds);
+                s_rows[i] = row;
+                const uint32_t bits = __ballot_sync(0xffffffffu, row >= 0);
+                if (lane == 0) s_valid[i >> 5] = bits;
+            }
         }
         mbar_arrive(&m->rows_ready);
         if (pt == 0) DSA_TRACE_MARK(1);
-        named_bar_sync(2, 128);
+        named_bar_sync(2, Cfg::GATHER);
+        // L2 prefetch of the first blocks' rows (this CTA's part of each row)
+        auto prefetch_block = [&](int jb) {
+            if (jb < nblk && pt < Cfg::ROWS) {
+                const int32_t row = s_rows[jb * Cfg::ROWS + pt];
+                if (row >= 0) {
+                    const uint8_t* r = kv_bytes + (int64_t)row * (kDqk * 2);
+                    if (crank == 0) {
+                        prefetch_l2(r, 512);
+                        prefetch_l2(r + 1024, 128);
+                    } else {
+                        prefetch_l2(r + 512, 512);
+                    }
+                }
+            }
+        };
+        for (int jb = 0; jb < Cfg::PF; ++jb) prefetch_block(jb);
         for (int jb = 0; jb < nblk; ++jb) {
             const int s = jb % Cfg::NS;
+            prefetch_block(jb + Cfg::PF);
             if (!mbar_wait(&m->kv_empty[s], ((jb / Cfg::NS) & 1) ^ 1, abort)) break;
+            if (pt == 0) DSA_TRACE_BLK(jb, 5);
             const uint32_t st = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
             const int32_t* rows = s_rows + jb * Cfg::ROWS;
-            for (int e = pt; e < Cfg::ROWS * nch; e += 128) {
-                const int r = e / nch, ch = e % nch;
-                const int kb = ch >> 3, q = ch & 7;
-                const int byte = crank == 0 ? (kb < 4 ? kb * 128 + q * 16 : 1024 + q * 16) : 512 + kb * 128 + q * 16;
+            // one warp per row: lane l copies 16 bytes of the row's 256 latent elements
+            // (one coalesced 512-byte read), lanes 0-7 of CTA 0 also the 64 RoPE elements
+            for (int r = gw; r < Cfg::ROWS; r += Cfg::GATHER / 32) {
                 const int32_t row = rows[r];
-                const void* src = kv_bytes + (row >= 0 ? (int64_t)row * (kDqk * 2) + byte : 0);
-                cp_async_16(st + kb * Cfg::KV_KB_BYTES + r * 128 + ((q ^ (r & 7)) << 4), src, row >= 0);
+                const bool ok_row = row >= 0;
+                const uint8_t* src_row = kv_bytes + (ok_row ? (int64_t)row * (kDqk * 2) : 0);
+                const uint32_t dst_row = st + r * 128;
+                const uint32_t sw = (uint32_t)(r & 7);
+                cp_async_16(dst_row + lane_kb_off + ((lane_q ^ sw) << 4), src_row + lane_byte, ok_row);
+                if (crank == 0 && lane < 8)
+                    cp_async_16(dst_row + 4 * Cfg::KV_KB_BYTES + ((lane_q ^ sw) << 4), src_row + 1024 + lane * 16, ok_row);
             }
             // the barrier receives this thread's arrival once its copies have landed
             cp_async_arrive_noinc(&m->kv_full[s]);
@@ -268,14 +339,16 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         const uint32_t x_full_peer = mapa_shared(smem_u32(&m->x_full), peer);
         const uint32_t x_free_peer = mapa_shared(smem_u32(&m->x_free), peer);
         const uint32_t x_peer_row = mapa_shared(smem_u32(s_x + h * Cfg::ROWS), peer);
+        const float* xrow = s_x + h * Cfg::ROWS;
         float mrun = -INFINITY, lrun = 0.0f;
         bool ok = nblk == 0 || mbar_wait(&m->rows_ready, 0, abort);
         for (int jb = 0; ok && jb < nblk; ++jb) {
             const int sb = jb & 1;
             // validity of the 64 rows of this block (same for every head)
-            const uint32_t vmask[2] = {s_valid[jb * 2], s_valid[jb * 2 + 1]};
+            const uint32_t v0 = s_valid[jb * 2], v1 = s_valid[jb * 2 + 1];
             if (!mbar_wait(&m->s_full[sb], (jb >> 1) & 1, abort)) { ok = false; break; }
             if (jb == 0 && h == 0) DSA_TRACE_MARK(2);
+            if (h == 0) DSA_TRACE_BLK(jb, 0);
             tc_fence_after();
             uint32_t a[32], c[32];
             tmem_ld32(tm_s + lane_off + sb * Cfg::ROWS, a);
@@ -285,53 +358,71 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             mbar_arrive(&m->s_empty[sb]);
             // exchange partial logits with the peer CTA
             if (!mbar_wait_cluster(&m->x_free, (jb & 1) ^ 1, abort)) { ok = false; break; }
+            if (h == 0) DSA_TRACE_BLK(jb, 1);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const uint32_t* src = q < 8 ? a : c;
-                const int o = (q & 7) * 4;
-                st_cluster_v4(x_peer_row + (uint32_t)(((q ^ (h & 15)) << 4)),
-                              __uint_as_float(src[o]), __uint_as_float(src[o + 1]),
-                              __uint_as_float(src[o + 2]), __uint_as_float(src[o + 3]));
-            }
+            for (int q = 0; q < 8; ++q)
+                st_cluster_v4(x_peer_row + (uint32_t)((q ^ (h & 15)) << 4), __uint_as_float(a[4 * q]),
+                              __uint_as_float(a[4 * q + 1]), __uint_as_float(a[4 * q + 2]),
+                              __uint_as_float(a[4 * q + 3]));
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                st_cluster_v4(x_peer_row + (uint32_t)(((q + 8) ^ (h & 15)) << 4), __uint_as_float(c[4 * q]),
+                              __uint_as_float(c[4 * q + 1]), __uint_as_float(c[4 * q + 2]),
+                              __uint_as_float(c[4 * q + 3]));
             mbar_arrive_remote(x_full_peer);
+            if (h == 0) DSA_TRACE_BLK(jb, 8);
             if (!mbar_wait_cluster(&m->x_full, jb & 1, abort)) { ok = false; break; }
+            if (h == 0) DSA_TRACE_BLK(jb, 2);
             float sv[64];
-            const float* xrow = s_x + h * Cfg::ROWS;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
+            for (int q = 0; q < 8; ++q) {
                 const float4 v = *reinterpret_cast<const float4*>(xrow + ((q ^ (h & 15)) << 2));
-                const uint32_t* src = q < 8 ? a : c;
-                const int o = (q & 7) * 4;
-                sv[q * 4 + 0] = __uint_as_float(src[o + 0]) + v.x;
-                sv[q * 4 + 1] = __uint_as_float(src[o + 1]) + v.y;
-                sv[q * 4 + 2] = __uint_as_float(src[o + 2]) + v.z;
-                sv[q * 4 + 3] = __uint_as_float(src[o + 3]) + v.w;
+                sv[4 * q + 0] = __uint_as_float(a[4 * q + 0]) + v.x;
+                sv[4 * q + 1] = __uint_as_float(a[4 * q + 1]) + v.y;
+                sv[4 * q + 2] = __uint_as_float(a[4 * q + 2]) + v.z;
+                sv[4 * q + 3] = __uint_as_float(a[4 * q + 3]) + v.w;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 v = *reinterpret_cast<const float4*>(xrow + (((q + 8) ^ (h & 15)) << 2));
+                sv[32 + 4 * q + 0] = __uint_as_float(c[4 * q + 0]) + v.x;
+                sv[32 + 4 * q + 1] = __uint_as_float(c[4 * q + 1]) + v.y;
+                sv[32 + 4 * q + 2] = __uint_as_float(c[4 * q + 2]) + v.z;
+                sv[32 + 4 * q + 3] = __uint_as_float(c[4 * q + 3]) + v.w;
             }
             mbar_arrive_remote(x_free_peer);
+            if (h == 0) DSA_TRACE_BLK(jb, 9);
             // online softmax in the log2 domain
-            float mx = -INFINITY;
+            float mxs[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mxs[u] = -INFINITY;
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
-                const bool v = (vmask[i >> 5] >> (i & 31)) & 1u;
-                sv[i] = v ? sv[i] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, sv[i]);
+                const uint32_t vw = i < 32 ? v0 : v1;
+                sv[i] = ((vw >> (i & 31)) & 1u) ? sv[i] * p.scale_log2 : -INFINITY;
+                mxs[i & 7] = fmaxf(mxs[i & 7], sv[i]);   // eight independent chains
             }
+            const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                                   fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
             const float mnew = fmaxf(mrun, mx);
             const bool rescale = mnew > mrun + 8.0f;
             const float muse = rescale ? mnew : mrun;
+            const bool none = muse == -INFINITY;
             uint32_t pk[32];
-            float rs = 0.0f;
+            float rss[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float p0 = muse == -INFINITY ? 0.0f : exp2f(sv[2 * i] - muse);
-                const float p1 = muse == -INFINITY ? 0.0f : exp2f(sv[2 * i + 1] - muse);
-                const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                const float2 pr = __bfloat1622float2(pb);
-                rs += pr.x + pr.y;
-                pk[i] = *reinterpret_cast<const uint32_t*>(&pb);
+                const float p0 = none ? 0.0f : exp2f(sv[2 * i] - muse);
+                const float p1 = none ? 0.0f : exp2f(sv[2 * i + 1] - muse);
+                pk[i] = pack_bf16(p0, p1);
+                // the row sum uses the bf16-rounded weights the MMA multiplies with
+                rss[i & 3] += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xFFFF0000u);
             }
+            const float rs = (rss[0] + rss[1]) + (rss[2] + rss[3]);
+            if (h == 0) DSA_TRACE_BLK(jb, 10);
             // P buffer free and O stable once the previous P.V has completed
             if (!mbar_wait(&m->p_empty, (jb & 1) ^ 1, abort)) { ok = false; break; }
+            if (h == 0) DSA_TRACE_BLK(jb, 3);
             tc_fence_after();
             if (rescale && jb > 0) {
                 const float f = exp2f(mrun - muse);
@@ -358,6 +449,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&m->p_full);
+            if (h == 0) DSA_TRACE_BLK(jb, 4);
         }
         // ---------------------------------------------------------------- epilogue
         if (h == 0) DSA_TRACE_MARK(3);
@@ -365,32 +457,32 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             if (h == 0) DSA_TRACE_MARK(4);
             tc_fence_after();
             const int dim0 = crank == 0 ? 0 : 256;
+            const bool empty = !(lrun > 0.0f);   // nothing selected: O was never written
             if (p.n_splits == 1) {
-                const float inv = lrun > 0.0f ? 1.0f / lrun : 0.0f;
+                const float inv = empty ? 0.0f : 1.0f / lrun;
                 for (int c0 = 0; c0 < 256; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tm_o + lane_off + c0, o);
                     tmem_wait_ld();
-                    if (!(lrun > 0.0f))   // nothing selected: O was never written
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = 0u;
                     if (h < p.H) {
                         uint16_t* dst = p.out + ((int64_t)t * p.H + h) * kDv + dim0 + c0;
 #pragma unroll
                         for (int i = 0; i < 32; i += 8) {
-                            uint32_t w4[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[i + 2 * e]) * inv,
-                                                                               __uint_as_float(o[i + 2 * e + 1]) * inv);
-                                w4[e] = *reinterpret_cast<const uint32_t*>(&v);
-                            }
-                            *reinterpret_cast<uint4*>(dst + i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            const float f0 = empty ? 0.f : __uint_as_float(o[i]) * inv;
+                            const float f1 = empty ? 0.f : __uint_as_float(o[i + 1]) * inv;
+                            const float f2 = empty ? 0.f : __uint_as_float(o[i + 2]) * inv;
+                            const float f3 = empty ? 0.f : __uint_as_float(o[i + 3]) * inv;
+                            const float f4 = empty ? 0.f : __uint_as_float(o[i + 4]) * inv;
+                            const float f5 = empty ? 0.f : __uint_as_float(o[i + 5]) * inv;
+                            const float f6 = empty ? 0.f : __uint_as_float(o[i + 6]) * inv;
+                            const float f7 = empty ? 0.f : __uint_as_float(o[i + 7]) * inv;
+                            *reinterpret_cast<uint4*>(dst + i) =
+                                make_uint4(pack_bf16(f0, f1), pack_bf16(f2, f3), pack_bf16(f4, f5), pack_bf16(f6, f7));
                         }
                     }
                 }
                 if (crank == 0 && h < p.H && p.lse)
-                    p.lse[(int64_t)t * p.H + h] = lrun > 0.0f ? (mrun + log2f(lrun)) * 0.69314718055994531f : -INFINITY;
+                    p.lse[(int64_t)t * p.H + h] = empty ? -INFINITY : (mrun + log2f(lrun)) * 0.69314718055994531f;
             } else {
                 // un-normalised partial: [t][split][dim chunk of 4][head][4]
                 float* po = p.part_o + (((int64_t)t * p.n_splits + split) * 128) * 128 * 4;
@@ -398,22 +490,27 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                     uint32_t o[32];
                     tmem_ld32(tm_o + lane_off + c0, o);
                     tmem_wait_ld();
-                    if (!(lrun > 0.0f))
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = 0u;
 #pragma unroll
                     for (int i = 0; i < 32; i += 4) {
                         const int chunk = (dim0 + c0 + i) >> 2;
-                        *reinterpret_cast<float4*>(po + ((int64_t)chunk * 128 + h) * 4) =
-                            make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]),
-                                        __uint_as_float(o[i + 2]), __uint_as_float(o[i + 3]));
+                        float4 v = make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]),
+                                               __uint_as_float(o[i + 2]), __uint_as_float(o[i + 3]));
+                        if (empty) v = make_float4(0.f, 0.f, 0.f, 0.f);
+                        *reinterpret_cast<float4*>(po + ((int64_t)chunk * 128 + h) * 4) = v;
                     }
                 }
-                if (crank == 0) {
-                    float* ml = p.part_ml + ((int64_t)t * p.n_splits + split) * 256;
-                    ml[h] = mrun;
-                    ml[128 + h] = lrun;
+                // (m, l) of this split, one copy per half so each half's merger reads its own
+                float* ml = p.part_ml + (((int64_t)t * p.n_splits + split) * 2 + crank) * 256;
+                ml[h] = mrun;
+                ml[128 + h] = lrun;
+                // the last CTA of this (token, half) to get here merges all splits
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (h == 0) {
+                    const uint32_t prev = atomicAdd(p.split_count + (int64_t)t * 2 + crank, 1u);
+                    m->last = prev == (uint32_t)p.n_splits - 1u;
                 }
+                named_bar_sync(1, 128);
             }
         }
         if (!ok) *abort = 1;
@@ -422,48 +519,58 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
+    if (p.n_splits > 1 && m->last && !m->abort) {
+        // merge the splits of this (token, half): weights 2^(m_s - M) per head
+        // (in the now idle exchange buffer), then every thread folds (head,
+        // 4-dim chunk) pairs, loads coalesced across heads
+        __threadfence();
+        const int S = p.n_splits;
+        const int dim0 = crank == 0 ? 0 : 256;
+        float* wsm = s_x;                  // [S][128]
+        float* linv = s_x + 32 * 128;      // [128]
+        for (int h = threadIdx.x; h < 128; h += Cfg::THREADS) {
+            float M = -INFINITY;
+            for (int s = 0; s < S; ++s)
+                M = fmaxf(M, __ldcg(p.part_ml + (((int64_t)t * S + s) * 2 + crank) * 256 + h));
+            float Lsum = 0.0f;
+            for (int s = 0; s < S; ++s) {
+                const float* mls = p.part_ml + (((int64_t)t * S + s) * 2 + crank) * 256;
+                const float ms = __ldcg(mls + h);
+                const float w = ms == -INFINITY ? 0.0f : exp2f(ms - M);
+                wsm[s * 128 + h] = w;
+                Lsum += w * __ldcg(mls + 128 + h);
+            }
+            linv[h] = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+            if (crank == 0 && h < p.H && p.lse)
+                p.lse[(int64_t)t * p.H + h] = Lsum > 0.0f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < 128 * 64; e += Cfg::THREADS) {
+            const int h = e & 127, chunk = (dim0 >> 2) + (e >> 7);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s = 0; s < S; ++s) {
+                const float ws = wsm[s * 128 + h];
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                    p.part_o + ((((int64_t)t * S + s) * 128 + chunk) * 128 + h) * 4));
+                acc.x += ws * v.x;
+                acc.y += ws * v.y;
+                acc.z += ws * v.z;
+                acc.w += ws * v.w;
+            }
+            const float inv = linv[h];
+            if (h < p.H)
+                *reinterpret_cast<uint2*>(p.out + ((int64_t)t * p.H + h) * kDv + chunk * 4) =
+                    make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+        }
+        if (threadIdx.x == 0) p.split_count[(int64_t)t * 2 + crank] = 0u;   // ready for the next call
+    }
     cluster_sync();   // no remote access may target an exited CTA
-    if (warp == 8) {
+    if (warp == 7) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
     if (threadIdx.x == 0 && m->abort) atomicCAS(p.status, 0u, (uint32_t)kStTimeout);
     if (threadIdx.x == 0) DSA_TRACE_MARK(9);
-}
-
-// Merge the row-split partials of each (token, head): weights 2^(m_s - M).
-__global__ void __launch_bounds__(256) sfa_combine_kernel(const __grid_constant__ SfaParams p) {
-    const int t = blockIdx.x / 64;
-    const int sub = blockIdx.x % 64;
-    const int pair = sub * 256 + threadIdx.x;      // (chunk, head) pair, 128 x 128
-    const int chunk = pair / 128, h = pair % 128;
-    const int S = p.n_splits;
-    const float* ml = p.part_ml + (int64_t)t * S * 256;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, ml[s * 256 + h]);
-    float Lsum = 0.0f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < S; ++s) {
-        const float ms = ml[s * 256 + h];
-        const float wgt = ms == -INFINITY ? 0.0f : exp2f(ms - M);
-        Lsum += wgt * ml[s * 256 + 128 + h];
-        const float4 v = *reinterpret_cast<const float4*>(
-            p.part_o + ((((int64_t)t * S + s) * 128 + chunk) * 128 + h) * 4);
-        acc.x += wgt * v.x;
-        acc.y += wgt * v.y;
-        acc.z += wgt * v.z;
-        acc.w += wgt * v.w;
-    }
-    if (h >= p.H) return;
-    const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    uint2 pk;
-    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(p.out + ((int64_t)t * p.H + h) * kDv + chunk * 4) = pk;
-    if (chunk == 0 && p.lse)
-        p.lse[(int64_t)t * p.H + h] = Lsum > 0.0f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace dsa
