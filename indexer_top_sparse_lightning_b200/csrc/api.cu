@@ -323,7 +323,8 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     CUtensorMap tm_q;
     const uint64_t dims[3] = {(uint64_t)kDqk, (uint64_t)at->H, (uint64_t)bt->num_tokens};
     const uint64_t strides[2] = {(uint64_t)kDqk * 2, (uint64_t)at->H * kDqk * 2};
-    const uint32_t box[3] = {64, (uint32_t)at->H, 1};
+    // each CTA of a pair loads its own 64 heads (heads past H read as zeros)
+    const uint32_t box[3] = {64, (uint32_t)(at->H < 64 ? at->H : 64), 1};
     if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, at->q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return DSA_ERR_CUDA;
     if (cudaFuncSetAttribute(&sfa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfaCfg::SMEM) !=

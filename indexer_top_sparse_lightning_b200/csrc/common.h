@@ -72,7 +72,7 @@ struct SfaParams {
     const int32_t* idx;       // [T, K]
     uint16_t* out;            // [T, H, 512] bf16 bits
     float* lse;               // [T, H] or null
-    float* part_o;            // split partials: [T, S, 128 chunks of 4 dims, 128 heads, 4]
+    float* part_o;            // split partials: [T, S, 128 heads, 512] (un-normalised)
     float* part_ml;           // [T, S, 2 halves, 2, 128] (m in log2 domain, l)
     uint32_t* split_count;    // [T, 2 halves] arrivals; zero between calls
     uint32_t* status;
