@@ -180,6 +180,14 @@ DSA_API int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexe
 /* Static description of a status code. */
 DSA_API const char* dsa_status_str(int32_t status);
 
+/*
+ * Text of the last failure an entry point recorded on the calling host thread
+ * (the CUDA call and its error name for DSA_ERR_CUDA), or "" if none.  The
+ * string is owned by the library and stays valid until the next call on that
+ * thread.
+ */
+DSA_API const char* dsa_last_error(void);
+
 /* Library version string. */
 DSA_API const char* dsa_version(void);
 

@@ -32,10 +32,14 @@ KEY_BF16 = 0
 KEY_FP8_E4M3 = 1
 
 
+DSA_ERR_CUDA = 4   # dsa_status code of a failed CUDA runtime / driver call
+
+
 class DsaError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = int(code)
-        super().__init__(f"{where}: {status_str(code)} (code {code})")
+        detail = last_error() if self.code == DSA_ERR_CUDA else ""
+        super().__init__(f"{where}: {status_str(code)} (code {code})" + (f": {detail}" if detail else ""))
 
 
 class _Batch(ctypes.Structure):
@@ -90,12 +94,18 @@ def load_library():
     lib.dsa_status_str.argtypes = [ctypes.c_int32]
     lib.dsa_status_str.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
+    lib.dsa_last_error.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
 
 def status_str(code: int) -> str:
     return load_library().dsa_status_str(int(code)).decode()
+
+
+def last_error() -> str:
+    """Text of the last failure the library recorded on this thread ("" if none)."""
+    return load_library().dsa_last_error().decode()
 
 
 def _ptr(t) -> Optional[int]:

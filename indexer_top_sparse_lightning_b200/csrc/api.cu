@@ -26,6 +26,17 @@ constexpr int kMaxSplitTokens = 128;      // row splits are only used for fewer 
 constexpr size_t kCounterBytes = kMaxSplitTokens * 2 * 4;
 constexpr size_t kHeaderBytes = kStatusBytes + kCounterBytes;
 
+// ------------------------------------------------------------------ last failure text (per host thread)
+thread_local char g_last_error[256] = "";
+
+dsa_status fail(dsa_status st, const char* what, cudaError_t e = cudaSuccess) {
+    if (e != cudaSuccess)
+        snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+    else
+        snprintf(g_last_error, sizeof g_last_error, "%s", what);
+    return st;
+}
+
 // ------------------------------------------------------------------ driver entry point (no libcuda link)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -45,7 +56,8 @@ EncodeTiledFn encode_fn() {
 }
 
 bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz) {
+              const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
+              CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t d[5], s[4];
@@ -57,7 +69,7 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* ba
         if (i + 1 < rank) s[i] = strides_bytes[i];
     }
     return fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct DevInfo {
@@ -167,7 +179,7 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
         const uint32_t box[3] = {64, (uint32_t)HI, (uint32_t)NQ};
         if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ix->q_idx, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_128B))
-            return DSA_ERR_CUDA;
+            return fail(DSA_ERR_CUDA, "indexer query tensor map encoding failed");
     }
     {
         const uint64_t dims[2] = {(uint64_t)DI, (uint64_t)bt->num_blocks * kPage};
@@ -176,18 +188,18 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
             const uint32_t box[2] = {(uint32_t)DI, (uint32_t)kPage};
             if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ix->k_cache, dims, strides, box,
                           CU_TENSOR_MAP_SWIZZLE_NONE))
-                return DSA_ERR_CUDA;
+                return fail(DSA_ERR_CUDA, "indexer key tensor map encoding failed");
         } else {
             const uint64_t strides[1] = {(uint64_t)DI * 2};
             const uint32_t box[2] = {64, (uint32_t)kPage};
             if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ix->k_cache, dims, strides, box,
                           CU_TENSOR_MAP_SWIZZLE_128B))
-                return DSA_ERR_CUDA;
+                return fail(DSA_ERR_CUDA, "indexer key tensor map encoding failed");
         }
     }
     auto kern = &indexer_topk_kernel<FP8, HI, DI, NQ>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
-        return DSA_ERR_CUDA;
+    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem))
+        return fail(DSA_ERR_CUDA, "indexer shared memory attribute", e);
 
     IndexerParams p;
     memset(&p, 0, sizeof p);
@@ -223,7 +235,7 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
         cfg.numAttrs = 0;
         p.t_begin = 0;
         p.t_end = bt->num_tokens;
-        if (cudaLaunchKernelEx(&cfg, kern, p, tm_q, tm_k) != cudaSuccess) return DSA_ERR_CUDA;
+        if (cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, tm_q, tm_k)) return fail(DSA_ERR_CUDA, "indexer launch", e);
         return DSA_OK;
     }
     // grouped mode: the CTAs of a group wait for one another, so they must be
@@ -236,7 +248,7 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
     for (int b0 = 0; b0 < bt->batch; b0 += pl.seqs_per_launch) {
         p.b_begin = b0;
         p.b_end = b0 + pl.seqs_per_launch < bt->batch ? b0 + pl.seqs_per_launch : bt->batch;
-        if (cudaLaunchKernelEx(&cfg, kern, p, tm_q, tm_k) != cudaSuccess) return DSA_ERR_CUDA;
+        if (cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, tm_q, tm_k)) return fail(DSA_ERR_CUDA, "indexer launch", e);
     }
     return DSA_OK;
 }
@@ -326,10 +338,10 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     // each CTA of a pair loads its own 64 heads (heads past H read as zeros)
     const uint32_t box[3] = {64, (uint32_t)(at->H < 64 ? at->H : 64), 1};
     if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, at->q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-        return DSA_ERR_CUDA;
-    if (cudaFuncSetAttribute(&sfa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SfaCfg::SMEM) !=
-        cudaSuccess)
-        return DSA_ERR_CUDA;
+        return fail(DSA_ERR_CUDA, "attention query tensor map encoding failed");
+    if (cudaError_t e = cudaFuncSetAttribute(&sfa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             SfaCfg::SMEM))
+        return fail(DSA_ERR_CUDA, "attention shared memory attribute", e);
     SfaParams p;
     memset(&p, 0, sizeof p);
     p.seq_lens = bt->seq_lens;
@@ -367,7 +379,8 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, &sfa_decode_kernel, p, tm_q) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaError_t e = cudaLaunchKernelEx(&cfg, &sfa_decode_kernel, p, tm_q))
+        return fail(DSA_ERR_CUDA, "attention launch", e);
     return DSA_OK;
 }
 
@@ -404,7 +417,7 @@ dsa_status indexer_topk(const dsa_batch* batch, const dsa_indexer_inputs* ix, in
     if (!out_idx) return DSA_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
     const DevInfo di = dev_info();
-    if (di.sms <= 0) return DSA_ERR_CUDA;
+    if (di.sms <= 0) return fail(DSA_ERR_CUDA, "device query failed");
     IdxPlan pl;
     LaunchFn fn = nullptr;
     if ((st = plan_indexer(batch, ix, di, pl, fn)) != DSA_OK) return st;
@@ -424,7 +437,8 @@ dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs* at, co
     if (!aligned16(out)) return DSA_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
     const DevInfo di = dev_info();
-    if (di.sms <= 0 || di.max_smem < SfaCfg::SMEM) return DSA_ERR_CUDA;
+    if (di.sms <= 0) return fail(DSA_ERR_CUDA, "device query failed");
+    if (di.max_smem < SfaCfg::SMEM) return fail(DSA_ERR_UNSUPPORTED, "device shared memory per block too small");
     const AttnPlan ap = plan_attn(batch, K, di);
     const size_t off = kHeaderBytes + idx_region_bytes(di);
     if (workspace_bytes < off + ap.part_bytes) return DSA_ERR_WORKSPACE;
@@ -453,11 +467,13 @@ dsa_status dsa_get_status(void* workspace, void* stream, int32_t* device_status)
     if (!workspace || !device_status) return DSA_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t v = 0;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
-    if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaError_t e = cudaStreamSynchronize(s)) return fail(DSA_ERR_CUDA, "stream synchronize", e);
+    if (cudaError_t e = cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost))
+        return fail(DSA_ERR_CUDA, "status read", e);
     const uint32_t zero = 0;
-    if (v != 0 && cudaMemcpy(workspace, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
-        return DSA_ERR_CUDA;
+    if (v != 0)
+        if (cudaError_t e = cudaMemcpy(workspace, &zero, sizeof zero, cudaMemcpyHostToDevice))
+            return fail(DSA_ERR_CUDA, "status clear", e);
     *device_status = (int32_t)v;
     return DSA_OK;
 }
@@ -488,6 +504,8 @@ const char* dsa_status_str(int32_t s) {
         default: return "unknown status";
     }
 }
+
+const char* dsa_last_error(void) { return g_last_error; }
 
 const char* dsa_version(void) { return "dsa-b200 0.1.0 (sm_100a)"; }
 

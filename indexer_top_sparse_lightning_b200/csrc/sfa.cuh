@@ -19,17 +19,19 @@
 //     value columns 128c..128c+127 and 256+128c..256+128c+127 of all 32 rows
 //     (B split by N); each CTA's tensor memory receives O for its 64 heads
 //     over all 512 columns.
-// Rows are gathered with 16-byte cp.async vector loads (one coalesced warp
-// read per row segment) into 128-byte-swizzled shared memory, and
-// prefetched into L2 two blocks ahead.  The online softmax keeps a lazy
-// reference max (O and l are rescaled only when the max grows by more than
-// 2^8).  With several row splits per token each CTA writes an un-normalised
-// partial O and (m, l); the last CTA of a (token, head half) to finish merges
-// the partials of all splits (arrival counted with a global atomic).
+// Rows are gathered with 16-byte vector loads into registers (one coalesced
+// warp read per row segment; the loads of the next block are in flight while
+// the current one is stored) and written to 128-byte-swizzled shared memory;
+// this CTA's own rows are prefetched into L2 a few blocks ahead.  The online
+// softmax keeps a lazy reference max (O and l are rescaled only when the max
+// grows by more than 2^8).  With several row splits per token each CTA writes
+// an un-normalised partial O and (m, l); the last CTA of a (token, head half)
+// to finish merges the partials of all splits (arrival counted with a global
+// atomic).
 //
-// Roles per CTA (256 threads): warps 0-3 softmax (thread L <-> TMEM lane L:
-// head 64c + L%64, rows or value columns of half L/64), warps 4-6 gather,
-// warp 7 TMEM allocation; in CTA 0 it issues the MMAs, in CTA 1 it forwards
+// Roles per CTA (384 threads): warps 0-3 softmax (thread L <-> TMEM lane L:
+// head 64c + L%64, rows or value columns of half L/64), warps 4-10 gather,
+// warp 11 TMEM allocation; in CTA 0 it issues the MMAs, in CTA 1 it forwards
 // "my rows landed" and "my Q landed" to CTA 0.
 #pragma once
 #include "common.h"
@@ -39,9 +41,9 @@ namespace dsa {
 
 struct SfaCfg {
     static constexpr int ROWS = 32;                     // selected rows per block (16 per CTA for S)
-    static constexpr int NS = 3;                        // gather stages in shared memory
+    static constexpr int NS = 4;                        // gather stages in shared memory
     static constexpr int NSB = 2;                       // logit / P buffers
-    static constexpr int PF = 2;                        // blocks prefetched into L2 ahead of the gather
+    static constexpr int PF = 8;                        // blocks prefetched into L2 ahead of the gather
     static constexpr int KBQ = 9;                       // 64-wide K blocks of a 576-wide row
     static constexpr int Q_BYTES = KBQ * 64 * 128;      // [64 heads x 64] per K block
     static constexpr int KOWN_KB = 16 * 128;            // own 16 rows x 64 elements, per K block
@@ -55,13 +57,13 @@ struct SfaCfg {
     static constexpr int MISC_BYTES = 1024;
     static constexpr int MAX_ROWS = 2048;               // rows of one split (K <= 2048)
     static constexpr int OFF_ROWS = OFF_MISC + MISC_BYTES;
-    static constexpr int OFF_VALID = OFF_ROWS + MAX_ROWS * 4;
-    static constexpr int OFF_XM = OFF_VALID + MAX_ROWS / 8;   // partner max exchange [2][128]
+    static constexpr int OFF_XM = OFF_ROWS + MAX_ROWS * 4;    // partner max exchange [2][128]
     static constexpr int SMEM = 1024 + OFF_XM + 2 * 128 * 4;
-    static constexpr int THREADS = 256;
-    static constexpr int GATHER = 96;                   // threads of warps 4-6
-    static constexpr int QK_CHAINS = 4;                 // independent accumulators per logit buffer
-    static constexpr int S_COLS = QK_CHAINS * 16;       // TMEM columns of one logit buffer
+    static constexpr int THREADS = 384;
+    static constexpr int GATHER = 224;                  // threads of warps 4-10
+    static constexpr int MMA_WARP = 11;                 // TMEM owner; MMA issuer (CTA 0) / forwarder (CTA 1)
+    static constexpr int GATHER_ITEMS = 16 * 72 + 16 * 32;   // 16-byte loads of one block per CTA
+    static constexpr int S_COLS = 16;                   // TMEM columns of one logit buffer
     static constexpr int TMEM_COLS = 512;               // O: [0,256), logit buffers from column 256
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, ROWS, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 256, false, true);
@@ -128,7 +130,6 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     uint8_t* s_p = smem + Cfg::OFF_P;
     SfaMisc* m = reinterpret_cast<SfaMisc*>(smem + Cfg::OFF_MISC);
     int32_t* s_rows = reinterpret_cast<int32_t*>(smem + Cfg::OFF_ROWS);
-    uint32_t* s_valid = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_VALID);
     float* s_xm = reinterpret_cast<float*>(smem + Cfg::OFF_XM);
     volatile int* abort = &m->abort;
 
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         mbar_init(&m->q_full, 1);
         mbar_init(&m->q_peer, 1);
         for (int i = 0; i < Cfg::NS; ++i) {
-            mbar_init(&m->kv_full[i], Cfg::GATHER);
+            mbar_init(&m->kv_full[i], Cfg::GATHER / 32);
             mbar_init(&m->kv_peer[i], 1);
             mbar_init(&m->kv_empty[i], 1);
         }
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         m->last = 0;
         fence_mbar_init();
     }
-    if (warp == 7) {
+    if (warp == Cfg::MMA_WARP) {
         tmem_alloc_2cta(&m->tmem_base, Cfg::TMEM_COLS);
         tmem_relinquish_2cta();
     }
@@ -181,70 +182,73 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     const uint32_t tm_s = tmem_base + 256;      // logit buffers, S_COLS columns each
     if (threadIdx.x == 0) DSA_TRACE_MARK(0);
 
-    if (warp == 7) {
+    if (warp == Cfg::MMA_WARP) {
+        // ---------------------------------------------------------------- own Q
         if (lane == 0) {
-            // ---------------------------------------------------------------- own Q
             const int hb = p.H < 64 ? p.H : 64;              // TMA box height
-            const bool load_q = head0 < p.H;
-            if (load_q) {
+            if (head0 < p.H) {
                 mbar_arrive_expect_tx(&m->q_full, Cfg::KBQ * 64 * hb * 2);
                 for (int kb = 0; kb < Cfg::KBQ; ++kb)
                     tma_load_3d(s_q + kb * 64 * 128, &tm_q, &m->q_full, kb * 64, head0, t);
             } else {
                 mbar_arrive(&m->q_full);
             }
-            volatile int no_abort = 0;
-            if (crank == 1) {
-                // ------------------------------------------------------------ forwarder
+        }
+        __syncwarp();
+        volatile int no_abort = 0;
+        if (crank == 1) {
+            // ------------------------------------------------------------ forwarder
+            if (lane == 0) {
                 bool ok = mbar_wait(&m->q_full, 0, abort);
                 if (ok) mbar_arrive_remote(mapa_shared(smem_u32(&m->q_peer), 0));
                 for (int jb = 0; ok && jb < nblk; ++jb) {
                     const int s = jb % Cfg::NS;
                     if (!mbar_wait(&m->kv_full[s], (jb / Cfg::NS) & 1, abort)) { ok = false; break; }
                     DSA_TRACE_BLK(jb, 1);
-                    // the rows were written by cp.async (generic proxy); CTA 0's MMA reads them
-                    // through the async proxy
-                    fence_proxy_async_smem();
                     mbar_arrive_remote(mapa_shared(smem_u32(&m->kv_peer[s]), 0));
                 }
                 if (!ok) *abort = 1;
-            } else {
-                // ------------------------------------------------------------ MMA issuer
-                bool ok = mbar_wait(&m->q_full, 0, abort) && mbar_wait_cluster(&m->q_peer, 0, abort);
-                tc_fence_after();
-                const uint32_t q_addr = smem_u32(s_q);
-                const uint32_t p_addr = smem_u32(s_p);
-                auto qk_ready = [&](int jb) -> bool {
-                    const int s = jb % Cfg::NS, b = jb % Cfg::NSB;
-                    const uint32_t ph = (jb / Cfg::NS) & 1;
-                    return mbar_test_wait(smem_u32(&m->kv_full[s]), ph) && mbar_test_wait_cluster(smem_u32(&m->kv_peer[s]), ph) &&
-                           mbar_test_wait_cluster(smem_u32(&m->s_empty[b]), ((jb / Cfg::NSB) & 1) ^ 1);
-                };
-                auto pv_ready = [&](int jb) -> bool {
-                    return mbar_test_wait_cluster(smem_u32(&m->p_full[jb % Cfg::NSB]), (jb / Cfg::NSB) & 1);
-                };
-                auto issue_qk = [&](int jb) {
-                    const int s = jb % Cfg::NS, b = jb % Cfg::NSB;
+            }
+            __syncwarp();
+        } else {
+            // ------------------------------------------------------------ MMA issuer
+            // The whole warp runs the schedule (decisions taken by lane 0 and
+            // broadcast); one elected lane issues each group of MMAs and its commits.
+            bool ok = __shfl_sync(0xffffffffu,
+                                  (int)(mbar_wait(&m->q_full, 0, abort) && mbar_wait(&m->q_peer, 0, abort)), 0);
+            tc_fence_after();
+            const uint32_t q_addr = smem_u32(s_q);
+            const uint32_t p_addr = smem_u32(s_p);
+            auto qk_ready = [&](int jb) -> bool {
+                const int s = jb % Cfg::NS, b = jb % Cfg::NSB;
+                const uint32_t ph = (jb / Cfg::NS) & 1;
+                return mbar_test_wait(smem_u32(&m->kv_full[s]), ph) && mbar_test_wait(smem_u32(&m->kv_peer[s]), ph) &&
+                       mbar_test_wait(smem_u32(&m->s_empty[b]), ((jb / Cfg::NSB) & 1) ^ 1);
+            };
+            auto pv_ready = [&](int jb) -> bool {
+                return mbar_test_wait(smem_u32(&m->p_full[jb % Cfg::NSB]), (jb / Cfg::NSB) & 1);
+            };
+            auto issue_qk = [&](int jb) {
+                const int s = jb % Cfg::NS, b = jb % Cfg::NSB;
+                if (elect_one()) {
                     DSA_TRACE_BLK(jb, 6);
-                    fence_proxy_async_smem();   // this CTA's cp.async rows -> async proxy
                     tc_fence_after();
                     const uint32_t kown = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
-                    // the 36 K steps go round-robin to QK_CHAINS accumulators, so that
-                    // consecutive MMAs never wait on each other's result; the softmax adds
-                    // the chains
-#pragma unroll 1
+#pragma unroll
                     for (int kb = 0; kb < Cfg::KBQ; ++kb)
 #pragma unroll
                         for (int k16 = 0; k16 < 4; ++k16)
-                            umma_bf16_2cta(tm_s + b * Cfg::S_COLS + (k16 % Cfg::QK_CHAINS) * 16,
-                                           sdesc_sw128(q_addr + kb * 8192 + k16 * 32, 16, 1024),
+                            umma_bf16_2cta(tm_s + b * Cfg::S_COLS, sdesc_sw128(q_addr + kb * 8192 + k16 * 32, 16, 1024),
                                            sdesc_sw128(kown + kb * Cfg::KOWN_KB + k16 * 32, 16, 1024),
-                                           Cfg::IDESC_QK, kb * 4 + k16 >= Cfg::QK_CHAINS);
+                                           Cfg::IDESC_QK, (kb | k16) != 0);
                     umma_commit_2cta(&m->s_full[b], 3);
                     DSA_TRACE_BLK(jb, 2);
-                };
-                auto issue_pv = [&](int jb) {
-                    const int s = jb % Cfg::NS, b = jb % Cfg::NSB;
+                }
+                __syncwarp();
+            };
+            auto issue_pv = [&](int jb) {
+                const int s = jb % Cfg::NS, b = jb % Cfg::NSB;
+                if (elect_one()) {
                     DSA_TRACE_BLK(jb, 7);
                     tc_fence_after();
                     const uint32_t vall = smem_u32(s_kv + s * Cfg::STAGE_BYTES + Cfg::KBQ * Cfg::KOWN_KB);
@@ -261,40 +265,43 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                     umma_commit_2cta(&m->kv_empty[s], 3);
                     umma_commit_2cta(&m->p_empty[b], 3);
                     DSA_TRACE_BLK(jb, 8);
-                };
-                int next_qk = 0, next_pv = 0;
-                uint64_t t_idle = 0;
-                while (ok && next_pv < nblk) {
-                    bool progressed = false;
-                    if (next_qk < nblk && next_qk < next_pv + Cfg::NSB && qk_ready(next_qk)) {
-                        issue_qk(next_qk++);
-                        progressed = true;
-                    } else if (next_pv < next_qk && pv_ready(next_pv)) {
-                        issue_pv(next_pv++);
-                        progressed = true;
-                    }
-                    if (progressed) {
-                        t_idle = 0;
-                    } else if (*abort) {
-                        ok = false;
-                    } else {
-                        const uint64_t now = globaltimer();
-                        if (t_idle == 0) t_idle = now;
-                        else if (now - t_idle > kWaitTimeoutNs) ok = false;
-                    }
                 }
+                __syncwarp();
+            };
+            int next_qk = 0, next_pv = 0;
+            uint64_t t_idle = 0;
+            while (ok && next_pv < nblk) {
+                const bool do_qk = __shfl_sync(0xffffffffu, (int)(next_qk < nblk && next_qk < next_pv + Cfg::NSB &&
+                                                                  qk_ready(next_qk)), 0);
+                const bool do_pv = !do_qk && __shfl_sync(0xffffffffu, (int)(next_pv < next_qk && pv_ready(next_pv)), 0);
+                if (do_qk) {
+                    issue_qk(next_qk++);
+                    t_idle = 0;
+                } else if (do_pv) {
+                    issue_pv(next_pv++);
+                    t_idle = 0;
+                } else {
+                    bool stop = *abort != 0;
+                    const uint64_t now = globaltimer();
+                    if (t_idle == 0) t_idle = now;
+                    else if (now - t_idle > kWaitTimeoutNs) stop = true;
+                    ok = !__shfl_sync(0xffffffffu, (int)stop, 0);
+                }
+            }
+            if (elect_one()) {
                 umma_commit_2cta(&m->o_full, 3);
                 umma_commit_2cta(&m->drain, 1);
-                mbar_wait(&m->drain, 0, &no_abort);
-                if (!ok) *abort = 1;
             }
-            // no TMA write may be in flight at exit
-            mbar_wait(&m->q_full, 0, &no_abort);
+            __syncwarp();
+            mbar_wait(&m->drain, 0, &no_abort);
+            if (!ok && lane == 0) *abort = 1;
         }
+        // no TMA write may be in flight at exit
+        if (lane == 0) mbar_wait(&m->q_full, 0, &no_abort);
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- row gather
         const int pt = threadIdx.x - 128;           // 0..GATHER-1
-        const int gw = pt >> 5;                      // gather warp 0..2
+        const int gw = pt >> 5;                      // gather warp 0..6
         const int b = token_sequence(p.cu_q, p.B, t);
         const int64_t L = __ldg(p.seq_lens + b);
         const int32_t* idx_t = p.idx + (int64_t)t * p.K;
@@ -327,61 +334,104 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                 if (blk[k] >= 0 && blk[k] < p.num_blocks) row = blk[k] * kPage + pos[k] % kPage;
                 else if (pos[k] >= 0 && blk[k] != -1) atomicCAS(p.status, 0u, (uint32_t)kStBounds);
                 s_rows[i] = row;
-                const uint32_t bits = __ballot_sync(0xffffffffu, row >= 0);
-                if (lane == 0) s_valid[i >> 5] = bits;
             }
         }
         mbar_arrive(&m->rows_ready);
-        if (pt == 0) DSA_TRACE_MARK(1);
         named_bar_sync(2, Cfg::GATHER);
-        // this CTA's own rows, prefetched into L2 ahead of the gather
+        // The gather: every thread owns IPT fixed 16-byte items i = pt + GATHER*u of a
+        // block and keeps the loads of one block in flight while it stores the
+        // previous one.
+        //   i < 1152        : own row i / 72, 16-byte chunk i % 72 (all 576 columns);
+        //                     chunks of this CTA's value columns are stored twice
+        //                     (logit operand and value operand)
+        //   1152 <= i < 1664: peer row j / 32 (j = i - 1152), value chunk j % 32 of this
+        //                     CTA's columns
+        //   i >= 1664       : none (both bounds are multiples of 32: warp-uniform)
+        // Skipped selections (row -1) load row 0; their logits are masked.
+        constexpr int IPT = (Cfg::GATHER_ITEMS + Cfg::GATHER - 1) / Cfg::GATHER;
+        constexpr int OWN_ITEMS = 16 * 72;
+        static_assert(OWN_ITEMS % 32 == 0 && Cfg::GATHER_ITEMS % 32 == 0 && Cfg::GATHER % 32 == 0, "warp-uniform items");
+        const int c = (int)crank;
         auto prefetch_block = [&](int jb) {
-            if (jb < nblk && pt < 16) {
-                const int32_t row = s_rows[jb * Cfg::ROWS + 16 * (int)crank + pt];
+            if (gw == 0 && jb < nblk && lane < 16) {
+                const int32_t row = s_rows[jb * Cfg::ROWS + 16 * c + lane];
                 if (row >= 0) prefetch_l2(kv_bytes + (int64_t)row * (kDqk * 2), kDqk * 2);
             }
         };
-        for (int jb = 0; jb < Cfg::PF; ++jb) prefetch_block(jb);
-        // lane roles within a warp: 16-byte chunk `lane` of a 512-byte segment
-        const uint32_t lane_q = (uint32_t)(lane & 7);
-        const uint32_t lane_kb = (uint32_t)(lane >> 3);
-        for (int jb = 0; jb < nblk; ++jb) {
-            const int s = jb % Cfg::NS;
-            prefetch_block(jb + Cfg::PF);
-            if (!mbar_wait(&m->kv_empty[s], ((jb / Cfg::NS) & 1) ^ 1, abort)) { *abort = 1; break; }
-            if (pt == 0) DSA_TRACE_BLK(jb, 5);
-            const uint32_t kown = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
-            const uint32_t vall = kown + Cfg::KBQ * Cfg::KOWN_KB;
-            const int32_t* rows = s_rows + jb * Cfg::ROWS;
-            // own rows: all 1152 bytes into the K blocks of the logit operand
-            for (int r = gw; r < 16; r += Cfg::GATHER / 32) {
-                const int32_t row = rows[16 * (int)crank + r];
-                const bool ok_row = row >= 0;
-                const uint8_t* src = kv_bytes + (ok_row ? (int64_t)row * (kDqk * 2) : 0);
-                const uint32_t sw = (uint32_t)(r & 7);
+        // Item descriptors are the same for every block: computed once.
+        //   src[u]: byte offset in the row (bits 0-10), row of the block (bits 16-20);
+        //           0xFFFFFFFF = no item
+        //   dst[u]: stage offset of the logit or value copy (bits 0-15) and of the
+        //           second (value) copy (bits 16-31, 0xFFFF = none)
+        uint32_t src[IPT], dst[IPT];
 #pragma unroll
-                for (int seg = 0; seg < 3; ++seg) {              // 72 chunks: 32 + 32 + 8
-                    const int ch = seg * 32 + lane;
-                    if (ch < 72) {
-                        const uint32_t kb = (uint32_t)ch >> 3, q = (uint32_t)ch & 7;
-                        cp_async_16(kown + kb * Cfg::KOWN_KB + r * 128 + ((q ^ sw) << 4), src + ch * 16, ok_row);
-                    }
-                }
+        for (int u = 0; u < IPT; ++u) {
+            const int i = pt + Cfg::GATHER * u;
+            src[u] = 0xFFFFFFFFu;
+            dst[u] = 0xFFFFFFFFu;
+            if (i < OWN_ITEMS) {
+                const int r = i / 72, ch = i % 72, kb = ch >> 3, q = ch & 7;
+                const int sw = (q ^ (r & 7)) << 4;
+                // value K blocks of this CTA: 2c, 2c+1 -> chunks 0, 1; 4+2c, 5+2c -> chunks 2, 3;
+                // row 16c + r of a value chunk has the same swizzle phase as row r
+                const int kr = kb - 2 * c;
+                const int vq = (kr == 0 || kr == 1) ? kr : ((kr == 4 || kr == 5) ? kr - 2 : -1);
+                src[u] = (uint32_t)(ch * 16) | ((uint32_t)(16 * c + r) << 16);
+                const uint32_t d2 = vq >= 0 ? (uint32_t)(Cfg::KBQ * Cfg::KOWN_KB + vq * Cfg::VALL_KB + (16 * c + r) * 128 + sw)
+                                            : 0xFFFFu;
+                dst[u] = (uint32_t)(kb * Cfg::KOWN_KB + r * 128 + sw) | (d2 << 16);
+            } else if (i < Cfg::GATHER_ITEMS) {
+                const int j = i - OWN_ITEMS;
+                const int v = j & 31, r = j >> 5;             // 8 chunks of each of 4 value K blocks
+                const int kbv = v >> 3;
+                const int kb = kbv < 2 ? 2 * c + kbv : 4 + 2 * c + (kbv - 2);
+                src[u] = (uint32_t)(kb * 128 + (v & 7) * 16) | ((uint32_t)(16 * (1 - c) + r) << 16);
+                dst[u] = (uint32_t)(Cfg::KBQ * Cfg::KOWN_KB + kbv * Cfg::VALL_KB + (16 * (1 - c) + r) * 128 +
+                                    (((v & 7) ^ (r & 7)) << 4)) | (0xFFFFu << 16);
             }
-            // all rows: this CTA's 256 value columns (two 128-column halves)
-            for (int r = gw; r < Cfg::ROWS; r += Cfg::GATHER / 32) {
-                const int32_t row = rows[r];
-                const bool ok_row = row >= 0;
-                const uint8_t* src = kv_bytes + (ok_row ? (int64_t)row * (kDqk * 2) : 0);
-                // chunk kb of the 4: columns 128*crank + 64*kb (kb < 2) or 256 + 128*crank + 64*(kb-2)
-                const int col0 = (lane_kb < 2 ? 128 * (int)crank + 64 * (int)lane_kb : 256 + 128 * (int)crank + 64 * ((int)lane_kb - 2));
-                cp_async_16(vall + lane_kb * Cfg::VALL_KB + r * 128 + ((lane_q ^ (uint32_t)(r & 7)) << 4),
-                            src + col0 * 2 + lane_q * 16, ok_row);
-            }
-            // the barrier receives this thread's arrival once its copies have landed
-            cp_async_arrive_noinc(&m->kv_full[s]);
         }
-        cp_async_wait_all();
+        static_assert(Cfg::STAGE_BYTES <= 0xFFFF, "stage offsets are packed in 16 bits");
+        auto load = [&](uint4 (&R)[IPT], int jb) {
+            const int32_t* rows = s_rows + jb * Cfg::ROWS;
+#pragma unroll
+            for (int u = 0; u < IPT; ++u) {
+                if (src[u] == 0xFFFFFFFFu) continue;          // warp-uniform
+                const int32_t r = rows[src[u] >> 16];
+                R[u] = ld_nc_v4(kv_bytes + (int64_t)(r < 0 ? 0 : r) * (kDqk * 2) + (src[u] & 0xFFFFu));
+            }
+        };
+        auto store = [&](const uint4 (&R)[IPT], int jb) -> bool {
+            const int s = jb % Cfg::NS;
+            if (!__all_sync(0xffffffffu, mbar_wait(&m->kv_empty[s], ((jb / Cfg::NS) & 1) ^ 1, abort))) return false;
+            if (pt == 0) DSA_TRACE_BLK(jb, 5);
+            const uint32_t base = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
+#pragma unroll
+            for (int u = 0; u < IPT; ++u) {
+                if (src[u] == 0xFFFFFFFFu) continue;
+                st_shared_v4(base + (dst[u] & 0xFFFFu), R[u]);
+                if ((dst[u] >> 16) != 0xFFFFu) st_shared_v4(base + (dst[u] >> 16), R[u]);
+            }
+            // generic-proxy stores -> visible to the tensor core, then one arrival per warp
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&m->kv_full[s]);
+            return true;
+        };
+        if (gw == 0 && lane == 0) DSA_TRACE_MARK(1);
+        for (int jb = 0; jb < Cfg::PF; ++jb) prefetch_block(jb);
+        uint4 ra[IPT], rb[IPT];
+        bool ok = true;
+        if (nblk > 0) load(ra, 0);
+        for (int jb = 0; ok && jb < nblk; jb += 2) {
+            prefetch_block(jb + Cfg::PF);
+            prefetch_block(jb + Cfg::PF + 1);
+            if (jb + 1 < nblk) load(rb, jb + 1);
+            ok = store(ra, jb);
+            if (!ok || jb + 1 >= nblk) break;
+            if (jb + 2 < nblk) load(ra, jb + 2);
+            ok = store(rb, jb + 1);
+        }
+        if (!ok && lane == 0) *abort = 1;
     } else {
         // ---------------------------------------------------------------- softmax + epilogue
         const int L = threadIdx.x;                   // TMEM lane
@@ -394,7 +444,17 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         bool ok = nblk == 0 || mbar_wait(&m->rows_ready, 0, abort);
         for (int jb = 0; jb < nblk; ++jb) {
             const int b = jb % Cfg::NSB;
-            const uint32_t vbits = (s_valid[jb] >> (16 * half)) & 0xFFFFu;
+            // validity of this lane's 16 rows (skipped selections hold row -1)
+            uint32_t vbits = 0;
+            {
+                const int4* r4 = reinterpret_cast<const int4*>(s_rows + jb * Cfg::ROWS + 16 * half);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int4 v = r4[q];
+                    vbits |= (uint32_t)(v.x >= 0) << (4 * q) | (uint32_t)(v.y >= 0) << (4 * q + 1) |
+                             (uint32_t)(v.z >= 0) << (4 * q + 2) | (uint32_t)(v.w >= 0) << (4 * q + 3);
+                }
+            }
             const bool got = __all_sync(0xffffffffu, ok && mbar_wait(&m->s_full[b], (jb / Cfg::NSB) & 1, abort));
             float sv[16];
             float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -402,18 +462,15 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                 if (jb == 0 && L == 0) DSA_TRACE_MARK(2);
                 if (L == 0) DSA_TRACE_BLK(jb, 0);
                 tc_fence_after();
-                static_assert(Cfg::QK_CHAINS == 4, "the chain sum below adds four 16-column groups");
-                uint32_t a[32], c[32];
-                tmem_ld32(tm_s + lane_off + b * Cfg::S_COLS, a);
-                tmem_ld32(tm_s + lane_off + b * Cfg::S_COLS + 32, c);
+                uint32_t a[16];
+                tmem_ld16(tm_s + lane_off + b * Cfg::S_COLS, a);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) arrive_leader(&m->s_empty[b], crank);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float x = (__uint_as_float(a[i]) + __uint_as_float(a[16 + i])) +
-                                    (__uint_as_float(c[i]) + __uint_as_float(c[16 + i]));
+                    const float x = __uint_as_float(a[i]);
                     sv[i] = ((vbits >> i) & 1u) ? x * p.scale_log2 : -INFINITY;
                     if (i & 1) mx1 = fmaxf(mx1, sv[i]);
                     else mx0 = fmaxf(mx0, sv[i]);
@@ -588,12 +645,13 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         }
         __syncthreads();
         // thread -> 4-column chunk c4 = tid % 128 of heads tid/128 + 2u, u < 32, so that
-        // a warp reads 512 contiguous bytes; the loads of 16 heads are issued
+        // a warp reads 512 contiguous bytes; the loads of 8 heads are issued
         // together, one split at a time
         const int c4 = threadIdx.x & 127;
-        constexpr int U = 16;
+        constexpr int U = 8;
+        static_assert(Cfg::THREADS >= 256, "the merge maps 256 threads onto 64 heads x 128 chunks");
 #pragma unroll 1
-        for (int u0 = 0; u0 < 32; u0 += U) {
+        for (int u0 = 0; threadIdx.x < 256 && u0 < 32; u0 += U) {
             float4 acc[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -625,7 +683,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         if (threadIdx.x == 0) p.split_count[(int64_t)t * 2 + crank] = 0u;   // ready for the next call
     }
     cluster_sync();   // no remote access may target an exited CTA, and no MMA may read a freed tile
-    if (warp == 7) {
+    if (warp == Cfg::MMA_WARP) {
         tc_fence_after();
         tmem_dealloc_2cta(tmem_base, Cfg::TMEM_COLS);
     }
