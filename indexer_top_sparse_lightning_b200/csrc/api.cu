@@ -117,6 +117,9 @@ dsa_status check_attn(const dsa_attn_inputs* at) {
     return DSA_OK;
 }
 
+size_t align256(size_t v);
+size_t group_region_bytes(int sms);
+
 // ------------------------------------------------------------------ indexer planning
 struct IdxPlan {
     int mode = 0;        // 0 grouped decode, 1 per-token
@@ -141,6 +144,7 @@ bool plan_for(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl) {
     const int cap = (di.max_smem - Cfg::FIXED_SMEM) / 4;
     if (cap < kTileKeys * NQ) return false;
     pl.score_cap = (cap / (kTileKeys * NQ)) * (kTileKeys * NQ);
+    if (pl.score_cap > kCandSlotKeys) pl.score_cap = (int)((kCandSlotKeys / (kTileKeys * NQ)) * (kTileKeys * NQ));
     pl.smem = Cfg::FIXED_SMEM + pl.score_cap * 4;
     pl.grid = di.sms;     // one CTA per SM (shared memory use allows no more)
     if (pl.mode == 1) {
@@ -213,6 +217,8 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
     p.status = status;
     p.group_ws = group_ws;
     p.group_ws_stride = group_ws_bytes(2, pl.grid);
+    p.cand = reinterpret_cast<uint32_t*>(group_ws + group_region_bytes(pl.grid));
+    p.cand_slot = kCandSlotKeys;
     p.B = bt->batch;
     p.T = bt->num_tokens;
     p.max_blocks = bt->max_blocks_per_seq;
@@ -322,12 +328,13 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace layout, the same for every shape on a given device:
 //   [status 256 B][split arrival counters 1 KB][indexer group region, fixed
-//   size][attention partials]
-// The indexer region is sized for the largest grouped launch (one group per
+//   size][indexer published-key slots, one per SM][attention partials]
+// The indexer regions are sized for the largest grouped launch (one group per
 // SM, two tokens per group), so calls of any shape sharing one workspace
-// never write attention partials over the indexer's zero-filled region.
+// never write attention partials over the indexer's barrier words.
+size_t group_region_bytes(int sms) { return align256((size_t)sms * (size_t)group_ws_bytes(2, sms)); }
 size_t idx_region_bytes(const DevInfo& di) {
-    return align256((size_t)di.sms * (size_t)group_ws_bytes(2, di.sms));
+    return group_region_bytes(di.sms) + align256((size_t)di.sms * (size_t)kCandSlotKeys * 4);
 }
 
 dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int32_t* idx, int K, void* out,
@@ -400,7 +407,7 @@ size_t dsa_workspace_size(const dsa_batch* batch, const dsa_indexer_inputs* ix, 
         IdxPlan pl;
         LaunchFn fn = nullptr;
         if (plan_indexer(batch, ix, di, pl, fn) != DSA_OK) return 0;
-        if (pl.group_ws > idx_region_bytes(di)) return 0;
+        if (pl.group_ws > group_region_bytes(di.sms)) return 0;
     }
     if (at) {
         if (check_attn(at) != DSA_OK) return 0;
@@ -421,8 +428,8 @@ dsa_status indexer_topk(const dsa_batch* batch, const dsa_indexer_inputs* ix, in
     IdxPlan pl;
     LaunchFn fn = nullptr;
     if ((st = plan_indexer(batch, ix, di, pl, fn)) != DSA_OK) return st;
-    if (pl.group_ws > idx_region_bytes(di)) return DSA_ERR_UNSUPPORTED;
-    if (workspace_bytes < kHeaderBytes + pl.group_ws) return DSA_ERR_WORKSPACE;
+    if (pl.group_ws > group_region_bytes(di.sms)) return DSA_ERR_UNSUPPORTED;
+    if (workspace_bytes < kHeaderBytes + idx_region_bytes(di)) return DSA_ERR_WORKSPACE;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     return fn(batch, ix, out_idx, out_score, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, pl,
               reinterpret_cast<cudaStream_t>(stream));

@@ -40,8 +40,10 @@ struct IndexerParams {
     int32_t* out_idx;
     float* out_score;
     uint32_t* status;
-    uint8_t* group_ws;        // mode 0: per-group sync + histograms + counts
+    uint8_t* group_ws;        // mode 0: per-group sync + publication headers
     int64_t group_ws_stride;  // bytes per group
+    uint32_t* cand;           // mode 0: published keys, cand_slot per CTA
+    int64_t cand_slot;        // keys per CTA slot (NQ tokens share it equally)
     int32_t B, T, max_blocks, num_blocks;
     int32_t b_begin, b_end;   // mode 0 launch range
     int32_t t_begin, t_end;   // mode 1 token range
@@ -52,11 +54,14 @@ struct IndexerParams {
 
 // Group workspace layout (mode 0), per group:
 //   [0,128)   sync {count, gen}
-//   hist[3][NQ][2048] u32
-//   cnt[max_ctas][NQ][2] u32
+//   hdr[max_ctas][NQ][4] u32: published key count, smallest published key,
+//             largest visible key, publication edge
 __host__ __device__ constexpr int64_t group_ws_bytes(int nq, int max_ctas) {
-    return 128 + 3LL * nq * 2048 * 4 + (int64_t)max_ctas * nq * 2 * 4;
+    return 128 + (int64_t)max_ctas * nq * 4 * 4;
 }
+
+// Published-key slot per CTA (keys; larger than any CTA's score capacity).
+constexpr int64_t kCandSlotKeys = 65536;
 
 template <int DI, bool FP8>
 struct KeyTileBytes {

@@ -58,7 +58,7 @@ struct IdxCfg {
     static constexpr int Q_BYTES = N * DI * 2;
     static constexpr int Q_TX = NQ * HI * DI * 2;             // bytes one Q load brings in
     static constexpr bool Q_PAD = NQ * HI < N;                // rows [NQ*HI, N) stay zero
-    static constexpr int HIST_WORDS = NQ * 2048;
+    static constexpr int HIST_WORDS = kBins;                  // select histograms
     static constexpr int W_FLOATS = NQ * HI;
     static constexpr int THREADS = FP8 ? 320 : 192;
     static constexpr int PRODUCER_WARP = 4;
@@ -74,8 +74,10 @@ struct IdxCfg {
     static constexpr int MISC_BYTES = 1024;
     static constexpr int MAX_PAGES = 512;                     // page ids of one work item, staged in smem
     static constexpr int OFF_BLK = OFF_MISC + MISC_BYTES;
-    static constexpr int OFF_LIST = OFF_BLK + MAX_PAGES * 4;   // select lists, u16 [NQ][4 warps][cap]
-    static constexpr int OFF_SCORE = OFF_LIST + NQ * 4 * kListCap * 2;
+    static constexpr int OFF_LIST = OFF_BLK + MAX_PAGES * 4;   // select list, u32 [kListCap]
+    static constexpr int OFF_SCORE = OFF_LIST + kListCap * 4;
+    // shared memory free during grouped select (the key stages and widened keys)
+    static constexpr int SCRATCH_BYTES = OFF_Q - OFF_STAGE;
     // dynamic shared memory = 1024 (alignment slack) + OFF_SCORE + score_cap * 4
     static constexpr int FIXED_SMEM = 1024 + OFF_SCORE;
 };
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         const __grid_constant__ CUtensorMap tm_k) {
     using Cfg = IdxCfg<FP8, HI, DI, NQ>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = align_shared(smem_raw, 1024);
     uint8_t* s_stage = smem + Cfg::OFF_STAGE;
     uint8_t* s_conv = smem + Cfg::OFF_CONV;
     uint8_t* s_q = smem + Cfg::OFF_Q;
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
     float* s_w = reinterpret_cast<float*>(smem + Cfg::OFF_W);
     IdxMisc* m = reinterpret_cast<IdxMisc*>(smem + Cfg::OFF_MISC);
     float* s_score = reinterpret_cast<float*>(smem + Cfg::OFF_SCORE);
-    uint16_t* s_list = reinterpret_cast<uint16_t*>(smem + Cfg::OFF_LIST);
+    uint32_t* s_list = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_LIST);
     volatile int* abort = &m->abort;
 
     const int warp = threadIdx.x >> 5;
@@ -427,20 +429,30 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 const int j = i / HI;
                 s_w[i] = (j < item.nq) ? __ldg(p.w + (int64_t)(item.t0 + j) * HI + (i % HI)) : 0.0f;
             }
-            for (int i = threadIdx.x; i < Cfg::HIST_WORDS; i += kEpiThreads) s_hist[i] = 0u;
+            if (threadIdx.x < NQ) {
+                m->sel.kmin[threadIdx.x] = 0xFFFFFFFFu;
+                m->sel.kmax[threadIdx.x] = 0u;
+            }
             GroupView gv{nullptr, nullptr, nullptr, item.G, item.rank};
             uint32_t gen = 0;
             if (item.G > 1) {
                 uint8_t* gw = p.group_ws + (int64_t)item.group * p.group_ws_stride;
                 gv.sync = reinterpret_cast<uint32_t*>(gw);
-                gv.hist = reinterpret_cast<uint32_t*>(gw + 128);
-                gv.cnt = gv.hist + 3 * NQ * 2048;
+                gv.hdr = reinterpret_cast<uint32_t*>(gw + 128);
+                // published-key slots of this group's CTAs (contiguous, rank order)
+                gv.cand = p.cand + (int64_t)((int)blockIdx.x - item.rank) * p.cand_slot;
                 // the group's barrier generation cannot move before this CTA arrives
                 if (threadIdx.x == 0) gen = ld_acquire_gpu(gv.sync + 1);
             }
             named_bar_sync(1, kEpiThreads);
             const int stride = item.tile_count * kTileKeys;   // score slots per token
             const int64_t chunk0 = (int64_t)item.tile_begin * kTileKeys;
+            uint32_t kmn[NQ], kmx[NQ];
+#pragma unroll
+            for (int j = 0; j < NQ; ++j) {
+                kmn[j] = 0xFFFFFFFFu;
+                kmx[j] = 0u;
+            }
             const int64_t npages = (item.L + kPage - 1) / kPage;
             for (int li = 0; li < item.tile_count; ++li, ++it) {
                 const int buf = it & 1;
@@ -502,19 +514,28 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                     if (j < item.nq) {
                         const float f = score[j] == 0.0f ? 0.0f : score[j];
                         s_score[j * stride + li * kTileKeys + row] = f;
-                        // pass-0 digit histogram; lanes with the same bin add once (scores of a
-                        // tile cluster in few bins, so plain atomics would serialize)
-                        const bool vis = pos <= item.pos[j];
-                        const uint32_t bin = order_key(f) >> 21;
-                        const uint32_t act = __ballot_sync(0xffffffffu, vis);
-                        if (vis) {
-                            const uint32_t peers = __match_any_sync(act, bin);
-                            if ((int)(__ffs(peers) - 1) == lane) atomicAdd(&s_hist[j * 2048 + bin], (uint32_t)__popc(peers));
+                        // range of the visible keys, for the select's first histogram
+                        if (pos <= item.pos[j]) {
+                            const uint32_t key = order_key(f);
+                            kmn[j] = min(kmn[j], key);
+                            kmx[j] = max(kmx[j], key);
                         }
                     }
                 }
             }
             if (!ok) break;
+#pragma unroll
+            for (int j = 0; j < NQ; ++j) {
+#pragma unroll
+                for (int o = 16; o; o >>= 1) {
+                    kmn[j] = min(kmn[j], __shfl_xor_sync(0xffffffffu, kmn[j], o));
+                    kmx[j] = max(kmx[j], __shfl_xor_sync(0xffffffffu, kmx[j], o));
+                }
+                if (lane == 0 && j < item.nq) {
+                    red_min_shared(&m->sel.kmin[j], kmn[j]);
+                    red_max_shared(&m->sel.kmax[j], kmx[j]);
+                }
+            }
             named_bar_sync(1, kEpiThreads);
             if (threadIdx.x == 0) DSA_TRACE_MARK(2);
 
@@ -550,7 +571,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 }
             }
             if (any_active &&
-                !topk_select<NQ>(p, gv, gen, s_score, stride, nloc, active, chunk0, item.t0, s_hist, s_list, &m->sel,
+                !topk_select<NQ>(p, gv, gen, s_score, stride, nloc, active, chunk0, item.t0, s_hist, s_list,
+                                 smem + Cfg::OFF_STAGE, Cfg::SCRATCH_BYTES, &m->sel,
                                  abort)) {
                 ok = false;
                 break;

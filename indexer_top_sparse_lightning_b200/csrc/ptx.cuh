@@ -166,6 +166,30 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Shared-memory atomics by explicit address space (a generic atomic on a
+// shared address takes a much slower path).
+__device__ __forceinline__ void red_add_shared(uint32_t* p, uint32_t v) {
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_min_shared(uint32_t* p, uint32_t v) {
+    asm volatile("red.shared.min.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_max_shared(uint32_t* p, uint32_t v) {
+    asm volatile("red.shared.max.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_shared(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.shared.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+    return old;
+}
+
+// The dynamic shared memory base rounded up to `align` bytes, as a pointer
+// into the shared window (pointer arithmetic, so the compiler keeps the
+// address space; an integer round trip would make every access generic).
+__device__ __forceinline__ uint8_t* align_shared(uint8_t* base, uint32_t align) {
+    return base + ((align - (smem_u32(base) & (align - 1u))) & (align - 1u));
+}
+
 // 16-byte read-only global load that does not allocate in L1.
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     uint4 v;

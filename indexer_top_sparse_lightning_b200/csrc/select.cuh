@@ -7,37 +7,49 @@
 // memory for the weighted aggregation and the Top-K pass; no intermediate
 // tensor goes to global memory).
 //
-// Scores are mapped to order-preserving 32-bit keys (-0 folded into +0).  The
-// K-th largest key T is found with three radix digits (11/11/10 bits); the
-// CTAs of a group add their digit histograms into a small global histogram
-// and meet at a bounded barrier.  Elements above T are selected; elements
-// equal to T are selected lowest position first.  The chunk of a CTA is a
-// contiguous position range and warp w of the four select warps owns a
-// contiguous quarter of it, so "warp order" is "position order" and every
-// count needed for the output offsets is a per-warp running count:
-//   pass-1 scan: elements whose first digit is above T's  (counted)
-//   pass-2 scan: elements matching the first digit whose second is above
-//                (counted); elements matching both digits are listed
-//   after T:     listed elements above / equal to T       (counted)
-// Indices are written in ascending position order with ballots and prefix
-// counts (no atomics on the output).
+// Scores are compared as order-preserving 32-bit keys (-0 folded into +0).
+// The K-th largest key T is found by range histograms in key space: 2048 bins
+// over [lo, hi] (bin = (key - lo) >> shift); the bin holding the K-th largest
+// element is either resolved exactly from a short list of its keys or becomes
+// the next, 2^11 times narrower, range.
+//
+// A group of G CTAs sharing one sequence meets once:
+//   1. each CTA publishes the keys at or above the lower edge e_r of the bin
+//      of its local c-th largest score, c = min(K, 2K/G + 32) (about twice its
+//      expected share of the Top-K), with its count and e_r;
+//   2. bounded group barrier;
+//   3. every CTA loads all published keys into shared memory (the key stages,
+//      idle by then) and finds T', the K-th largest published key.  If
+//      T' >= e_r for every r, every key >= T' was published, so T = T'.
+//      Otherwise (a CTA held far more than its share) the CTAs with e_r > T'
+//      publish every key >= T', the group meets again, and the K-th largest
+//      of the enlarged set is exact (T >= T', and all keys >= T' are in it).
+//   4. per lower-ranked CTA, the published keys above / equal to T give this
+//      CTA's output offset and its share of the tied elements.
+// Elements above T are selected; elements equal to T are selected lowest
+// position first (CTAs own contiguous position ranges in rank order, and
+// within a CTA warp w owns the w-th quarter).  Indices are written in
+// ascending position order with ballots and prefix counts.
 #pragma once
 #include "common.h"
 #include "ptx.cuh"
 
 namespace dsa {
 
-constexpr int kListCap = 256;   // listed (two-digit match) elements per warp and token
+constexpr int kBins = 2048;      // range histogram bins (11 bits)
+constexpr int kListCap = 1024;   // keys of the threshold bin resolved exactly
 
 struct SelectSmem {
     uint32_t scan[8];
-    uint32_t wcnt[4][4][2];     // [token][warp][gt, eq]
-    uint32_t wallow[4][4];      // [token][warp] tied elements the warp may take
-    uint32_t sel_bin[4];
-    uint32_t sel_kk[4];
-    uint32_t sel_take[4];
-    uint32_t sel_base[4];
-    uint32_t list_n[4][4];      // [token][warp]
+    uint32_t kmin[4], kmax[4];   // order keys of the visible local scores, per token (from the epilogue)
+    uint32_t res_bin, res_kk, res_cnt;
+    uint32_t fill;               // list / published-key fill counter
+    uint32_t cmin;               // smallest published key
+    uint32_t wcnt[4][2];         // [warp][gt, eq]
+    uint32_t wallow[4];
+    uint32_t edge[4];            // this CTA's publication edge, per token
+    uint32_t wpub[4][4];         // [token][warp] published elements
+    uint32_t g_lo, g_hi, g_total, g_resident, g_max_edge;
 };
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) {
@@ -96,23 +108,24 @@ __device__ __forceinline__ uint32_t epi_exclusive_scan(uint32_t v, uint32_t* scr
     return before + x - v;
 }
 
-// Radix step: the bin of the histogram (nb bins, higher bin = larger keys)
-// holding the kk-th largest element, and the rank of that element in the bin.
-__device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t kk, uint32_t* scratch,
-                                         uint32_t* out_bin, uint32_t* out_kk) {
+// The bin (of nb, higher bin = larger keys) holding the kk-th largest counted
+// element, the rank of that element inside the bin and the bin's count, in
+// sm->res_*.  kk must not exceed the total count.
+__device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t kk, SelectSmem* sm) {
     const int per = nb / kEpiThreads;
     const int hi_bin = nb - 1 - (int)threadIdx.x * per;
     uint32_t s = 0;
     for (int i = 0; i < per; ++i) s += hist[hi_bin - i];
     uint32_t total;
-    const uint32_t before = epi_exclusive_scan(s, scratch, &total);
+    const uint32_t before = epi_exclusive_scan(s, sm->scan, &total);
     if (before < kk && kk <= before + s) {
         uint32_t c = before;
         for (int i = 0; i < per; ++i) {
             const uint32_t h = hist[hi_bin - i];
             if (c + h >= kk) {
-                *out_bin = (uint32_t)(hi_bin - i);
-                *out_kk = kk - c;
+                sm->res_bin = (uint32_t)(hi_bin - i);
+                sm->res_kk = kk - c;
+                sm->res_cnt = h;
                 break;
             }
             c += h;
@@ -121,301 +134,554 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t 
     named_bar_sync(1, kEpiThreads);
 }
 
-// Add this CTA's digit histogram (nonzero bins) into the group histogram.
-__device__ __forceinline__ void push_hist(const uint32_t* local, uint32_t* global, int nb) {
-    for (int i = threadIdx.x; i < nb; i += kEpiThreads) {
-        const uint32_t v = local[i];
-        if (v) atomicAdd(global + i, v);
+// Histogram increment; a warp whose lanes all hit one bin (ties) adds once.
+// Called by all 32 lanes of a warp.
+__device__ __forceinline__ void hist_add(uint32_t* hist, bool in, uint32_t bin) {
+    const uint32_t b0 = __shfl_sync(0xffffffffu, bin, 0);
+    if (__all_sync(0xffffffffu, in && bin == b0)) {
+        if ((threadIdx.x & 31) == 0) red_add_shared(hist + b0, 32u);
+    } else if (in) {
+        red_add_shared(hist + bin, 1u);
     }
 }
 
-// Replace the local histogram by the group's: every load in flight at once.
-__device__ __forceinline__ void pull_hist(uint32_t* local, const uint32_t* global, int nb) {
-    constexpr int V = 2048 / (4 * kEpiThreads);   // uint4 per thread for 2048 bins
-    uint4 v[V];
+constexpr int kU = 4;   // keys per thread and loop iteration (independent loads in flight)
+
+// Histogram of the stream's keys in [lo, hi], bin = (key - lo) >> shift.
+template <class Stream>
+__device__ void stream_hist(const Stream& st, uint32_t lo, uint32_t hi, int shift, uint32_t* hist) {
+    const int n = st.size();
+    for (int i0 = 0; i0 < n; i0 += kEpiThreads * kU) {
+        uint32_t k[kU];
 #pragma unroll
-    for (int u = 0; u < V; ++u) {
-        const int i = (u * kEpiThreads + (int)threadIdx.x) * 4;
-        v[u] = i < nb ? __ldcg(reinterpret_cast<const uint4*>(global + i)) : make_uint4(0, 0, 0, 0);
-    }
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+            k[u] = i < n ? st.key(i) : 0u;
+        }
 #pragma unroll
-    for (int u = 0; u < V; ++u) {
-        const int i = (u * kEpiThreads + (int)threadIdx.x) * 4;
-        if (i < nb) *reinterpret_cast<uint4*>(local + i) = v[u];
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+            hist_add(hist, i < n && k[u] >= lo && k[u] <= hi, (k[u] - lo) >> shift);
+        }
     }
 }
 
-// Loads 4 x 32 consecutive scores of a warp's range (lane-strided), keyed.
-struct KeyBatch {
-    uint32_t key[4];
-    bool in[4];
+// Appends the stream's keys in [lo, hi] to dst (any order); sm->fill counts them.
+template <class Stream, class Sink>
+__device__ void stream_collect(const Stream& st, uint32_t lo, uint32_t hi, uint32_t* fill, Sink sink) {
+    const int n = st.size();
+    const int lane = threadIdx.x & 31;
+    for (int i0 = 0; i0 < n; i0 += kEpiThreads * kU) {
+        uint32_t k[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+            k[u] = i < n ? st.key(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+            const bool in = i < n && k[u] >= lo && k[u] <= hi;
+            const uint32_t m = __ballot_sync(0xffffffffu, in);
+            uint32_t at = 0;
+            if (lane == 0 && m) at = atom_add_shared(fill, (uint32_t)__popc(m));
+            at = __shfl_sync(0xffffffffu, at, 0);
+            if (in) sink(at + __popc(m & ((1u << lane) - 1u)), k[u]);
+        }
+    }
+}
+
+// Right shift that maps [lo, hi] onto at most kBins bins.
+__device__ __forceinline__ int range_shift(uint32_t lo, uint32_t hi) {
+    const int bits = 32 - __clz(hi - lo);        // hi - lo < 2^bits
+    return bits > 11 ? bits - 11 : 0;
+}
+
+// Streams of keys with a flat index: this CTA's scores (shared memory floats),
+// published keys loaded into shared memory (ranks padded to 4 with key 0,
+// which no score maps to), or the same read in place from global memory.
+struct ScoreStream {
+    const float* s;
+    int n;
+    __device__ __forceinline__ int size() const { return n; }
+    __device__ __forceinline__ uint32_t key(int i) const { return order_key(s[i]); }
 };
-__device__ __forceinline__ KeyBatch load_keys(const float* s, int i0, int end, int lane) {
-    KeyBatch kb;
-    float f[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * 32 + lane;
-        kb.in[u] = i < end;
-        f[u] = kb.in[u] ? s[i] : 0.0f;
+struct SmemKeyStream {
+    const uint32_t* k;
+    int n;
+    __device__ __forceinline__ int size() const { return n; }
+    __device__ __forceinline__ uint32_t key(int i) const { return k[i]; }
+};
+struct GlobalKeyStream {
+    const uint32_t* rt;        // shared rank table [G] {count, flat offset}
+    const uint32_t* cand;      // slot of rank 0
+    int64_t slot;              // keys between the slots of consecutive ranks
+    int G, n;
+    __device__ __forceinline__ int size() const { return n; }
+    __device__ uint32_t key(int i) const {
+        int lo = 0, hi = G - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if ((int)rt[2 * mid + 1] <= i) lo = mid; else hi = mid - 1;
+        }
+        const uint32_t e = (uint32_t)i - rt[2 * lo + 1];
+        return e < rt[2 * lo] ? __ldcg(cand + lo * slot + e) : 0u;
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) kb.key[u] = order_key(f[u]);
-    return kb;
+};
+
+// Exact kk-th largest key among the n keys in `list` (radix select, 8-bit
+// digits); uses hist[0..255].
+__device__ uint32_t list_select(const uint32_t* list, int n, uint32_t kk, uint32_t* hist, SelectSmem* sm) {
+    uint32_t prefix = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = threadIdx.x; i < 256; i += kEpiThreads) hist[i] = 0u;
+        named_bar_sync(1, kEpiThreads);
+        const uint32_t hmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+        for (int i0 = 0; i0 < n; i0 += kEpiThreads) {
+            const int i = i0 + (int)threadIdx.x;
+            const uint32_t key = i < n ? list[i] : 0u;
+            const bool in = i < n && (key & hmask) == (prefix & hmask);
+            hist_add(hist, in, (key >> shift) & 255u);
+        }
+        named_bar_sync(1, kEpiThreads);
+        find_bin(hist, 256, kk, sm);
+        prefix |= sm->res_bin << shift;
+        kk = sm->res_kk;
+    }
+    return prefix;
+}
+
+// The kk-th largest key of the stream among its keys in [lo, hi] (kk no more
+// than their count): range histograms, then the exact step on the short list
+// of the final bin.
+template <class Stream>
+__device__ uint32_t find_threshold(const Stream& st, uint32_t lo, uint32_t hi, uint32_t kk, uint32_t* hist,
+                                   uint32_t* list, SelectSmem* sm) {
+    while (lo != hi) {
+        const int shift = range_shift(lo, hi);
+        for (int i = threadIdx.x; i < kBins; i += kEpiThreads) hist[i] = 0u;
+        named_bar_sync(1, kEpiThreads);
+        stream_hist(st, lo, hi, shift, hist);
+        named_bar_sync(1, kEpiThreads);
+        find_bin(hist, kBins, kk, sm);
+        const uint32_t b = sm->res_bin, cnt = sm->res_cnt;
+        kk = sm->res_kk;
+        const uint32_t blo = lo + (b << shift);
+        if (shift == 0) return blo;                       // the bin is one key
+        const uint32_t bhi = min(hi, blo + ((1u << shift) - 1u));
+        if (cnt <= (uint32_t)kListCap) {
+            if (threadIdx.x == 0) sm->fill = 0u;
+            named_bar_sync(1, kEpiThreads);
+            stream_collect(st, blo, bhi, &sm->fill, [&](uint32_t at, uint32_t key) { list[at] = key; });
+            named_bar_sync(1, kEpiThreads);
+            return list_select(list, (int)cnt, kk, hist, sm);
+        }
+        lo = blo;
+        hi = bhi;
+    }
+    return lo;
 }
 
 struct GroupView {
     uint32_t* sync;     // {count, gen}
-    uint32_t* hist;     // [3][NQ][2048]
-    uint32_t* cnt;      // [ranks][NQ][2]
+    uint32_t* hdr;      // [ranks][NQ][4]: published count, smallest published key, largest key, edge
+    uint32_t* cand;     // published keys: slot of the group's first CTA
     int G, rank;
 };
 
 // Exact Top-K of NQ tokens' score rows held in shared memory (s_score, token
 // j at j*stride, nloc[j] valid entries starting at position chunk0).
 // Writes out_idx/out_score rows [t0 + j] in ascending position order.
-// Called by the 128 select threads; the pass-0 (top 11 bits) histogram of
-// every visible element must already be in s_hist[j*2048 ...].
+// Called by the 128 select threads; sm->kmin/kmax[j] hold the smallest and
+// largest key of the visible scores.  s_hist holds kBins words, s_list
+// kListCap; `scratch` (scratch_bytes, 16-byte aligned) is shared memory that
+// is free in grouped work (the key stages).
 template <int NQ>
 __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_t& gen, float* s_score,
                             int stride, const int (&nloc)[NQ], const bool (&active)[NQ], int64_t chunk0,
-                            int64_t t0, uint32_t* s_hist, uint16_t* s_list, SelectSmem* sm, volatile int* abort) {
+                            int64_t t0, uint32_t* s_hist, uint32_t* s_list, uint8_t* scratch, int scratch_bytes,
+                            SelectSmem* sm, volatile int* abort) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lt_mask = (1u << lane) - 1u;
-    uint32_t prefix[NQ], kk[NQ];
-#pragma unroll
-    for (int j = 0; j < NQ; ++j) { prefix[j] = 0; kk[j] = (uint32_t)p.K; }
-    // per-warp running counts of elements above the (partial) threshold
-    uint32_t wgt[NQ];
-#pragma unroll
-    for (int j = 0; j < NQ; ++j) wgt[j] = 0;
+    const uint32_t K = (uint32_t)p.K;
+    const int G = gv.G;
+    const int64_t slot_keys = p.cand_slot / NQ;
 
-    auto quarter = [&](int j, int& beg, int& end) {
-        const int qlen = ((nloc[j] + 4 * 32 - 1) / (4 * 32)) * 32;
-        beg = warp * qlen;
-        end = min(nloc[j], beg + qlen);
+    // warp w owns the w-th quarter of a token's elements (quarters are multiples of 32)
+    int qlen[NQ], list_off[NQ];
+    int list_words = 0;     // u16 entries of all per-warp lists
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+        qlen[j] = ((nloc[j] + 4 * 32 - 1) / (4 * 32)) * 32;
+        list_off[j] = list_words;
+        list_words += 4 * qlen[j];
+    }
+    // Grouped work keeps, per warp, the position-ordered list of its published
+    // elements (a superset of its selected ones) when the lists take at most
+    // half of the scratch; otherwise its whole quarter is scanned again.
+    const int list_bytes = ((list_words * 2 + 15) / 16) * 16;
+    const bool lists = G > 1 && 2 * list_bytes <= scratch_bytes;
+    uint16_t* s_lists = reinterpret_cast<uint16_t*>(scratch);
+    uint8_t* gscratch = scratch + (lists ? list_bytes : 0);
+    const int gscratch_bytes = scratch_bytes - (lists ? list_bytes : 0);
+
+    // The n-th element of warp `warp`'s sequence for token j: in list mode the
+    // listed local indices, otherwise its quarter.
+    auto seq_len = [&](int j) -> int {
+        if (lists) return (int)sm->wpub[j][warp];
+        const int beg = warp * qlen[j];
+        return max(0, min(nloc[j], beg + qlen[j]) - beg);
+    };
+    auto seq_idx = [&](int j, int t) -> int {
+        return lists ? (int)s_lists[list_off[j] + warp * qlen[j] + t] : warp * qlen[j] + t;
     };
 
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int nb = pass == 2 ? 1024 : 2048;
-        if (pass > 0) {
-            for (int i = threadIdx.x; i < NQ * 2048; i += kEpiThreads) s_hist[i] = 0u;
-            named_bar_sync(1, kEpiThreads);
+    // ---- publication (grouped work)
+    auto my_slot = [&](int j) { return gv.cand + (int64_t)gv.rank * p.cand_slot + j * slot_keys; };
+    // per-warp counts (and lists) of the elements with key >= edge
+    auto build = [&](int j, uint32_t edge) {
+        const float* sj = s_score + j * stride;
+        const int beg = warp * qlen[j];
+        const int end = min(nloc[j], beg + qlen[j]);
+        uint16_t* lw = s_lists + list_off[j] + warp * qlen[j];
+        uint32_t n = 0;
+        for (int i0 = beg; i0 < end; i0 += 32 * kU) {
+            uint32_t k[kU];
 #pragma unroll
-            for (int j = 0; j < NQ; ++j) {
-                if (!active[j]) continue;
-                const float* sj = s_score + j * stride;
-                uint32_t* hj = s_hist + j * 2048;
-                int beg, end;
-                quarter(j, beg, end);
-                uint32_t gt = 0, n_list = 0;
-                uint16_t* wl = s_list + (j * 4 + warp) * kListCap;
-                // pass 1: match the first digit; pass 2: match the first two digits
-                const int mshift = pass == 1 ? 21 : 10;
-                const uint32_t want = prefix[j] >> mshift;
-                const uint32_t d1 = prefix[j] >> 21;
-                for (int i0 = beg; i0 < end; i0 += 128) {
-                    const KeyBatch kb = load_keys(sj, i0, end, lane);
+            for (int u = 0; u < kU; ++u) {
+                const int i = i0 + u * 32 + lane;
+                k[u] = i < end ? order_key(sj[i]) : 0u;
+            }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t hi = kb.key[u] >> mshift;
-                        // above the threshold at this digit, and not already counted at the previous one
-                        const bool above = hi > want && (pass == 1 || (kb.key[u] >> 21) == d1);
-                        gt += __popc(__ballot_sync(0xffffffffu, kb.in[u] && above));
-                        const bool match = kb.in[u] && hi == want;
-                        if (match) atomicAdd(hj + ((kb.key[u] >> shift) & (nb - 1)), 1u);
-                        if (pass == 2) {
-                            const uint32_t mm = __ballot_sync(0xffffffffu, match);
-                            const uint32_t at = n_list + __popc(mm & lt_mask);
-                            if (match && at < kListCap) wl[at] = (uint16_t)(i0 + u * 32 + lane);
-                            n_list += __popc(mm);
+            for (int u = 0; u < kU; ++u) {
+                const int i = i0 + u * 32 + lane;
+                const bool in = i < end && k[u] >= edge;
+                const uint32_t m = __ballot_sync(0xffffffffu, in);
+                if (lists && in) lw[n + __popc(m & lt_mask)] = (uint16_t)i;
+                n += __popc(m);
+            }
+        }
+        if (lane == 0) sm->wpub[j][warp] = n;
+    };
+    // publish token j's elements >= edge (after build): keys in warp order, header
+    auto publish = [&](int j, uint32_t edge) {
+        build(j, edge);
+        if (threadIdx.x == 0) sm->cmin = 0xFFFFFFFFu;
+        named_bar_sync(1, kEpiThreads);
+        const float* sj = s_score + j * stride;
+        uint32_t off = 0, tot = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            if (w < warp) off += sm->wpub[j][w];
+            tot += sm->wpub[j][w];
+        }
+        uint32_t* slot = my_slot(j) + off;
+        uint32_t kmn = 0xFFFFFFFFu;
+        if (lists) {
+            const uint16_t* lw = s_lists + list_off[j] + warp * qlen[j];
+            const int n = (int)sm->wpub[j][warp];
+            for (int q0 = 0; q0 < n; q0 += 32 * kU) {
+                uint32_t k[kU];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int t = q0 + u * 32 + lane;
+                    k[u] = t < n ? order_key(sj[lw[t]]) : 0xFFFFFFFFu;
+                }
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int t = q0 + u * 32 + lane;
+                    if (t < n) __stcg(slot + t, k[u]);
+                    kmn = min(kmn, k[u]);
+                }
+            }
+        } else {
+            const int beg = warp * qlen[j];
+            const int end = min(nloc[j], beg + qlen[j]);
+            uint32_t o = 0;
+            for (int i0 = beg; i0 < end; i0 += 32) {
+                const int i = i0 + lane;
+                const uint32_t key = i < end ? order_key(sj[i]) : 0u;
+                const bool in = i < end && key >= edge;
+                const uint32_t m = __ballot_sync(0xffffffffu, in);
+                if (in) {
+                    __stcg(slot + o + __popc(m & lt_mask), key);
+                    kmn = min(kmn, key);
+                }
+                o += __popc(m);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+        if (lane == 0) red_min_shared(&sm->cmin, kmn);
+        named_bar_sync(1, kEpiThreads);
+        if (threadIdx.x == 0) {
+            sm->edge[j] = edge;
+            uint32_t* h = gv.hdr + ((int64_t)gv.rank * NQ + j) * 4;
+            __stcg(reinterpret_cast<uint4*>(h), make_uint4(tot, sm->cmin, sm->kmax[j], edge));
+        }
+        named_bar_sync(1, kEpiThreads);
+    };
+
+    // rank table and (if they fit) all published keys of token j in shared memory
+    uint32_t* rt = reinterpret_cast<uint32_t*>(gscratch);
+    uint32_t* keys = rt + ((2 * G + 3) & ~3);
+    auto gather = [&](int j) {
+        if (threadIdx.x == 0) {
+            uint32_t lo = 0xFFFFFFFFu, hi = 0u, off = 0u, emax = 0u;
+            for (int r = 0; r < G; ++r) {
+                const uint4 h = __ldcg(reinterpret_cast<const uint4*>(gv.hdr + ((int64_t)r * NQ + j) * 4));
+                rt[2 * r] = h.x;
+                rt[2 * r + 1] = off;
+                off += (h.x + 3u) & ~3u;
+                if (h.x) {
+                    lo = min(lo, h.y);
+                    hi = max(hi, h.z);
+                }
+                emax = max(emax, h.w);
+            }
+            sm->g_lo = lo;
+            sm->g_hi = hi;
+            sm->g_total = off;
+            sm->g_max_edge = emax;
+            sm->g_resident = (int64_t)((2 * G + 3) & ~3) * 4 + (int64_t)off * 4 <= (int64_t)gscratch_bytes;
+        }
+        named_bar_sync(1, kEpiThreads);
+        if (sm->g_resident) {
+            // the scratch last held TMA-written key tiles
+            fence_proxy_async_smem();
+            // 16-byte vectors of the concatenated (padded) ranks, eight loads in
+            // flight per thread; vector v belongs to the rank whose offset range holds 4v
+            const int nv = (int)(sm->g_total >> 2);
+            for (int v0 = 0; v0 < nv; v0 += kEpiThreads * 8) {
+                uint4 x[8];
+                uint32_t cnt[8], e4[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int v = v0 + u * kEpiThreads + (int)threadIdx.x;
+                    x[u] = make_uint4(0, 0, 0, 0);
+                    cnt[u] = 0;
+                    e4[u] = 0;
+                    if (v < nv) {
+                        int lo = 0, hi = G - 1;
+                        while (lo < hi) {
+                            const int mid = (lo + hi + 1) >> 1;
+                            if (rt[2 * mid + 1] <= 4u * (uint32_t)v) lo = mid; else hi = mid - 1;
                         }
+                        cnt[u] = rt[2 * lo];
+                        e4[u] = 4u * (uint32_t)v - rt[2 * lo + 1];
+                        const uint32_t* src = gv.cand + (int64_t)lo * p.cand_slot + j * slot_keys;
+                        x[u] = __ldcg(reinterpret_cast<const uint4*>(src + e4[u]));
                     }
                 }
-                wgt[j] += gt;
-                if (pass == 2 && lane == 0) sm->list_n[j][warp] = n_list;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int v = v0 + u * kEpiThreads + (int)threadIdx.x;
+                    if (v < nv) {
+                        const uint32_t e = e4[u], n = cnt[u];   // keys past the count read as 0
+                        uint4 y = x[u];
+                        if (e + 1u > n) y.x = 0u;
+                        if (e + 2u > n) y.y = 0u;
+                        if (e + 3u > n) y.z = 0u;
+                        if (e + 4u > n) y.w = 0u;
+                        *reinterpret_cast<uint4*>(keys + 4 * v) = y;
+                    }
+                }
             }
             named_bar_sync(1, kEpiThreads);
         }
-        if (gv.G > 1) {
-            uint32_t* gh = gv.hist + pass * NQ * 2048;
-#pragma unroll
-            for (int j = 0; j < NQ; ++j)
-                if (active[j]) push_hist(s_hist + j * 2048, gh + j * 2048, nb);
-            if (!group_barrier(gv.sync, gv.G, gen, p.status, abort)) return false;
-#pragma unroll
-            for (int j = 0; j < NQ; ++j)
-                if (active[j]) pull_hist(s_hist + j * 2048, gh + j * 2048, nb);
-            // the histogram of the previous pass has been read by every CTA
-            if (gv.rank == 0 && pass > 0) {
-                uint32_t* prev = gv.hist + (pass - 1) * NQ * 2048;
-                for (int i = threadIdx.x * 4; i < NQ * 2048; i += kEpiThreads * 4)
-                    *reinterpret_cast<uint4*>(prev + i) = make_uint4(0, 0, 0, 0);
-            }
-            named_bar_sync(1, kEpiThreads);
-        }
+    };
+    auto group_T = [&](int j) -> uint32_t {
+        if (sm->g_resident)
+            return find_threshold(SmemKeyStream{keys, (int)sm->g_total}, sm->g_lo, sm->g_hi, K, s_hist, s_list, sm);
+        return find_threshold(GlobalKeyStream{rt, gv.cand + j * slot_keys, p.cand_slot, G, (int)sm->g_total},
+                              sm->g_lo, sm->g_hi, K, s_hist, s_list, sm);
+    };
+
+    if (G > 1) {
+        // ---- 1. publish: the keys at or above an estimate of the local c-th
+        // largest, c about twice this CTA's expected share of the Top-K.  The
+        // estimate is the matching rank of a strided sample of 512 scores,
+        // with 25% slack; a low estimate only costs the second round.
+        const uint32_t c = min(K, 2u * K / (uint32_t)G + 32u);
 #pragma unroll
         for (int j = 0; j < NQ; ++j) {
             if (!active[j]) continue;
-            find_bin(s_hist + j * 2048, nb, kk[j], sm->scan, &sm->sel_bin[j], &sm->sel_kk[j]);
-            prefix[j] |= sm->sel_bin[j] << shift;
-            kk[j] = sm->sel_kk[j];
+            uint32_t edge = 0u;      // publish every key
+            if (nloc[j] > (int)c && sm->kmin[j] != sm->kmax[j]) {
+                const float* sj = s_score + j * stride;
+                const int S = min(nloc[j], 512);
+                const int step = nloc[j] / S;
+                for (int i = threadIdx.x; i < S; i += kEpiThreads) s_list[i] = order_key(sj[i * step]);
+                named_bar_sync(1, kEpiThreads);
+                const uint64_t want = ((uint64_t)c * 5u * (uint64_t)S) / (4u * (uint64_t)nloc[j]) + 8u;
+                const uint32_t r = want < (uint64_t)S ? (uint32_t)want : (uint32_t)S;
+                edge = list_select(s_list, S, r, s_hist, sm);
+            }
+            publish(j, edge);
         }
-        if (threadIdx.x == 0) DSA_TRACE_MARK(3 + pass);
+        if (threadIdx.x == 0) DSA_TRACE_MARK(3);
+        if (!group_barrier(gv.sync, G, gen, p.status, abort)) return false;
+        if (threadIdx.x == 0) DSA_TRACE_MARK(4);
     }
 
-    // ---- per-warp counts above / equal to the exact threshold T = prefix
-    bool overflow = false;
-#pragma unroll
-    for (int j = 0; j < NQ; ++j)
-        if (active[j])
-            for (int w = 0; w < 4; ++w) overflow |= sm->list_n[j][w] > (uint32_t)kListCap;
 #pragma unroll
     for (int j = 0; j < NQ; ++j) {
-        uint32_t gt = 0, eq = 0;
-        if (active[j]) {
-            const float* sj = s_score + j * stride;
-            if (!overflow) {
-                const uint16_t* wl = s_list + (j * 4 + warp) * kListCap;
-                const uint32_t n = sm->list_n[j][warp];
-                for (uint32_t i = lane; i < n; i += 32) {
-                    const uint32_t key = order_key(sj[wl[i]]);
-                    gt += key > prefix[j];
-                    eq += key == prefix[j];
+        if (!active[j]) continue;
+        const float* sj = s_score + j * stride;
+        uint32_t T, take = 0, base = 0;
+        if (G == 1) {
+            // ---- exact threshold over this CTA's own scores
+            T = find_threshold(ScoreStream{sj, nloc[j]}, sm->kmin[j], sm->kmax[j], K, s_hist, s_list, sm);
+        } else {
+            // ---- 2. threshold over the published keys
+            gather(j);
+            if (threadIdx.x == 0) DSA_TRACE_MARK(13);
+            T = group_T(j);
+            if (threadIdx.x == 0) DSA_TRACE_MARK(14);
+            if (sm->g_max_edge > T) {
+                // some CTA held more than it published (every CTA sees the same
+                // keys, so all take this branch): once every CTA has read the
+                // first publication, the CTAs whose edge is above T publish all
+                // their keys >= T, and the threshold of the enlarged set is exact
+                const uint32_t t1 = T;
+                if (!group_barrier(gv.sync, G, gen, p.status, abort)) return false;
+                if (sm->edge[j] > t1) publish(j, t1);
+                if (!group_barrier(gv.sync, G, gen, p.status, abort)) return false;
+                gather(j);
+                T = group_T(j);
+            }
+            // ---- 3. lower ranks' published keys above / equal to T (warp w takes ranks w, w+4, ...)
+            uint32_t gt_b = 0, eq_b = 0, gt_all = 0;
+            const bool res = sm->g_resident;
+            const GlobalKeyStream gs{rt, gv.cand + j * slot_keys, p.cand_slot, G, (int)sm->g_total};
+            for (int r = warp; r < G; r += 4) {
+                const uint32_t n = rt[2 * r], off = rt[2 * r + 1];
+                uint32_t g = 0, e = 0;
+                for (uint32_t i0 = 0; i0 < n; i0 += 32 * kU) {
+                    uint32_t k[kU];
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        const uint32_t i = i0 + u * 32 + lane;
+                        k[u] = i < n ? (res ? keys[off + i] : gs.key((int)(off + i))) : 0u;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        g += k[u] > T;
+                        e += k[u] == T;
+                    }
                 }
 #pragma unroll
                 for (int o = 16; o; o >>= 1) {
-                    gt += __shfl_xor_sync(0xffffffffu, gt, o);
-                    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+                    g += __shfl_xor_sync(0xffffffffu, g, o);
+                    e += __shfl_xor_sync(0xffffffffu, e, o);
                 }
-                gt += wgt[j];
-            } else {
-                // too many ties near the threshold for the lists: count directly
-                int beg, end;
-                quarter(j, beg, end);
-                for (int i0 = beg; i0 < end; i0 += 128) {
-                    const KeyBatch kb = load_keys(sj, i0, end, lane);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        gt += __popc(__ballot_sync(0xffffffffu, kb.in[u] && kb.key[u] > prefix[j]));
-                        eq += __popc(__ballot_sync(0xffffffffu, kb.in[u] && kb.key[u] == prefix[j]));
-                    }
+                gt_all += g;
+                if (r < gv.rank) {
+                    gt_b += g;
+                    eq_b += e;
                 }
             }
             if (lane == 0) {
-                sm->wcnt[j][warp][0] = gt;
-                sm->wcnt[j][warp][1] = eq;
+                sm->wcnt[warp][0] = gt_b;
+                sm->wcnt[warp][1] = eq_b;
+                sm->wallow[warp] = gt_all;
+            }
+            named_bar_sync(1, kEpiThreads);
+            uint32_t gtb = 0, eqb = 0, gta = 0;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                gtb += sm->wcnt[w][0];
+                eqb += sm->wcnt[w][1];
+                gta += sm->wallow[w];
+            }
+            named_bar_sync(1, kEpiThreads);
+            // K - (keys above T) tied keys are taken, lowest ranks first
+            const uint32_t need_eq = K - gta;
+            base = gtb + min(need_eq, eqb);
+            take = need_eq > eqb ? need_eq - eqb : 0u;
+        }
+        if (threadIdx.x == 0) DSA_TRACE_MARK(5);
+
+        // ---- per-warp counts of this CTA's elements above / equal to T, over
+        // the warp's position-ordered sequence (list or quarter)
+        const int n = seq_len(j);
+        uint32_t gt = 0, eq = 0;
+        for (int q0 = 0; q0 < n; q0 += 32 * kU) {
+            uint32_t k[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int t = q0 + u * 32 + lane;
+                k[u] = t < n ? order_key(sj[seq_idx(j, t)]) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int t = q0 + u * 32 + lane;
+                gt += __popc(__ballot_sync(0xffffffffu, t < n && k[u] > T));
+                eq += __popc(__ballot_sync(0xffffffffu, t < n && k[u] == T));
             }
         }
-    }
-    named_bar_sync(1, kEpiThreads);
-    uint32_t cgt[NQ], ceq[NQ], gt_before[NQ], eq_before[NQ], weq[NQ];
+        if (lane == 0) {
+            sm->wcnt[warp][0] = gt;
+            sm->wcnt[warp][1] = eq;
+        }
+        named_bar_sync(1, kEpiThreads);
+        uint32_t gt_before = 0, eq_before = 0, cgt = 0, ceq = 0, weq = 0;
 #pragma unroll
-    for (int j = 0; j < NQ; ++j) {
-        cgt[j] = ceq[j] = gt_before[j] = eq_before[j] = weq[j] = 0;
-        if (!active[j]) continue;
         for (int w = 0; w < 4; ++w) {
-            const uint32_t g = sm->wcnt[j][w][0], e = sm->wcnt[j][w][1];
-            if (w < warp) { gt_before[j] += g; eq_before[j] += e; }
-            if (w == warp) weq[j] = e;
-            cgt[j] += g;
-            ceq[j] += e;
-        }
-    }
-    uint32_t take[NQ], base[NQ];
-#pragma unroll
-    for (int j = 0; j < NQ; ++j) { take[j] = min(kk[j], ceq[j]); base[j] = 0; }
-    if (gv.G > 1) {
-        // split the tied elements (lowest positions first, i.e. lower ranks
-        // first) and the output offsets across the group
-        if (threadIdx.x == 0) {
-#pragma unroll
-            for (int j = 0; j < NQ; ++j) {
-                if (!active[j]) continue;
-                __stcg(gv.cnt + (gv.rank * NQ + j) * 2, cgt[j]);
-                __stcg(gv.cnt + (gv.rank * NQ + j) * 2 + 1, ceq[j]);
+            const uint32_t g = sm->wcnt[w][0], e = sm->wcnt[w][1];
+            if (w < warp) {
+                gt_before += g;
+                eq_before += e;
             }
+            if (w == warp) weq = e;
+            cgt += g;
+            ceq += e;
         }
-        if (!group_barrier(gv.sync, gv.G, gen, p.status, abort)) return false;
-        // counts of the lower ranks: loaded by many threads at once into shared
-        // memory (the histogram area is free now), then combined in rank order
-        // by one thread, because the tie split depends on the running total
-        uint2* cnt_s = reinterpret_cast<uint2*>(s_hist);
-        for (int i = threadIdx.x; i < gv.rank * NQ; i += kEpiThreads)
-            cnt_s[i] = __ldcg(reinterpret_cast<const uint2*>(gv.cnt) + i);
+        if (G == 1) take = K - cgt;          // this CTA holds every element
+        take = min(take, ceq);
+        if (threadIdx.x == 0) DSA_TRACE_MARK(6);
+        // ---- this warp's share of the tied elements, output offsets
+        const uint32_t allow = take > eq_before ? min(take - eq_before, weq) : 0u;
         named_bar_sync(1, kEpiThreads);
-        if (threadIdx.x == 0) {
-#pragma unroll
-            for (int j = 0; j < NQ; ++j) {
-                if (!active[j]) continue;
-                uint32_t eqb = 0, ob = 0;
-                for (int r = 0; r < gv.rank; ++r) {
-                    const uint2 c = cnt_s[r * NQ + j];
-                    ob += c.x + (kk[j] > eqb ? min(kk[j] - eqb, c.y) : 0u);
-                    eqb += c.y;
-                }
-                sm->sel_take[j] = kk[j] > eqb ? min(kk[j] - eqb, ceq[j]) : 0u;
-                sm->sel_base[j] = ob;
-            }
-        }
-        if (gv.rank == 0) {
-            // every CTA of the group has read the last pass's histogram
-            uint32_t* last = gv.hist + 2 * NQ * 2048;
-            for (int i = threadIdx.x * 4; i < NQ * 2048; i += kEpiThreads * 4)
-                *reinterpret_cast<uint4*>(last + i) = make_uint4(0, 0, 0, 0);
-        }
+        if (lane == 0) sm->wallow[warp] = allow;
         named_bar_sync(1, kEpiThreads);
-#pragma unroll
-        for (int j = 0; j < NQ; ++j) {
-            take[j] = sm->sel_take[j];
-            base[j] = sm->sel_base[j];
-        }
-    }
-    if (threadIdx.x == 0) DSA_TRACE_MARK(6);
-    // ---- this warp's share of the tied elements, output offsets
-    uint32_t allow[NQ];
-#pragma unroll
-    for (int j = 0; j < NQ; ++j) {
-        allow[j] = take[j] > eq_before[j] ? min(take[j] - eq_before[j], weq[j]) : 0u;
-        if (lane == 0) sm->wallow[j][warp] = allow[j];
-    }
-    named_bar_sync(1, kEpiThreads);
-    // ---- emission in ascending position order
-#pragma unroll
-    for (int j = 0; j < NQ; ++j) {
-        if (!active[j]) continue;
-        uint32_t out = base[j] + gt_before[j];
-        for (int w = 0; w < warp; ++w) out += sm->wallow[j][w];
-        int beg, end;
-        quarter(j, beg, end);
-        const float* sj = s_score + j * stride;
+        // ---- emission in ascending position order
+        uint32_t out = base + gt_before;
+        for (int w = 0; w < warp; ++w) out += sm->wallow[w];
         int32_t* oi = p.out_idx + (t0 + j) * p.K;
         float* os = p.out_score ? p.out_score + (t0 + j) * p.K : nullptr;
         uint32_t eq_seen = 0;
-        for (int i0 = beg; i0 < end; i0 += 128) {
-            const KeyBatch kb = load_keys(sj, i0, end, lane);
+        for (int q0 = 0; q0 < n; q0 += 32 * kU) {
+            float f[kU];
+            int ix[kU];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const bool is_gt = kb.in[u] && kb.key[u] > prefix[j];
-                const bool is_eq = kb.in[u] && kb.key[u] == prefix[j];
+            for (int u = 0; u < kU; ++u) {
+                const int t = q0 + u * 32 + lane;
+                ix[u] = t < n ? seq_idx(j, t) : 0;
+                f[u] = t < n ? sj[ix[u]] : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int t = q0 + u * 32 + lane;
+                const uint32_t key = order_key(f[u]);
+                const bool is_gt = t < n && key > T;
+                const bool is_eq = t < n && key == T;
                 const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
-                const bool sel = is_gt || (is_eq && eq_seen + __popc(eqm & lt_mask) < allow[j]);
+                const bool sel = is_gt || (is_eq && eq_seen + __popc(eqm & lt_mask) < allow);
                 const uint32_t selm = __ballot_sync(0xffffffffu, sel);
                 if (sel) {
                     const uint32_t o = out + __popc(selm & lt_mask);
-                    if (o < (uint32_t)p.K) {
-                        const int i = i0 + u * 32 + lane;
-                        oi[o] = (int32_t)(chunk0 + i);
-                        if (os) os[o] = sj[i];
+                    if (o < K) {
+                        oi[o] = (int32_t)(chunk0 + ix[u]);
+                        if (os) os[o] = f[u];
                     }
                 }
                 out += __popc(selm);
                 eq_seen += __popc(eqm);
             }
         }
+        named_bar_sync(1, kEpiThreads);
     }
-    named_bar_sync(1, kEpiThreads);
     return true;
 }
 

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     sfa_decode_kernel(const __grid_constant__ SfaParams p, const __grid_constant__ CUtensorMap tm_q) {
     using Cfg = SfaCfg;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = align_shared(smem_raw, 1024);
     uint8_t* s_q = smem + Cfg::OFF_Q;
     uint8_t* s_kv = smem + Cfg::OFF_KV;
     uint8_t* s_p = smem + Cfg::OFF_P;

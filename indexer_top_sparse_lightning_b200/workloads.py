@@ -175,7 +175,8 @@ def _quantize_fp8_groups(x: np.ndarray, group: int = 64):
 
 def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=128, K=2048,
                   key_dtype="bf16", int_inputs=False, w_dist="u8", shuffle=True,
-                  planted_k: int = 0, seed: int = 0, with_kv: bool = True) -> Workload:
+                  planted_k: int = 0, planted_tail: bool = False, seed: int = 0,
+                  with_kv: bool = True) -> Workload:
     """Draw one synthetic step.
 
     seq_lens: per-sequence cached lengths (including the step's own tokens).
@@ -183,7 +184,8 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
     w_dist: "u8" -> U(0,1)/sqrt(H_I); "u" -> U(0,1); "u256" -> U(0,1) rounded to 2^-8;
             "ones" -> all 1 (integer scores with many ties when int_inputs is set).
     int_inputs: indexer q/k drawn as integers in [-4, 4] (exact fp32 scores).
-    planted_k: if > 0 (single sequence), plant a dominant set of that many positions.
+    planted_k: if > 0 (single sequence, one token), plant a dominant set of that many
+               positions: seed-chosen, or the last planted_k positions if planted_tail.
     """
     seq_lens = np.asarray(seq_lens, dtype=np.int32)
     B = int(seq_lens.shape[0])
@@ -214,27 +216,35 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
     r = _rng(seed, 4)
     n_keys = num_blocks * BLOCK
     planted = None
+    plant_rows = plant_vals = None
+    if planted_k:
+        # keys along the query's head-weighted direction, far above the N(0,1) keys
+        assert B == 1 and T == 1
+        rp = _rng(seed, 5)
+        L = int(seq_lens[0])
+        if planted_tail:
+            planted = np.arange(L - planted_k, L, dtype=np.int64)
+        else:
+            planted = np.sort(rp.choice(L, size=planted_k, replace=False)).astype(np.int64)
+        qf = bf16_bits_to_f32(q_idx[0]).astype(np.float64)          # [H_I, D_I]
+        dirn = (w[0].astype(np.float64)[:, None] * qf).sum(axis=0)
+        dirn /= np.linalg.norm(dirn)
+        alpha = 4.0 * math.sqrt(D_I)
+        plant_rows = table[0, planted // BLOCK].astype(np.int64) * BLOCK + planted % BLOCK
+        plant_vals = (alpha * dirn[None, :] + 0.1 * rp.standard_normal((planted_k, D_I))).astype(np.float32)
     if key_dtype == "bf16":
         if int_inputs:
             k_f = r.integers(-4, 5, size=(n_keys, D_I)).astype(np.float32)
             k_idx = to_bf16_bits(k_f).reshape(num_blocks, BLOCK, D_I)
         else:
             k_idx = _normal_bf16(seed, 4, (num_blocks, BLOCK, D_I))
+        if planted_k:
+            k_idx.reshape(n_keys, D_I)[plant_rows] = to_bf16_bits(plant_vals)
         k_scale = None
     else:
         k_f = r.standard_normal((n_keys, D_I), dtype=np.float32)
         if planted_k:
-            assert B == 1 and T == 1
-            rp = _rng(seed, 5)
-            L = int(seq_lens[0])
-            planted = np.sort(rp.choice(L, size=planted_k, replace=False)).astype(np.int64)
-            qf = bf16_bits_to_f32(q_idx[0]).astype(np.float64)          # [H_I, D_I]
-            dirn = (w[0].astype(np.float64)[:, None] * qf).sum(axis=0)
-            dirn /= np.linalg.norm(dirn)
-            alpha = 4.0 * math.sqrt(D_I)
-            phys = table[0, planted // BLOCK].astype(np.int64) * BLOCK + planted % BLOCK
-            noise = rp.standard_normal((planted_k, D_I))
-            k_f[phys] = (alpha * dirn[None, :] + 0.1 * noise).astype(np.float32)
+            k_f[plant_rows] = plant_vals
         codes, scale = _quantize_fp8_groups(k_f, 64)
         k_idx = codes.reshape(num_blocks, BLOCK, D_I)
         k_scale = scale.reshape(num_blocks, BLOCK, D_I // 64)

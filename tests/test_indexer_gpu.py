@@ -32,6 +32,17 @@ def test_tie_heavy_groups_split_ties_by_position():
     assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
 
 
+@pytest.mark.parametrize("key_dtype", ["bf16", "fp8"])
+def test_topk_concentrated_in_few_ctas(key_dtype):
+    # the whole Top-K in the last 2048 positions: the CTAs holding them publish
+    # too few keys at first and the group needs its second round
+    wl = W.make_workload("tail", seq_lens=[32768], nq=1, H_I=64, D_I=128, H=1, K=2048, key_dtype=key_dtype,
+                         planted_k=2048, planted_tail=True, seed=11, with_kv=False)
+    idx, score = run_indexer(wl)
+    np.testing.assert_array_equal(idx[0], wl.planted.astype(np.int32))
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
 @pytest.mark.parametrize("H_I,D_I", [(64, 128), (32, 64), (16, 128), (8, 128)])
 def test_bf16_decode_ragged_tails(H_I, D_I):
     wl = W.make_workload("small", seq_lens=[1000, 5000, 9999], nq=1, H_I=H_I, D_I=D_I, H=1, K=512, seed=3,
