@@ -23,7 +23,7 @@ namespace {
 
 constexpr size_t kStatusBytes = 256;
 constexpr int kMaxSplitTokens = 128;      // row splits are only used for fewer tokens than this
-constexpr size_t kCounterBytes = kMaxSplitTokens * 2 * 4;
+constexpr size_t kCounterBytes = kMaxSplitTokens * 2 * 2 * 4;   // split arrivals and ready counts
 constexpr size_t kHeaderBytes = kStatusBytes + kCounterBytes;
 
 // ------------------------------------------------------------------ last failure text (per host thread)
@@ -372,6 +372,7 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
         p.part_o = reinterpret_cast<float*>(part);
         p.part_ml = reinterpret_cast<float*>(part + (size_t)bt->num_tokens * ap.splits * 128 * kDv * 4);
         p.split_count = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(status) + kStatusBytes);
+        p.split_ready = p.split_count + kMaxSplitTokens * 2;
     }
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof cfg);

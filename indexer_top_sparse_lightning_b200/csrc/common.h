@@ -77,9 +77,10 @@ struct SfaParams {
     const int32_t* idx;       // [T, K]
     uint16_t* out;            // [T, H, 512] bf16 bits
     float* lse;               // [T, H] or null
-    float* part_o;            // split partials: [T, S, 128 heads, 512] (un-normalised)
-    float* part_ml;           // [T, S, 2 halves, 2, 128] (m in log2 domain, l)
+    float* part_o;            // split partials: [T, S, 2 head halves, 512 columns, 64 heads] (un-normalised)
+    float* part_ml;           // [T, S, 2 head halves, 64 heads, 2] (m in log2 domain, l)
     uint32_t* split_count;    // [T, 2 halves] arrivals; zero between calls
+    uint32_t* split_ready;    // [T, 2 halves] partials written; zero between calls
     uint32_t* status;
     int32_t B, T, H, K, max_blocks, num_blocks;
     int32_t n_splits, rows_per_split;

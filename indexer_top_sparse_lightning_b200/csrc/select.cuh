@@ -229,9 +229,36 @@ struct GlobalKeyStream {
     }
 };
 
-// Exact kk-th largest key among the n keys in `list` (radix select, 8-bit
-// digits); uses hist[0..255].
+// Exact kk-th largest key among the n keys in `list`.  Short lists: every
+// element counts the larger and equal ones (broadcast reads, one barrier);
+// longer ones: radix select with 8-bit digits in hist[0..255].
 __device__ uint32_t list_select(const uint32_t* list, int n, uint32_t kk, uint32_t* hist, SelectSmem* sm) {
+    if (n <= 2 * kEpiThreads) {
+        uint32_t mine[2];
+        uint32_t gt[2] = {0u, 0u}, eq[2] = {0u, 0u};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = (int)threadIdx.x + u * kEpiThreads;
+            mine[u] = i < n ? list[i] : 0u;
+        }
+        for (int i = 0; i < n; ++i) {
+            const uint32_t x = list[i];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                gt[u] += x > mine[u];
+                eq[u] += x == mine[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = (int)threadIdx.x + u * kEpiThreads;
+            if (i < n && gt[u] < kk && kk <= gt[u] + eq[u]) sm->res_bin = mine[u];   // equal keys write one value
+        }
+        named_bar_sync(1, kEpiThreads);
+        const uint32_t T = sm->res_bin;
+        named_bar_sync(1, kEpiThreads);
+        return T;
+    }
     uint32_t prefix = 0;
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += kEpiThreads) hist[i] = 0u;
@@ -500,7 +527,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
     if (G > 1) {
         // ---- 1. publish: the keys at or above an estimate of the local c-th
         // largest, c about twice this CTA's expected share of the Top-K.  The
-        // estimate is the matching rank of a strided sample of 512 scores,
+        // estimate is the matching rank of a strided sample of 256 scores,
         // with 25% slack; a low estimate only costs the second round.
         const uint32_t c = min(K, 2u * K / (uint32_t)G + 32u);
 #pragma unroll
@@ -509,7 +536,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
             uint32_t edge = 0u;      // publish every key
             if (nloc[j] > (int)c && sm->kmin[j] != sm->kmax[j]) {
                 const float* sj = s_score + j * stride;
-                const int S = min(nloc[j], 512);
+                const int S = min(nloc[j], 2 * kEpiThreads);
                 const int step = nloc[j] / S;
                 for (int i = threadIdx.x; i < S; i += kEpiThreads) s_list[i] = order_key(sj[i * step]);
                 named_bar_sync(1, kEpiThreads);

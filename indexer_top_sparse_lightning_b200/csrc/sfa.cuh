@@ -24,10 +24,10 @@
 // the current one is stored) and written to 128-byte-swizzled shared memory;
 // this CTA's own rows are prefetched into L2 a few blocks ahead.  The online
 // softmax keeps a lazy reference max (O and l are rescaled only when the max
-// grows by more than 2^8).  With several row splits per token each CTA writes
-// an un-normalised partial O and (m, l); the last CTA of a (token, head half)
-// to finish merges the partials of all splits (arrival counted with a global
-// atomic).
+// grows by more than 2^8).  With several row splits per token, the last CTA of
+// a (token, head half) to finish (arrival counted with a global atomic) merges
+// the other splits' un-normalised partials and (m, l) into its own O, which
+// never leaves tensor memory.
 //
 // Roles per CTA (384 threads): warps 0-3 softmax (thread L <-> TMEM lane L:
 // head 64c + L%64, rows or value columns of half L/64), warps 4-10 gather,
@@ -581,35 +581,99 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                 if (half == 0 && head < p.H && p.lse)
                     p.lse[(int64_t)t * p.H + head] = empty ? -INFINITY : (mrun + log2f(ltot)) * 0.69314718055994531f;
             } else {
-                // un-normalised partial: [t][split][head][512]
-                float* po = p.part_o + (((int64_t)t * p.n_splits + split) * 128 + head) * kDv;
-                for (int c0 = 0; c0 < 256; c0 += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(tm_o + lane_off + c0, o);
-                    tmem_wait_ld();
-                    const int col = (c0 < 128 ? 128 * half + c0 : 256 + 128 * half + (c0 - 128));
+                // Several row splits: the arrival order picks the CTA that merges
+                // (the last to arrive); it waits only for CTAs that arrived before
+                // it, and those wait for nothing, so no residency assumption is made.
+                const int S = p.n_splits;
+                uint32_t* arrive = p.split_count + (int64_t)t * 2 + crank;
+                uint32_t* ready = p.split_ready + (int64_t)t * 2 + crank;
+                if (L == 0) m->last = atomicAdd(arrive, 1u) == (uint32_t)S - 1u;
+                named_bar_sync(1, 128);
+                // un-normalised partials [t][split][head half][512 columns][64 heads] and
+                // their (m, l) [t][split][head half][64][2]: a warp stores 32 heads of one column
+                auto part = [&](int sp) { return p.part_o + (((int64_t)t * S + sp) * 2 + crank) * (kDv * 64); };
+                auto pml = [&](int sp) { return p.part_ml + (((int64_t)t * S + sp) * 2 + crank) * (64 * 2); };
+                if (!m->last) {
+                    float* dst = part(split);
+                    for (int c0 = 0; c0 < 256; c0 += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(tm_o + lane_off + c0, o);
+                        tmem_wait_ld();
+                        const int col = (c0 < 128 ? 128 * half + c0 : 256 + 128 * half + (c0 - 128));
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        float4 v = make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]),
-                                               __uint_as_float(o[i + 2]), __uint_as_float(o[i + 3]));
-                        if (empty) v = make_float4(0.f, 0.f, 0.f, 0.f);
-                        *reinterpret_cast<float4*>(po + col + i) = v;
+                        for (int i = 0; i < 32; ++i) __stcg(dst + (col + i) * 64 + hl, empty ? 0.0f : __uint_as_float(o[i]));
+                    }
+                    if (half == 0) __stcg(reinterpret_cast<float2*>(pml(split)) + hl, make_float2(mrun, ltot));
+                    __threadfence();
+                    named_bar_sync(1, 128);
+                    if (L == 0) atomicAdd(ready, 1u);
+                } else {
+                    if (L == 0) {
+                        const uint64_t t0 = globaltimer();
+                        while (ld_acquire_gpu(ready) < (uint32_t)S - 1u) {
+                            if (globaltimer() - t0 > kWaitTimeoutNs) {
+                                atomicCAS(p.status, 0u, (uint32_t)kStTimeout);
+                                *abort = 1;
+                                break;
+                            }
+                        }
+                    }
+                    named_bar_sync(1, 128);
+                    if (!*abort) {
+                        // weights 2^(m_s - M) per split (own split from registers), kept in the idle Q buffer
+                        float* wts = reinterpret_cast<float*>(s_q);     // [S][128 threads]
+                        float M = mrun;
+                        for (int sp = 0; sp < S; ++sp)
+                            if (sp != split) M = fmaxf(M, __ldcg(reinterpret_cast<const float2*>(pml(sp)) + hl).x);
+                        float Lsum = 0.0f;
+                        for (int sp = 0; sp < S; ++sp) {
+                            const float2 v = sp == split ? make_float2(mrun, ltot)
+                                                         : __ldcg(reinterpret_cast<const float2*>(pml(sp)) + hl);
+                            const float w = (M == -INFINITY || v.x == -INFINITY) ? 0.0f : exp2f(v.x - M);
+                            wts[sp * 128 + L] = w;
+                            Lsum += w * v.y;
+                        }
+                        const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+                        for (int c0 = 0; c0 < 256; c0 += 32) {
+                            uint32_t o[32];
+                            tmem_ld32(tm_o + lane_off + c0, o);
+                            tmem_wait_ld();
+                            const int col = (c0 < 128 ? 128 * half + c0 : 256 + 128 * half + (c0 - 128));
+                            // splits folded in index order whichever CTA merges: the result is
+                            // the same bits on every call
+                            float acc[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+                            for (int sp = 0; sp < S; ++sp) {
+                                const float w = wts[sp * 128 + L];
+                                if (w == 0.0f) continue;
+                                if (sp == split) {
+#pragma unroll
+                                    for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, __uint_as_float(o[i]), acc[i]);
+                                } else {
+                                    const float* src = part(sp) + col * 64 + hl;
+#pragma unroll
+                                    for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, __ldcg(src + i * 64), acc[i]);
+                                }
+                            }
+                            if (head < p.H) {
+                                uint16_t* dst = p.out + ((int64_t)t * p.H + head) * kDv + col;
+#pragma unroll
+                                for (int i = 0; i < 32; i += 8)
+                                    *reinterpret_cast<uint4*>(dst + i) =
+                                        make_uint4(pack_bf16(acc[i] * inv, acc[i + 1] * inv), pack_bf16(acc[i + 2] * inv, acc[i + 3] * inv),
+                                                   pack_bf16(acc[i + 4] * inv, acc[i + 5] * inv), pack_bf16(acc[i + 6] * inv, acc[i + 7] * inv));
+                            }
+                        }
+                        if (half == 0 && head < p.H && p.lse)
+                            p.lse[(int64_t)t * p.H + head] = Lsum > 0.0f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+                        // every other split has arrived and signalled: ready for the next call
+                        if (L == 0) {
+                            *arrive = 0u;
+                            *ready = 0u;
+                        }
                     }
                 }
-                // (m, l) of this split and head
-                if (half == 0) {
-                    float* ml = p.part_ml + (((int64_t)t * p.n_splits + split) * 2 + crank) * 256;
-                    ml[hl] = mrun;
-                    ml[128 + hl] = ltot;
-                }
-                // the last CTA of this (token, head half) to get here merges all splits
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (L == 0) {
-                    const uint32_t prev = atomicAdd(p.split_count + (int64_t)t * 2 + crank, 1u);
-                    m->last = prev == (uint32_t)p.n_splits - 1u;
-                }
-                named_bar_sync(1, 128);
             }
         }
         if (!ok) *abort = 1;
@@ -618,70 +682,6 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
-    if (p.n_splits > 1 && m->last && !m->abort) {
-        // merge the splits of this (token, head half): weights 2^(m_s - M) per head
-        // (in the now idle Q buffer), then every thread folds (head, 4-column
-        // chunk) pairs, loads coalesced across heads
-        __threadfence();
-        const int S = p.n_splits;
-        float* wsm = reinterpret_cast<float*>(s_q);     // [S][64], S <= 64
-        float* linv = wsm + 64 * 64;                      // [64]
-        for (int hl = threadIdx.x; hl < 64; hl += Cfg::THREADS) {
-            float M = -INFINITY;
-            for (int s = 0; s < S; ++s)
-                M = fmaxf(M, __ldcg(p.part_ml + (((int64_t)t * S + s) * 2 + crank) * 256 + hl));
-            float Lsum = 0.0f;
-            for (int s = 0; s < S; ++s) {
-                const float* mls = p.part_ml + (((int64_t)t * S + s) * 2 + crank) * 256;
-                const float ms = __ldcg(mls + hl);
-                const float w = ms == -INFINITY ? 0.0f : exp2f(ms - M);
-                wsm[s * 64 + hl] = w;
-                Lsum += w * __ldcg(mls + 128 + hl);
-            }
-            linv[hl] = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
-            const int head = head0 + hl;
-            if (head < p.H && p.lse)
-                p.lse[(int64_t)t * p.H + head] = Lsum > 0.0f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
-        }
-        __syncthreads();
-        // thread -> 4-column chunk c4 = tid % 128 of heads tid/128 + 2u, u < 32, so that
-        // a warp reads 512 contiguous bytes; the loads of 8 heads are issued
-        // together, one split at a time
-        const int c4 = threadIdx.x & 127;
-        constexpr int U = 8;
-        static_assert(Cfg::THREADS >= 256, "the merge maps 256 threads onto 64 heads x 128 chunks");
-#pragma unroll 1
-        for (int u0 = 0; threadIdx.x < 256 && u0 < 32; u0 += U) {
-            float4 acc[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-            for (int s = 0; s < S; ++s) {
-                const float4* src = reinterpret_cast<const float4*>(p.part_o) +
-                                    (((int64_t)t * S + s) * 128 + head0 + (threadIdx.x >> 7) + 2 * u0) * 128 + c4;
-                float4 v[U];
-#pragma unroll
-                for (int u = 0; u < U; ++u) v[u] = __ldcg(src + (int64_t)u * 2 * 128);
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const float ws = wsm[s * 64 + (threadIdx.x >> 7) + 2 * (u0 + u)];
-                    acc[u].x += ws * v[u].x;
-                    acc[u].y += ws * v[u].y;
-                    acc[u].z += ws * v[u].z;
-                    acc[u].w += ws * v[u].w;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int hl = (threadIdx.x >> 7) + 2 * (u0 + u);
-                const float inv = linv[hl];
-                if (head0 + hl < p.H)
-                    *reinterpret_cast<uint2*>(p.out + ((int64_t)t * p.H + head0 + hl) * kDv + c4 * 4) =
-                        make_uint2(pack_bf16(acc[u].x * inv, acc[u].y * inv), pack_bf16(acc[u].z * inv, acc[u].w * inv));
-            }
-        }
-        if (threadIdx.x == 0) p.split_count[(int64_t)t * 2 + crank] = 0u;   // ready for the next call
-    }
     cluster_sync();   // no remote access may target an exited CTA, and no MMA may read a freed tile
     if (warp == Cfg::MMA_WARP) {
         tc_fence_after();
