@@ -526,23 +526,33 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
 
     if (G > 1) {
         // ---- 1. publish: the keys at or above an estimate of the local c-th
-        // largest, c about twice this CTA's expected share of the Top-K.  The
-        // estimate is the matching rank of a strided sample of 256 scores,
-        // with 25% slack; a low estimate only costs the second round.
+        // largest, c about twice this CTA's expected share of the Top-K: the
+        // matching rank (with 25% slack) of a strided sample of 256 scores,
+        // read off a range histogram of the sample -- the lower edge of its
+        // bin.  A low estimate only costs the second round.
         const uint32_t c = min(K, 2u * K / (uint32_t)G + 32u);
 #pragma unroll
         for (int j = 0; j < NQ; ++j) {
             if (!active[j]) continue;
             uint32_t edge = 0u;      // publish every key
-            if (nloc[j] > (int)c && sm->kmin[j] != sm->kmax[j]) {
+            const uint32_t lo = sm->kmin[j], hi = sm->kmax[j];
+            if (nloc[j] > (int)c && lo != hi) {
                 const float* sj = s_score + j * stride;
                 const int S = min(nloc[j], 2 * kEpiThreads);
                 const int step = nloc[j] / S;
-                for (int i = threadIdx.x; i < S; i += kEpiThreads) s_list[i] = order_key(sj[i * step]);
+                const int shift = range_shift(lo, hi);
+                for (int i = threadIdx.x; i < kBins; i += kEpiThreads) s_hist[i] = 0u;
+                named_bar_sync(1, kEpiThreads);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int i = (int)threadIdx.x + u * kEpiThreads;
+                    const uint32_t key = i < S ? order_key(sj[i * step]) : 0u;
+                    hist_add(s_hist, i < S, (key - lo) >> shift);
+                }
                 named_bar_sync(1, kEpiThreads);
                 const uint64_t want = ((uint64_t)c * 5u * (uint64_t)S) / (4u * (uint64_t)nloc[j]) + 8u;
-                const uint32_t r = want < (uint64_t)S ? (uint32_t)want : (uint32_t)S;
-                edge = list_select(s_list, S, r, s_hist, sm);
+                find_bin(s_hist, kBins, want < (uint64_t)S ? (uint32_t)want : (uint32_t)S, sm);
+                edge = lo + (sm->res_bin << shift);
             }
             publish(j, edge);
         }
