@@ -151,6 +151,31 @@ DSA_API dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * sparse_mla_attn without a caller workspace (the pages have no counterpart:
+ * this is a convenience of this library).  For callers that cannot provide
+ * device memory for the workspace -- code that must not allocate on the
+ * device, or that has no device allocator at hand.  The function itself
+ * allocates nothing: it uses a fixed 20 MiB scratch array inside the library
+ * module (status word, split counters, split partials), zero when the module
+ * loads and left zeroed by every call that completes without a device error.
+ * Arguments, layouts and results are those of sparse_mla_attn.
+ *  - The first call on a device looks up that device's scratch address (with
+ *    the device current); make it before any latency-critical use.
+ *  - Shapes whose split plan needs more scratch than 20 MiB are rejected with
+ *    DSA_ERR_WORKSPACE (dsa_last_error() gives both sizes); on a 148-SM B200
+ *    every shape fits.
+ *  - All calls on a device share the one scratch: calls whose device work
+ *    overlaps in time (other streams, other host threads) race and must not
+ *    be issued.
+ *  - Errors found by the kernels go to the scratch's status word, which this
+ *    API does not expose; use sparse_mla_attn when device-side status is
+ *    needed.
+ */
+DSA_API dsa_status sparse_mla_attn_static(const dsa_batch* batch, const dsa_attn_inputs* at,
+                                          const int32_t* idx, int32_t K, void* out, float* lse,
+                                          void* stream);
+
+/*
  * The whole decode step: indexer_topk then sparse_mla_attn on one stream,
  * without a host synchronization in between.  out_idx [T, K] is required
  * (it carries the index list between the stages); out_score and lse may be

@@ -36,9 +36,10 @@ DSA_ERR_CUDA = 4   # dsa_status code of a failed CUDA runtime / driver call
 
 
 class DsaError(RuntimeError):
-    def __init__(self, code: int, where: str):
+    def __init__(self, code: int, where: str, detail: str = ""):
         self.code = int(code)
-        detail = last_error() if self.code == DSA_ERR_CUDA else ""
+        if not detail and self.code == DSA_ERR_CUDA:
+            detail = last_error()
         super().__init__(f"{where}: {status_str(code)} (code {code})" + (f": {detail}" if detail else ""))
 
 
@@ -83,6 +84,9 @@ def load_library():
     lib.sparse_mla_attn.argtypes = [P(_Batch), P(_Attn), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
     lib.sparse_mla_attn.restype = ctypes.c_int
+    lib.sparse_mla_attn_static.argtypes = [P(_Batch), P(_Attn), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p]
+    lib.sparse_mla_attn_static.restype = ctypes.c_int
     lib.dsa_decode.argtypes = [P(_Batch), P(_Indexer), P(_Attn), ctypes.c_void_p, ctypes.c_void_p,
                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                ctypes.c_void_p]
@@ -268,6 +272,27 @@ def sparse_mla_attn(batch: Batch, q, kv_cache, idx, sm_scale: float, *, out=None
                              _ptr(buf), buf.numel(), _stream(stream))
     if rc != 0:
         raise DsaError(rc, "sparse_mla_attn")
+    return out, lse
+
+
+def sparse_mla_attn_static(batch: Batch, q, kv_cache, idx, sm_scale: float, *, out=None, lse=None,
+                           want_lse: bool = True, stream=None):
+    """sparse_mla_attn without a workspace: the library's fixed scratch is used
+    (calls on one device must not overlap).  Returns (out, lse)."""
+    import torch
+    lib = load_library()
+    at, T = _attn_struct(q, kv_cache, sm_scale)
+    _check(idx, "idx", torch.int32, 2, (T, None))
+    K = int(idx.shape[1])
+    cb = batch.c(T)
+    if out is None:
+        out = torch.empty((T, q.shape[1], 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((T, q.shape[1]), dtype=torch.float32, device=q.device)
+    rc = lib.sparse_mla_attn_static(ctypes.byref(cb), ctypes.byref(at), _ptr(idx), K, _ptr(out), _ptr(lse),
+                                    _stream(stream))
+    if rc != 0:
+        raise DsaError(rc, "sparse_mla_attn_static", last_error())
     return out, lse
 
 

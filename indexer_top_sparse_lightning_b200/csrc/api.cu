@@ -392,6 +392,39 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     return DSA_OK;
 }
 
+// ------------------------------------------------------------------ allocation-free attention
+// Scratch of sparse_mla_attn_static: the status word, the split counters and
+// the split partials, in module memory (zero when the module loads).  20 MiB
+// holds every split plan on a 148-SM B200 (at most 74 token-splits of 258 KB).
+constexpr size_t kStaticScratchBytes = size_t(20) << 20;
+__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+// Device address of the scratch for the current device, looked up once per
+// device (the first call on a device does the lookup).
+uint8_t* static_scratch(dsa_status* st) {
+    static std::mutex mu;
+    static uint8_t* addr[64] = {};
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev)) {
+        *st = fail(DSA_ERR_CUDA, "current device query", e);
+        return nullptr;
+    }
+    if (dev < 0 || dev >= 64) {
+        *st = fail(DSA_ERR_UNSUPPORTED, "device ordinal above 63");
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch)) {
+            *st = fail(DSA_ERR_CUDA, "static scratch address lookup", e);
+            return nullptr;
+        }
+        addr[dev] = reinterpret_cast<uint8_t*>(ptr);
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -452,6 +485,30 @@ dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs* at, co
     if (workspace_bytes < off + ap.part_bytes) return DSA_ERR_WORKSPACE;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + off, ap,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status sparse_mla_attn_static(const dsa_batch* batch, const dsa_attn_inputs* at, const int32_t* idx, int32_t K,
+                                  void* out, float* lse, void* stream) {
+    dsa_status st = check_batch(batch);
+    if (st != DSA_OK) return st;
+    if ((st = check_attn(at)) != DSA_OK) return st;
+    if (!idx || !out || K < 1 || K > kMaxTopK) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(out)) return DSA_ERR_INVALID_ARG;
+    const DevInfo di = dev_info();
+    if (di.sms <= 0) return fail(DSA_ERR_CUDA, "device query failed");
+    if (di.max_smem < SfaCfg::SMEM) return fail(DSA_ERR_UNSUPPORTED, "device shared memory per block too small");
+    const AttnPlan ap = plan_attn(batch, K, di);
+    const size_t need = kHeaderBytes + ap.part_bytes;
+    if (need > kStaticScratchBytes) {
+        snprintf(g_last_error, sizeof g_last_error,
+                 "sparse_mla_attn_static: this shape needs %zu bytes of scratch, the static scratch holds %zu", need,
+                 kStaticScratchBytes);
+        return DSA_ERR_WORKSPACE;
+    }
+    uint8_t* ws = static_scratch(&st);
+    if (!ws) return st;
+    return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, ap,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
