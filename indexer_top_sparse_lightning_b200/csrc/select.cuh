@@ -283,13 +283,16 @@ __device__ uint32_t list_select(const uint32_t* list, int n, uint32_t kk, uint32
 // of the final bin.
 template <class Stream>
 __device__ uint32_t find_threshold(const Stream& st, uint32_t lo, uint32_t hi, uint32_t kk, uint32_t* hist,
-                                   uint32_t* list, SelectSmem* sm) {
+                                   uint32_t* list, SelectSmem* sm, bool first_hist_ready = false) {
     while (lo != hi) {
         const int shift = range_shift(lo, hi);
-        for (int i = threadIdx.x; i < kBins; i += kEpiThreads) hist[i] = 0u;
-        named_bar_sync(1, kEpiThreads);
-        stream_hist(st, lo, hi, shift, hist);
-        named_bar_sync(1, kEpiThreads);
+        if (!first_hist_ready) {
+            for (int i = threadIdx.x; i < kBins; i += kEpiThreads) hist[i] = 0u;
+            named_bar_sync(1, kEpiThreads);
+            stream_hist(st, lo, hi, shift, hist);
+            named_bar_sync(1, kEpiThreads);
+        }
+        first_hist_ready = false;
         find_bin(hist, kBins, kk, sm);
         const uint32_t b = sm->res_bin, cnt = sm->res_cnt;
         kk = sm->res_kk;
@@ -474,8 +477,13 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         }
         named_bar_sync(1, kEpiThreads);
         if (sm->g_resident) {
+            // the first range histogram of the threshold search is built while loading
+            const uint32_t glo = sm->g_lo, ghi = sm->g_hi;
+            const int shift0 = glo < ghi ? range_shift(glo, ghi) : 0;
+            for (int i = threadIdx.x; i < kBins; i += kEpiThreads) s_hist[i] = 0u;
             // the scratch last held TMA-written key tiles
             fence_proxy_async_smem();
+            named_bar_sync(1, kEpiThreads);
             // 16-byte vectors of the concatenated (padded) ranks, eight loads in
             // flight per thread; vector v belongs to the rank whose offset range holds 4v
             const int nv = (int)(sm->g_total >> 2);
@@ -511,7 +519,17 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
                         if (e + 3u > n) y.z = 0u;
                         if (e + 4u > n) y.w = 0u;
                         *reinterpret_cast<uint4*>(keys + 4 * v) = y;
+                        x[u] = y;
                     }
+                }
+                // histogram adds by all lanes (padding keys 0 are below glo and not counted)
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int v = v0 + u * kEpiThreads + (int)threadIdx.x;
+                    const uint32_t w4[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        hist_add(s_hist, v < nv && w4[q] >= glo && w4[q] <= ghi, (w4[q] - glo) >> shift0);
                 }
             }
             named_bar_sync(1, kEpiThreads);
@@ -519,7 +537,8 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
     };
     auto group_T = [&](int j) -> uint32_t {
         if (sm->g_resident)
-            return find_threshold(SmemKeyStream{keys, (int)sm->g_total}, sm->g_lo, sm->g_hi, K, s_hist, s_list, sm);
+            return find_threshold(SmemKeyStream{keys, (int)sm->g_total}, sm->g_lo, sm->g_hi, K, s_hist, s_list, sm,
+                                  true);
         return find_threshold(GlobalKeyStream{rt, gv.cand + j * slot_keys, p.cand_slot, G, (int)sm->g_total},
                               sm->g_lo, sm->g_hi, K, s_hist, s_list, sm);
     };

@@ -29,9 +29,9 @@
 // the other splits' un-normalised partials and (m, l) into its own O, which
 // never leaves tensor memory.
 //
-// Roles per CTA (384 threads): warps 0-3 softmax (thread L <-> TMEM lane L:
-// head 64c + L%64, rows or value columns of half L/64), warps 4-10 gather,
-// warp 11 TMEM allocation; in CTA 0 it issues the MMAs, in CTA 1 it forwards
+// Roles per CTA (512 threads): warps 0-3 softmax (thread L <-> TMEM lane L:
+// head 64c + L%64, rows or value columns of half L/64), warps 4-14 gather,
+// warp 15 TMEM allocation; in CTA 0 it issues the MMAs, in CTA 1 it forwards
 // "my rows landed" and "my Q landed" to CTA 0.
 #pragma once
 #include "common.h"
@@ -43,7 +43,7 @@ struct SfaCfg {
     static constexpr int ROWS = 32;                     // selected rows per block (16 per CTA for S)
     static constexpr int NS = 4;                        // gather stages in shared memory
     static constexpr int NSB = 2;                       // logit / P buffers
-    static constexpr int PF = 8;                        // blocks prefetched into L2 ahead of the gather
+    static constexpr int PF = 2;                        // blocks prefetched into L2 ahead of the gather
     static constexpr int KBQ = 9;                       // 64-wide K blocks of a 576-wide row
     static constexpr int Q_BYTES = KBQ * 64 * 128;      // [64 heads x 64] per K block
     static constexpr int KOWN_KB = 16 * 128;            // own 16 rows x 64 elements, per K block
@@ -59,9 +59,9 @@ struct SfaCfg {
     static constexpr int OFF_ROWS = OFF_MISC + MISC_BYTES;
     static constexpr int OFF_XM = OFF_ROWS + MAX_ROWS * 4;    // partner max exchange [2][128]
     static constexpr int SMEM = 1024 + OFF_XM + 2 * 128 * 4;
-    static constexpr int THREADS = 384;
-    static constexpr int GATHER = 224;                  // threads of warps 4-10
-    static constexpr int MMA_WARP = 11;                 // TMEM owner; MMA issuer (CTA 0) / forwarder (CTA 1)
+    static constexpr int THREADS = 512;
+    static constexpr int GATHER = 352;                  // threads of warps 4-14
+    static constexpr int MMA_WARP = 15;                 // TMEM owner; MMA issuer (CTA 0) / forwarder (CTA 1)
     static constexpr int GATHER_ITEMS = 16 * 72 + 16 * 32;   // 16-byte loads of one block per CTA
     static constexpr int S_COLS = 16;                   // TMEM columns of one logit buffer
     static constexpr int TMEM_COLS = 512;               // O: [0,256), logit buffers from column 256
@@ -271,14 +271,17 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             int next_qk = 0, next_pv = 0;
             uint64_t t_idle = 0;
             while (ok && next_pv < nblk) {
-                const bool do_qk = __shfl_sync(0xffffffffu, (int)(next_qk < nblk && next_qk < next_pv + Cfg::NSB &&
-                                                                  qk_ready(next_qk)), 0);
-                const bool do_pv = !do_qk && __shfl_sync(0xffffffffu, (int)(next_pv < next_qk && pv_ready(next_pv)), 0);
-                if (do_qk) {
-                    issue_qk(next_qk++);
-                    t_idle = 0;
-                } else if (do_pv) {
+                // P.V (four short MMAs that free a P buffer and a row stage) goes first
+                // when a block's probabilities are ready; otherwise a block's logits go
+                // ahead as soon as its rows and its logit buffer are free (the softmax of
+                // block jb-NSB has read it), overlapping the softmax of earlier blocks
+                const bool do_pv = __shfl_sync(0xffffffffu, (int)(next_pv < next_qk && pv_ready(next_pv)), 0);
+                const bool do_qk = !do_pv && __shfl_sync(0xffffffffu, (int)(next_qk < nblk && qk_ready(next_qk)), 0);
+                if (do_pv) {
                     issue_pv(next_pv++);
+                    t_idle = 0;
+                } else if (do_qk) {
+                    issue_qk(next_qk++);
                     t_idle = 0;
                 } else {
                     bool stop = *abort != 0;
@@ -301,7 +304,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- row gather
         const int pt = threadIdx.x - 128;           // 0..GATHER-1
-        const int gw = pt >> 5;                      // gather warp 0..6
+        const int gw = pt >> 5;                      // gather warp 0..10
         const int b = token_sequence(p.cu_q, p.B, t);
         const int64_t L = __ldg(p.seq_lens + b);
         const int32_t* idx_t = p.idx + (int64_t)t * p.K;
@@ -419,6 +422,8 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         };
         if (gw == 0 && lane == 0) DSA_TRACE_MARK(1);
         for (int jb = 0; jb < Cfg::PF; ++jb) prefetch_block(jb);
+        // two register buffers: the loads of the next block are in flight while a
+        // block is stored
         uint4 ra[IPT], rb[IPT];
         bool ok = true;
         if (nblk > 0) load(ra, 0);
