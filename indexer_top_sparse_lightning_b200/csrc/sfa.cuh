@@ -19,9 +19,9 @@
 //     value columns 128c..128c+127 and 256+128c..256+128c+127 of all 32 rows
 //     (B split by N); each CTA's tensor memory receives O for its 64 heads
 //     over all 512 columns.
-// Rows are gathered with 16-byte vector loads into registers (one coalesced
-// warp read per row segment; the loads of the next block are in flight while
-// the current one is stored) and written to 128-byte-swizzled shared memory;
+// Rows are gathered with 16-byte asynchronous copies into the stages (one
+// coalesced warp read per row segment; every free stage has its copies in
+// flight) and written to 128-byte-swizzled shared memory;
 // this CTA's own rows are prefetched into L2 a few blocks ahead.  The online
 // softmax keeps a lazy reference max (O and l are rescaled only when the max
 // grows by more than 2^8).  With several row splits per token, the last CTA of
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         mbar_init(&m->q_full, 1);
         mbar_init(&m->q_peer, 1);
         for (int i = 0; i < Cfg::NS; ++i) {
-            mbar_init(&m->kv_full[i], Cfg::GATHER / 32);
+            mbar_init(&m->kv_full[i], Cfg::GATHER);
             mbar_init(&m->kv_peer[i], 1);
             mbar_init(&m->kv_empty[i], 1);
         }
@@ -205,6 +205,9 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                     const int s = jb % Cfg::NS;
                     if (!mbar_wait(&m->kv_full[s], (jb / Cfg::NS) & 1, abort)) { ok = false; break; }
                     DSA_TRACE_BLK(jb, 1);
+                    // the rows were written by cp.async (generic proxy); CTA 0's MMA reads
+                    // them through the async proxy
+                    fence_proxy_async_smem();
                     mbar_arrive_remote(mapa_shared(smem_u32(&m->kv_peer[s]), 0));
                 }
                 if (!ok) *abort = 1;
@@ -214,16 +217,27 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             // ------------------------------------------------------------ MMA issuer
             // The whole warp runs the schedule (decisions taken by lane 0 and
             // broadcast); one elected lane issues each group of MMAs and its commits.
-            bool ok = __shfl_sync(0xffffffffu,
-                                  (int)(mbar_wait(&m->q_full, 0, abort) && mbar_wait(&m->q_peer, 0, abort)), 0);
+            int q_ok = 0;
+            if (lane == 0) q_ok = mbar_wait(&m->q_full, 0, abort) && mbar_wait(&m->q_peer, 0, abort);
+            bool ok = __shfl_sync(0xffffffffu, q_ok, 0);
             tc_fence_after();
             const uint32_t q_addr = smem_u32(s_q);
             const uint32_t p_addr = smem_u32(s_p);
             auto qk_ready = [&](int jb) -> bool {
                 const int s = jb % Cfg::NS, b = jb % Cfg::NSB;
                 const uint32_t ph = (jb / Cfg::NS) & 1;
+#ifdef DSA_TRACE
+                const bool a = mbar_test_wait(smem_u32(&m->kv_full[s]), ph);
+                const bool c = mbar_test_wait(smem_u32(&m->kv_peer[s]), ph);
+                const bool e = mbar_test_wait(smem_u32(&m->s_empty[b]), ((jb / Cfg::NSB) & 1) ^ 1);
+                if (a && g_dsa_trace_blk[jb & 63][12] == 0) DSA_TRACE_BLK(jb, 12);
+                if (c && g_dsa_trace_blk[jb & 63][13] == 0) DSA_TRACE_BLK(jb, 13);
+                if (e && g_dsa_trace_blk[jb & 63][14] == 0) DSA_TRACE_BLK(jb, 14);
+                return a && c && e;
+#else
                 return mbar_test_wait(smem_u32(&m->kv_full[s]), ph) && mbar_test_wait(smem_u32(&m->kv_peer[s]), ph) &&
                        mbar_test_wait(smem_u32(&m->s_empty[b]), ((jb / Cfg::NSB) & 1) ^ 1);
+#endif
             };
             auto pv_ready = [&](int jb) -> bool {
                 return mbar_test_wait(smem_u32(&m->p_full[jb % Cfg::NSB]), (jb / Cfg::NSB) & 1);
@@ -232,6 +246,7 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                 const int s = jb % Cfg::NS, b = jb % Cfg::NSB;
                 if (elect_one()) {
                     DSA_TRACE_BLK(jb, 6);
+                    fence_proxy_async_smem();   // this CTA's cp.async rows -> async proxy
                     tc_fence_after();
                     const uint32_t kown = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
 #pragma unroll
@@ -275,8 +290,14 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                 // when a block's probabilities are ready; otherwise a block's logits go
                 // ahead as soon as its rows and its logit buffer are free (the softmax of
                 // block jb-NSB has read it), overlapping the softmax of earlier blocks
-                const bool do_pv = __shfl_sync(0xffffffffu, (int)(next_pv < next_qk && pv_ready(next_pv)), 0);
-                const bool do_qk = !do_pv && __shfl_sync(0xffffffffu, (int)(next_qk < nblk && qk_ready(next_qk)), 0);
+                // (lane 0 probes the barriers: 32 lanes probing one mbarrier serialise)
+                int pv_ok = 0, qk_ok = 0;
+                if (lane == 0) {
+                    pv_ok = next_pv < next_qk && pv_ready(next_pv);
+                    qk_ok = !pv_ok && next_qk < nblk && qk_ready(next_qk);
+                }
+                const bool do_pv = __shfl_sync(0xffffffffu, pv_ok, 0);
+                const bool do_qk = __shfl_sync(0xffffffffu, qk_ok, 0);
                 if (do_pv) {
                     issue_pv(next_pv++);
                     t_idle = 0;
@@ -394,48 +415,35 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             }
         }
         static_assert(Cfg::STAGE_BYTES <= 0xFFFF, "stage offsets are packed in 16 bits");
-        auto load = [&](uint4 (&R)[IPT], int jb) {
+        // one block: 16-byte asynchronous copies straight into the stage (own-row
+        // value chunks copied twice), then this thread's arrival on the stage's
+        // barrier once its copies have landed; a thread runs ahead as far as the
+        // free stages allow
+        auto issue = [&](int jb) -> bool {
+            const int s = jb % Cfg::NS;
+            if (!__all_sync(0xffffffffu, mbar_wait(&m->kv_empty[s], ((jb / Cfg::NS) & 1) ^ 1, abort))) return false;
+            if (pt == 0) DSA_TRACE_BLK(jb, 5);
+            const uint32_t base = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
             const int32_t* rows = s_rows + jb * Cfg::ROWS;
 #pragma unroll
             for (int u = 0; u < IPT; ++u) {
                 if (src[u] == 0xFFFFFFFFu) continue;          // warp-uniform
                 const int32_t r = rows[src[u] >> 16];
-                R[u] = ld_nc_v4(kv_bytes + (int64_t)(r < 0 ? 0 : r) * (kDqk * 2) + (src[u] & 0xFFFFu));
+                const uint8_t* g = kv_bytes + (int64_t)(r < 0 ? 0 : r) * (kDqk * 2) + (src[u] & 0xFFFFu);
+                cp_async_16(base + (dst[u] & 0xFFFFu), g, true);
+                if ((dst[u] >> 16) != 0xFFFFu) cp_async_16(base + (dst[u] >> 16), g, true);
             }
-        };
-        auto store = [&](const uint4 (&R)[IPT], int jb) -> bool {
-            const int s = jb % Cfg::NS;
-            if (!__all_sync(0xffffffffu, mbar_wait(&m->kv_empty[s], ((jb / Cfg::NS) & 1) ^ 1, abort))) return false;
-            if (pt == 0) DSA_TRACE_BLK(jb, 5);
-            const uint32_t base = smem_u32(s_kv + s * Cfg::STAGE_BYTES);
-#pragma unroll
-            for (int u = 0; u < IPT; ++u) {
-                if (src[u] == 0xFFFFFFFFu) continue;
-                st_shared_v4(base + (dst[u] & 0xFFFFu), R[u]);
-                if ((dst[u] >> 16) != 0xFFFFu) st_shared_v4(base + (dst[u] >> 16), R[u]);
-            }
-            // generic-proxy stores -> visible to the tensor core, then one arrival per warp
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&m->kv_full[s]);
+            cp_async_arrive_noinc(&m->kv_full[s]);
             return true;
         };
         if (gw == 0 && lane == 0) DSA_TRACE_MARK(1);
         for (int jb = 0; jb < Cfg::PF; ++jb) prefetch_block(jb);
-        // two register buffers: the loads of the next block are in flight while a
-        // block is stored
-        uint4 ra[IPT], rb[IPT];
         bool ok = true;
-        if (nblk > 0) load(ra, 0);
-        for (int jb = 0; ok && jb < nblk; jb += 2) {
+        for (int jb = 0; ok && jb < nblk; ++jb) {
             prefetch_block(jb + Cfg::PF);
-            prefetch_block(jb + Cfg::PF + 1);
-            if (jb + 1 < nblk) load(rb, jb + 1);
-            ok = store(ra, jb);
-            if (!ok || jb + 1 >= nblk) break;
-            if (jb + 2 < nblk) load(ra, jb + 2);
-            ok = store(rb, jb + 1);
+            ok = issue(jb);
         }
+        cp_async_wait_all();
         if (!ok && lane == 0) *abort = 1;
     } else {
         // ---------------------------------------------------------------- softmax + epilogue
