@@ -146,7 +146,9 @@ bool plan_for(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl) {
     pl.score_cap = (cap / (kTileKeys * NQ)) * (kTileKeys * NQ);
     if (pl.score_cap > kCandSlotKeys) pl.score_cap = (int)((kCandSlotKeys / (kTileKeys * NQ)) * (kTileKeys * NQ));
     pl.smem = Cfg::FIXED_SMEM + pl.score_cap * 4;
-    pl.grid = di.sms;     // one CTA per SM (shared memory use allows no more)
+    // one CTA per SM (shared memory use allows no more); a group's select reads
+    // at most 256 publication headers
+    pl.grid = di.sms < 256 ? di.sms : 256;
     if (pl.mode == 1) {
         if (bt->max_seq_len > pl.score_cap) return false;
         pl.seqs_per_launch = bt->batch;

@@ -217,15 +217,13 @@ struct GlobalKeyStream {
     const uint32_t* cand;      // slot of rank 0
     int64_t slot;              // keys between the slots of consecutive ranks
     int G, n;
+    mutable int cur = 0;       // rank of this thread's last index (indices mostly increase)
     __device__ __forceinline__ int size() const { return n; }
     __device__ uint32_t key(int i) const {
-        int lo = 0, hi = G - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if ((int)rt[2 * mid + 1] <= i) lo = mid; else hi = mid - 1;
-        }
-        const uint32_t e = (uint32_t)i - rt[2 * lo + 1];
-        return e < rt[2 * lo] ? __ldcg(cand + lo * slot + e) : 0u;
+        if ((int)rt[2 * cur + 1] > i) cur = 0;
+        while (cur + 1 < G && (int)rt[2 * (cur + 1) + 1] <= i) ++cur;
+        const uint32_t e = (uint32_t)i - rt[2 * cur + 1];
+        return e < rt[2 * cur] ? __ldcg(cand + cur * slot + e) : 0u;
     }
 };
 
@@ -456,23 +454,52 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
     uint32_t* rt = reinterpret_cast<uint32_t*>(gscratch);
     uint32_t* keys = rt + ((2 * G + 3) & ~3);
     auto gather = [&](int j) {
+        // headers of ranks tid and tid + 128 (G <= 256), read together; flat offsets
+        // of the (4-padded) ranks by a prefix over rank order
+        static_assert(kEpiThreads == 128, "two header slots per thread cover 256 ranks");
+        uint4 h[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int r = (int)threadIdx.x + u * kEpiThreads;
+            h[u] = r < G ? __ldcg(reinterpret_cast<const uint4*>(gv.hdr + ((int64_t)r * NQ + j) * 4))
+                         : make_uint4(0u, 0xFFFFFFFFu, 0u, 0u);
+        }
         if (threadIdx.x == 0) {
-            uint32_t lo = 0xFFFFFFFFu, hi = 0u, off = 0u, emax = 0u;
-            for (int r = 0; r < G; ++r) {
-                const uint4 h = __ldcg(reinterpret_cast<const uint4*>(gv.hdr + ((int64_t)r * NQ + j) * 4));
-                rt[2 * r] = h.x;
-                rt[2 * r + 1] = off;
-                off += (h.x + 3u) & ~3u;
-                if (h.x) {
-                    lo = min(lo, h.y);
-                    hi = max(hi, h.z);
+            sm->g_lo = 0xFFFFFFFFu;
+            sm->g_hi = 0u;
+            sm->g_max_edge = 0u;
+        }
+        uint32_t tot0, tot1;
+        const uint32_t off0 = epi_exclusive_scan((h[0].x + 3u) & ~3u, sm->scan, &tot0);
+        const uint32_t off1 = tot0 + epi_exclusive_scan((h[1].x + 3u) & ~3u, sm->scan, &tot1);
+        uint32_t lo = 0xFFFFFFFFu, hi = 0u, emax = 0u;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int r = (int)threadIdx.x + u * kEpiThreads;
+            if (r < G) {
+                rt[2 * r] = h[u].x;
+                rt[2 * r + 1] = u == 0 ? off0 : off1;
+                if (h[u].x) {
+                    lo = min(lo, h[u].y);
+                    hi = max(hi, h[u].z);
                 }
-                emax = max(emax, h.w);
+                emax = max(emax, h[u].w);
             }
-            sm->g_lo = lo;
-            sm->g_hi = hi;
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+            emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+        }
+        if ((threadIdx.x & 31) == 0) {
+            red_min_shared(&sm->g_lo, lo);
+            red_max_shared(&sm->g_hi, hi);
+            red_max_shared(&sm->g_max_edge, emax);
+        }
+        if (threadIdx.x == 0) {
+            const uint32_t off = tot0 + tot1;
             sm->g_total = off;
-            sm->g_max_edge = emax;
             sm->g_resident = (int64_t)((2 * G + 3) & ~3) * 4 + (int64_t)off * 4 <= (int64_t)gscratch_bytes;
         }
         named_bar_sync(1, kEpiThreads);
@@ -546,7 +573,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
     if (G > 1) {
         // ---- 1. publish: the keys at or above an estimate of the local c-th
         // largest, c about twice this CTA's expected share of the Top-K: the
-        // matching rank (with 25% slack) of a strided sample of 256 scores,
+        // matching rank (with 25% slack) of a strided sample of 512 scores,
         // read off a range histogram of the sample -- the lower edge of its
         // bin.  A low estimate only costs the second round.
         const uint32_t c = min(K, 2u * K / (uint32_t)G + 32u);
@@ -557,19 +584,21 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
             const uint32_t lo = sm->kmin[j], hi = sm->kmax[j];
             if (nloc[j] > (int)c && lo != hi) {
                 const float* sj = s_score + j * stride;
-                const int S = min(nloc[j], 2 * kEpiThreads);
+                const int S = min(nloc[j], 4 * kEpiThreads);
                 const int step = nloc[j] / S;
                 const int shift = range_shift(lo, hi);
                 for (int i = threadIdx.x; i < kBins; i += kEpiThreads) s_hist[i] = 0u;
                 named_bar_sync(1, kEpiThreads);
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     const int i = (int)threadIdx.x + u * kEpiThreads;
                     const uint32_t key = i < S ? order_key(sj[i * step]) : 0u;
                     hist_add(s_hist, i < S, (key - lo) >> shift);
                 }
                 named_bar_sync(1, kEpiThreads);
-                const uint64_t want = ((uint64_t)c * 5u * (uint64_t)S) / (4u * (uint64_t)nloc[j]) + 8u;
+                // the sample rank matching 1.25 c of nloc, plus two
+                const uint64_t want = ((uint64_t)c * 5u * (uint64_t)S + 4u * (uint64_t)nloc[j] - 1u) /
+                                          (4u * (uint64_t)nloc[j]) + 2u;
                 find_bin(s_hist, kBins, want < (uint64_t)S ? (uint32_t)want : (uint32_t)S, sm);
                 edge = lo + (sm->res_bin << shift);
             }
@@ -600,42 +629,44 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
                 // first publication, the CTAs whose edge is above T publish all
                 // their keys >= T, and the threshold of the enlarged set is exact
                 const uint32_t t1 = T;
+                if (threadIdx.x == 0) DSA_TRACE_MARK(12);
                 if (!group_barrier(gv.sync, G, gen, p.status, abort)) return false;
                 if (sm->edge[j] > t1) publish(j, t1);
                 if (!group_barrier(gv.sync, G, gen, p.status, abort)) return false;
                 gather(j);
                 T = group_T(j);
             }
-            // ---- 3. lower ranks' published keys above / equal to T (warp w takes ranks w, w+4, ...)
+            // ---- 3. published keys above / equal to T: all ranks, and ranks below this
+            // one -- the ranks lie in rank order in the flat key index, so "below" is
+            // the prefix [0, offset of this rank)
             uint32_t gt_b = 0, eq_b = 0, gt_all = 0;
-            const bool res = sm->g_resident;
-            const GlobalKeyStream gs{rt, gv.cand + j * slot_keys, p.cand_slot, G, (int)sm->g_total};
-            for (int r = warp; r < G; r += 4) {
-                const uint32_t n = rt[2 * r], off = rt[2 * r + 1];
-                uint32_t g = 0, e = 0;
-                for (uint32_t i0 = 0; i0 < n; i0 += 32 * kU) {
+            const uint32_t mine = rt[2 * gv.rank + 1];
+            auto count = [&](const auto& st) {
+                const int n = st.size();
+                for (int i0 = 0; i0 < n; i0 += kEpiThreads * kU) {
                     uint32_t k[kU];
 #pragma unroll
                     for (int u = 0; u < kU; ++u) {
-                        const uint32_t i = i0 + u * 32 + lane;
-                        k[u] = i < n ? (res ? keys[off + i] : gs.key((int)(off + i))) : 0u;
+                        const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+                        k[u] = i < n ? st.key(i) : 0u;
                     }
 #pragma unroll
                     for (int u = 0; u < kU; ++u) {
-                        g += k[u] > T;
-                        e += k[u] == T;
+                        const uint32_t i = (uint32_t)(i0 + u * kEpiThreads + (int)threadIdx.x);
+                        const bool low = i < mine;
+                        gt_all += k[u] > T;
+                        gt_b += low && k[u] > T;
+                        eq_b += low && k[u] == T;
                     }
                 }
+            };
+            if (sm->g_resident) count(SmemKeyStream{keys, (int)sm->g_total});
+            else count(GlobalKeyStream{rt, gv.cand + j * slot_keys, p.cand_slot, G, (int)sm->g_total});
 #pragma unroll
-                for (int o = 16; o; o >>= 1) {
-                    g += __shfl_xor_sync(0xffffffffu, g, o);
-                    e += __shfl_xor_sync(0xffffffffu, e, o);
-                }
-                gt_all += g;
-                if (r < gv.rank) {
-                    gt_b += g;
-                    eq_b += e;
-                }
+            for (int o = 16; o; o >>= 1) {
+                gt_b += __shfl_xor_sync(0xffffffffu, gt_b, o);
+                eq_b += __shfl_xor_sync(0xffffffffu, eq_b, o);
+                gt_all += __shfl_xor_sync(0xffffffffu, gt_all, o);
             }
             if (lane == 0) {
                 sm->wcnt[warp][0] = gt_b;
