@@ -57,6 +57,16 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def peaks_tensor():
+    """Dense bf16 tensor peak: the sustained GEMM figure (a prefill step runs for many milliseconds)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "indexer_top_sparse_lightning_b200", "csrc")
@@ -194,22 +204,33 @@ def run_ours(args, rank, world, local_rank):
     out = torch.empty((T, wl.H, 512), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
-    ev_i0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_i1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    key_bytes = wl.key_bytes()
+    kv_bytes = wl.kv_bytes()
+    step_bytes = key_bytes + kv_bytes
+    # Inputs smaller than twice the L2 would be partly served from L2 on the next step: flush between steps
+    # (outside the per-step events) and time each step on its own.
+    flush = step_bytes < 2 * L2_BYTES
+    scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
 
     def step(i=None):
         if i is not None:
-            ev_i0[i].record(stream)
+            ev[i][0].record(stream)
         dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], K, k_scale=d["k_scale"], out_idx=out_idx,
                          want_score=False, workspace=ws)
         if i is not None:
-            ev_i1[i].record(stream)
+            ev[i][1].record(stream)
         dsa.sparse_mla_attn(batch, d["q"], d["kv"], out_idx, wl.sm_scale, out=out, want_lse=False, workspace=ws)
+        if i is not None:
+            ev[i][2].record(stream)
 
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     t_warm = time.time()
     for _ in range(max(3, args.warmup)):
+        if flush:
+            scrub.zero_()
         step()
     torch.cuda.synchronize()
     if dsa.get_status(ws) != 0:
@@ -223,14 +244,20 @@ def run_ours(args, rank, world, local_rank):
     t_start = time.time()
     e0.record(stream)
     for i in range(args.steps):
+        if flush:
+            scrub.zero_()
         step(i)
     e1.record(stream)
     torch.cuda.synchronize()
     t_end = time.time()
     if world > 1:
         dist.barrier()
-    ms_total = e0.elapsed_time(e1)
-    idx_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev_i0, ev_i1))
+    per_step = [a.elapsed_time(c) for a, _, c in ev]
+    idx_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    sfa_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    ms_total = sum(per_step) if flush else e0.elapsed_time(e1)
+    q = statistics.quantiles(per_step, n=10) if len(per_step) > 1 else per_step * 9
+    pct = {"p10": q[0], "p50": statistics.median(per_step), "p90": q[-1]}
     # keep the GPU busy long enough for the clock sampler if the timed region was short
     soak_end = t_end
     if t_end - t_start < 1.0:
@@ -243,10 +270,36 @@ def run_ours(args, rank, world, local_rank):
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
 
-    t = torch.tensor([ms_total, idx_ms], dtype=torch.float64, device=dev)
+    # the same step captured once in a CUDA graph and replayed (launch overhead removed)
+    graph_ms = None
+    if not flush:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        ga = torch.cuda.Event(enable_timing=True)
+        gb = torch.cuda.Event(enable_timing=True)
+        ga.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        gb.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = ga.elapsed_time(gb) / args.steps
+        del g
+        if dsa.get_status(ws) != 0:
+            raise RuntimeError("device reported an error in the graph replays")
+
+    t = torch.tensor([ms_total, idx_ms, sfa_ms, graph_ms or 0.0], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, idx_ms = float(t[0]), float(t[1])
+    ms_total, idx_ms, sfa_ms, graph_ms = float(t[0]), float(t[1]), float(t[2]), (float(t[3]) or None)
     ms_step = ms_total / args.steps
 
     # ------------------------------------------------------------ end to end through the public API
@@ -270,14 +323,16 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(args.e2e_steps):
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.e2e_steps)]
+    for a, b in ee:
+        if flush:
+            scrub.zero_()
+        a.record(stream)
         e2e_step()
-    b.record(stream)
+        b.record(stream)
     torch.cuda.synchronize()
-    t = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+    e2e_total = (sum(a.elapsed_time(b) for a, b in ee) if flush else ee[0][0].elapsed_time(ee[-1][1]))
+    t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     e2e_ms = float(t[0]) / args.e2e_steps
@@ -287,30 +342,50 @@ def run_ours(args, rank, world, local_rank):
                                        k_scale=d["k_scale"])
     if rank != 0:
         return
-    key_bytes = wl.key_bytes()
-    kv_bytes = wl.kv_bytes()
-    step_bytes = key_bytes + kv_bytes
     peak, peak_kind = peaks()
     idx_gbs = key_bytes / (idx_ms * 1e-3) / 1e9
+    sfa_gbs = kv_bytes / (sfa_ms * 1e-3) / 1e9
     step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
     tokens_total = T * world
     clocks = sampler.summary(t_start, t_end) or sampler.summary(t_warm, soak_end)
     window = "timed region" if sampler.summary(t_start, t_end) else "warm-up + timed + soak of the same step"
+    l2 = (f"L2 flushed between steps ({2 * L2_BYTES / 1e6:.0f} MB written outside the per-step events): "
+          f"{step_bytes / 1e6:.1f} MB read per step vs {L2_BYTES / 1e6:.0f} MB L2" if flush else
+          f"inputs larger than L2: {step_bytes / 1e6:.1f} MB read per step vs {L2_BYTES / 1e6:.0f} MB L2, no flush")
+    if wl.T > 64:
+        # prefill: the indexer's causal q.k contraction is tensor-bound
+        tf_peak, tf_kind = peaks_tensor()
+        flops = wl.indexer_flops()
+        roof = {"kernel": "indexer_topk_kernel", "bound": "tensor", "achieved": flops / (idx_ms * 1e-3) / 1e12,
+                "peak": tf_peak, "peak_kind": tf_kind, "unit": "TFLOP/s",
+                "frac": flops / (idx_ms * 1e-3) / 1e12 / tf_peak, "traffic": None, "ms_per_launch": idx_ms,
+                "algorithmic_flops_per_launch": flops}
+    else:
+        roof = {"kernel": "indexer_topk_kernel", "bound": "hbm", "achieved": idx_gbs, "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": idx_gbs / peak,
+                "traffic": ncu_traffic("indexer_topk_kernel") if args.workload == "batch32" else None,
+                "ms_per_launch": idx_ms, "algorithmic_bytes_per_launch": key_bytes}
     line = {
         "metric": METRIC, "value": tokens_total / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": describe(wl), "global_batch": tokens_total, "seq_len": int(wl.seq_lens.max()),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"inputs larger than L2: {step_bytes / 1e6:.1f} MB read per step vs "
-                         f"{L2_BYTES / 1e6:.0f} MB L2, no flush"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "l2": l2},
         "hbm": {"bytes_per_step": step_bytes, "indexer_key_bytes": key_bytes, "gathered_kv_bytes": kv_bytes,
                 "step_gbs": step_gbs, "frac_of_8tbs": step_gbs / SPEC_HBM_GBS,
                 "frac_of_measured": step_gbs / peak},
-        "roofline": {"kernel": "indexer_topk_kernel", "bound": "hbm", "achieved": idx_gbs, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": idx_gbs / peak,
-                     "traffic": ncu_traffic("indexer_topk_kernel"), "ms_per_launch": idx_ms,
-                     "algorithmic_bytes_per_launch": key_bytes},
+        "roofline": roof,
+        "kernels": {
+            "indexer_topk_kernel": {"ms_per_launch": idx_ms, "gbs": idx_gbs, "frac_of_measured_hbm": idx_gbs / peak,
+                                    "algorithmic_bytes": key_bytes},
+            "sfa_decode_kernel": {"ms_per_launch": sfa_ms, "gbs": sfa_gbs, "frac_of_measured_hbm": sfa_gbs / peak,
+                                  "algorithmic_bytes": kv_bytes,
+                                  "traffic": ncu_traffic("sfa_decode_kernel") if args.workload == "batch32" else None},
+        },
+        "step_ms_percentiles": pct,
+        "graph": {"ms_per_step": graph_ms, "value": tokens_total / (graph_ms * 1e-3) if graph_ms else None,
+                  "note": "the same step captured once in a CUDA graph and replayed back to back"
+                  if graph_ms else "not taken: steps are separated by L2 flushes"},
         "e2e": {"value": tokens_total / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches * args.steps,

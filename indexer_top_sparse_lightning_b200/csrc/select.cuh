@@ -310,6 +310,82 @@ __device__ uint32_t find_threshold(const Stream& st, uint32_t lo, uint32_t hi, u
     return lo;
 }
 
+// The kk-th largest key of a long stream whose keys span [lo, hi].  A strided
+// sample of 512 keys brackets it: the sample ranks kk*S/n -/+ (4 sigma + 4)
+// give a window [wlo, whi]; one pass counts the keys above the window and
+// histograms those inside it.  If the kk-th largest lies inside (above < kk
+// <= above + inside), the search goes on in the window with kk - above;
+// otherwise over the whole range.  Either way the result is exact.
+template <class Stream>
+__device__ uint32_t sampled_threshold(const Stream& st, uint32_t lo, uint32_t hi, uint32_t kk, uint32_t* hist,
+                                      uint32_t* list, SelectSmem* sm) {
+    constexpr int S = 4 * kEpiThreads;
+    const int n = st.size();
+    if (n < 8 * S || lo == hi) return find_threshold(st, lo, hi, kk, hist, list, sm);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int step = n / S;
+    const int shift = range_shift(lo, hi);
+    for (int i = threadIdx.x; i < kBins; i += kEpiThreads) hist[i] = 0u;
+    named_bar_sync(1, kEpiThreads);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const uint32_t key = st.key(((int)threadIdx.x + u * kEpiThreads) * step);
+        hist_add(hist, true, (key - lo) >> shift);
+    }
+    named_bar_sync(1, kEpiThreads);
+    const float r = (float)kk * (float)S / (float)n;
+    const float pr = r / (float)S;
+    const float slack = 4.0f * sqrtf((float)S * pr * (1.0f - pr)) + 4.0f;
+    const uint32_t r_hi = (uint32_t)fmaxf(1.0f, floorf(r - slack));
+    const uint32_t r_lo = (uint32_t)fminf((float)S, ceilf(r + slack));
+    find_bin(hist, kBins, r_hi, sm);
+    const uint32_t b_hi = sm->res_bin;
+    find_bin(hist, kBins, r_lo, sm);
+    const uint32_t b_lo = sm->res_bin;
+    const uint32_t wlo = lo + (b_lo << shift);
+    const uint32_t whi = min(hi, lo + (b_hi << shift) + ((1u << shift) - 1u));
+    const int wshift = range_shift(wlo, whi);
+    for (int i = threadIdx.x; i < kBins; i += kEpiThreads) hist[i] = 0u;
+    named_bar_sync(1, kEpiThreads);
+    uint32_t above = 0, inside = 0;
+    for (int i0 = 0; i0 < n; i0 += kEpiThreads * kU) {
+        uint32_t k[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+            k[u] = i < n ? st.key(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+            const bool in = i < n && k[u] >= wlo && k[u] <= whi;
+            above += (i < n && k[u] > whi);
+            inside += in;
+            hist_add(hist, in, (k[u] - wlo) >> wshift);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        above += __shfl_xor_sync(0xffffffffu, above, o);
+        inside += __shfl_xor_sync(0xffffffffu, inside, o);
+    }
+    if (lane == 0) {
+        sm->wcnt[warp][0] = above;
+        sm->wcnt[warp][1] = inside;
+    }
+    named_bar_sync(1, kEpiThreads);
+    above = inside = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        above += sm->wcnt[w][0];
+        inside += sm->wcnt[w][1];
+    }
+    named_bar_sync(1, kEpiThreads);
+    if (above < kk && kk <= above + inside)
+        return find_threshold(st, wlo, whi, kk - above, hist, list, sm, true);
+    return find_threshold(st, lo, hi, kk, hist, list, sm);
+}
+
 struct GroupView {
     uint32_t* sync;     // {count, gen}
     uint32_t* hdr;      // [ranks][NQ][4]: published count, smallest published key, largest key, edge
@@ -616,7 +692,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         uint32_t T, take = 0, base = 0;
         if (G == 1) {
             // ---- exact threshold over this CTA's own scores
-            T = find_threshold(ScoreStream{sj, nloc[j]}, sm->kmin[j], sm->kmax[j], K, s_hist, s_list, sm);
+            T = sampled_threshold(ScoreStream{sj, nloc[j]}, sm->kmin[j], sm->kmax[j], K, s_hist, s_list, sm);
         } else {
             // ---- 2. threshold over the published keys
             gather(j);

@@ -112,6 +112,11 @@ class Workload:
             per += 4 * (self.D_I // 64)
         return int(np.sum(self.seq_lens.astype(np.int64))) * per
 
+    def indexer_flops(self) -> int:
+        """Tensor-core work of the indexer: 2 * H_I * D_I per visible (token, position) pair."""
+        vis = self.token_pos().astype(np.int64) + 1
+        return int(np.sum(vis)) * 2 * self.H_I * self.D_I
+
     def kv_bytes(self) -> int:
         """Latent-cache bytes gathered by sparse attention: min(K, visible) rows per token."""
         vis = self.token_pos() + 1

@@ -32,6 +32,34 @@ def test_tie_heavy_groups_split_ties_by_position():
     assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
 
 
+def test_tie_heavy_long_rows_one_cta_per_token_bit_exact():
+    # many tokens of one sequence (one CTA per token) with rows long enough for
+    # the sampled window of the single-CTA select; integer scores tie heavily
+    wl = W.make_workload("ties3", seq_lens=[9000], nq=3, H_I=8, D_I=64, H=1, K=1024, int_inputs=True,
+                         w_dist="ones", seed=12, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
+
+
+def test_single_cta_select_when_the_sample_misses_the_top():
+    # the largest scores sit only at positions a strided sample of 512 never
+    # reads (position % 17 == 1 with rows of ~9000 keys, sample stride 17), so
+    # the sampled window lies below the K-th score and the exact search over
+    # the whole range must take over
+    wl = W.make_workload("miss", seq_lens=[9000], nq=3, H_I=8, D_I=64, H=1, K=256, int_inputs=True,
+                         w_dist="u256", seed=13, with_kv=False)
+    q = W.bf16_bits_to_f32(wl.q_idx).astype(np.float64)          # [T, H_I, D_I]
+    dirn = np.sign(np.einsum("th,thd->d", wl.w.astype(np.float64), q))
+    dirn[dirn == 0] = 1.0
+    planted = np.arange(1, 9000, 17)
+    rows = wl.block_table[0, planted // 64].astype(np.int64) * 64 + planted % 64
+    k = wl.k_idx.reshape(-1, wl.D_I)
+    k[rows] = W.to_bf16_bits((4.0 * dirn)[None, :].repeat(len(rows), 0).astype(np.float32))
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
+    assert np.isin(idx, planted).mean() > 0.9
+
+
 @pytest.mark.parametrize("key_dtype", ["bf16", "fp8"])
 def test_topk_concentrated_in_few_ctas(key_dtype):
     # the whole Top-K in the last 2048 positions: the CTAs holding them publish
