@@ -479,7 +479,6 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                     float acc = 0.0f;
                     if (j < item.nq) {
                         constexpr int CW = HI < 32 ? HI : 32;
-                        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
                         for (int c0 = 0; c0 < HI; c0 += CW) {
                             uint32_t a0[32], a1[32];
@@ -495,25 +494,16 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                                 if (FP8 && Cfg::KB > 1) tmem_ld8(tb + Cfg::N + col, *reinterpret_cast<uint32_t(*)[8]>(a1));
                             }
                             tmem_wait_ld();
-                            // four partial sums (independent FMA chains); head weights as float4
-                            const float4* w4 = reinterpret_cast<const float4*>(s_w + j * HI + c0);
 #pragma unroll
-                            for (int h4 = 0; h4 < CW / 4; ++h4) {
-                                const float4 wv = w4[h4];
-                                const float wq[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int h = h4 * 4 + e;
-                                    float x = __uint_as_float(a0[h]);
-                                    if (FP8) {
-                                        x = x * sc[0];
-                                        if (Cfg::KB > 1) x = fmaf(__uint_as_float(a1[h]), sc[1], x);
-                                    }
-                                    part[e] = fmaf(wq[e], fmaxf(x, 0.0f), part[e]);
+                            for (int h = 0; h < CW; ++h) {
+                                float x = __uint_as_float(a0[h]);
+                                if (FP8) {
+                                    x = x * sc[0];
+                                    if (Cfg::KB > 1) x = fmaf(__uint_as_float(a1[h]), sc[1], x);
                                 }
+                                acc = fmaf(s_w[j * HI + c0 + h], fmaxf(x, 0.0f), acc);
                             }
                         }
-                        acc = (part[0] + part[1]) + (part[2] + part[3]);
                     }
                     score[j] = acc;
                 }

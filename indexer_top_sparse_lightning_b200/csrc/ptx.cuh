@@ -107,7 +107,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t addr, uint32_t pa
 }
 
 // Bounded wait for the phase with the given parity.  Returns false on
-// timeout or when *abort becomes non-zero (another role gave up).
+// timeout or when *abort becomes non-zero (another role gave up).  A wait
+// that has lasted more than 2 us (another role is in a long phase, e.g. a
+// Top-K pass) sleeps between probes, so that the probing lanes do not take
+// shared-memory pipe slots from the warps doing that work.
+__device__ __forceinline__ void wait_backoff(uint64_t waited_ns) {
+    if (waited_ns > 2000) __nanosleep(waited_ns > 20000 ? 1000u : 200u);
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
@@ -117,7 +123,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(a, parity)) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+        const uint64_t dt = globaltimer() - t0;
+        if (dt > kWaitTimeoutNs) return false;
+        wait_backoff(dt);
     }
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -129,7 +137,9 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait_cluster(a, parity)) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kWaitTimeoutNs) return false;
+        const uint64_t dt = globaltimer() - t0;
+        if (dt > kWaitTimeoutNs) return false;
+        wait_backoff(dt);
     }
 }
 

@@ -767,21 +767,28 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
 
         // ---- per-warp counts of this CTA's elements above / equal to T, over
         // the warp's position-ordered sequence (list or quarter)
+        // (float compares against T's value: the same order as the keys for
+        // finite scores, and -0 == +0 like the folded keys)
         const int n = seq_len(j);
+        const float Tf = key_to_float(T);
         uint32_t gt = 0, eq = 0;
         for (int q0 = 0; q0 < n; q0 += 32 * kU) {
-            uint32_t k[kU];
+            float f[kU];
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const int t = q0 + u * 32 + lane;
-                k[u] = t < n ? order_key(sj[seq_idx(j, t)]) : 0u;
+                f[u] = t < n ? sj[seq_idx(j, t)] : -__int_as_float(0x7f800000);
             }
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
-                const int t = q0 + u * 32 + lane;
-                gt += __popc(__ballot_sync(0xffffffffu, t < n && k[u] > T));
-                eq += __popc(__ballot_sync(0xffffffffu, t < n && k[u] == T));
+                gt += f[u] > Tf;
+                eq += f[u] == Tf;
             }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            gt += __shfl_xor_sync(0xffffffffu, gt, o);
+            eq += __shfl_xor_sync(0xffffffffu, eq, o);
         }
         if (lane == 0) {
             sm->wcnt[warp][0] = gt;
@@ -826,9 +833,8 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const int t = q0 + u * 32 + lane;
-                const uint32_t key = order_key(f[u]);
-                const bool is_gt = t < n && key > T;
-                const bool is_eq = t < n && key == T;
+                const bool is_gt = t < n && f[u] > Tf;
+                const bool is_eq = t < n && f[u] == Tf;
                 const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
                 const bool sel = is_gt || (is_eq && eq_seen + __popc(eqm & lt_mask) < allow);
                 const uint32_t selm = __ballot_sync(0xffffffffu, sel);
