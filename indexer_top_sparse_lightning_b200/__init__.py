@@ -24,8 +24,7 @@ __all__ = ["Batch", "Workspace", "indexer_topk", "sparse_mla_attn", "dsa_decode"
            "DsaError", "library_path", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# DSA_LIBRARY selects another build of the same library (e.g. a tracing build)
-_LIB_PATH = os.environ.get("DSA_LIBRARY") or os.path.join(_HERE, "libdsa.so")
+_LIB_PATH = os.path.join(_HERE, "libdsa.so")
 _lib = None
 
 KEY_BF16 = 0

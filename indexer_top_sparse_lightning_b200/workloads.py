@@ -187,7 +187,9 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
     seq_lens: per-sequence cached lengths (including the step's own tokens).
     nq: query tokens per sequence (int, or a list); tokens are the last nq positions.
     w_dist: "u8" -> U(0,1)/sqrt(H_I); "u" -> U(0,1); "u256" -> U(0,1) rounded to 2^-8;
-            "ones" -> all 1 (integer scores with many ties when int_inputs is set).
+            "ones" -> all 1 (integer scores with many ties when int_inputs is set);
+            "signed" -> U(-1,1) (rounded to 2^-8 when int_inputs is set, so that fp32
+            scores stay exact): negative weights give negative scores.
     int_inputs: indexer q/k drawn as integers in [-4, 4] (exact fp32 scores).
     planted_k: if > 0 (single sequence, one token), plant a dominant set of that many
                positions: seed-chosen, or the last planted_k positions if planted_tail.
@@ -215,6 +217,11 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
         w = u.astype(np.float32)
     elif w_dist == "ones":
         w = np.ones((T, H_I), dtype=np.float32)
+    elif w_dist == "signed":
+        v = 2.0 * u - 1.0
+        if int_inputs:
+            v = np.round(v * 256.0) / 256.0
+        w = v.astype(np.float32)
     else:
         w = (u / math.sqrt(H_I)).astype(np.float32)
 

@@ -75,17 +75,17 @@ def test_cuda_graph_capture_matches_eager():
 
 @pytest.mark.slow
 def test_batch32_decode_sampled():
-    check(W.preset("batch32"), [0, 17, 31], exact=False)
+    check(W.preset("batch32"), np.arange(0, 32, 3), exact=False)
 
 
 @pytest.mark.slow
 def test_prefill16k_sampled():
-    check(W.preset("prefill16k"), [0, 2047, 2048, 16383], exact=False)
+    check(W.preset("prefill16k"), [0, 2047, 2048, 5000, 11111, 16383], exact=False)
 
 
 @pytest.mark.slow
 def test_ragged_decode_sampled():
-    check(W.preset("ragged"), [0, 1, 9, 15], exact=False)
+    check(W.preset("ragged"), np.arange(16), exact=False)
 
 
 @pytest.mark.slow

@@ -94,6 +94,36 @@ def test_fp8_keys(nq):
     assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
 
 
+@pytest.mark.parametrize("seq_lens,nq", [([3000], 1), ([20000, 9000, 130], [1, 2, 1])],
+                         ids=["one_cta", "groups"])
+def test_signed_weights_integer_inputs_bit_exact(seq_lens, nq):
+    # w in [-1, 1] on a 2^-8 grid with integer q/k: exact fp32 scores of either sign,
+    # many of them negative; the order keys of negative scores and the -0/+0 fold
+    # decide the selection, which must equal the oracle's bit for bit
+    wl = W.make_workload("neg_int", seq_lens=seq_lens, nq=nq, H_I=8, D_I=64, H=1, K=1024, int_inputs=True,
+                         w_dist="signed", seed=14, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
+
+
+@pytest.mark.parametrize("key_dtype,nq", [("bf16", 1), ("bf16", 2), ("fp8", 1), ("fp8", 2)])
+def test_signed_weights_general_inputs(key_dtype, nq):
+    # K above half the context: the K-th score is negative for most tokens
+    wl = W.make_workload("neg", seq_lens=[3000, 17000, 700], nq=nq, H_I=64, D_I=128, H=1, K=2048,
+                         key_dtype=key_dtype, w_dist="signed", seed=15, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+@pytest.mark.parametrize("H_I,D_I", [(8, 64), (16, 64), (32, 64), (16, 128)])
+def test_fp8_keys_other_shapes(H_I, D_I):
+    # one scale group per key when D_I = 64
+    wl = W.make_workload("fp8s", seq_lens=[1000, 6000, 13000], nq=[1, 2, 1], H_I=H_I, D_I=D_I, H=1, K=512,
+                         key_dtype="fp8", seed=16, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
 def test_contexts_around_k():
     # fewer visible than K: every visible position, -1 padded; around the boundary
     lens = [1, 63, 64, 65, 127, 128, 129, 2047, 2048, 2049, 4100]
@@ -161,7 +191,7 @@ def test_out_of_range_block_id_is_reported_not_fatal():
 def test_batch32_full_size_sampled():
     wl = W.preset("batch32", with_kv=False)
     idx, score = run_indexer(wl)
-    tok = np.array([0, 13, 31])
+    tok = np.arange(wl.T)                                # every token of the batch
     assert_topk(wl, tok, idx[tok], score[tok], exact=False)
 
 
@@ -169,7 +199,8 @@ def test_batch32_full_size_sampled():
 def test_prefill16k_full_size_sampled():
     wl = W.preset("prefill16k", with_kv=False)
     idx, score = run_indexer(wl)
-    tok = np.array([0, 1, 2046, 2047, 2048, 9000, 16383])
+    # 64 evenly spaced tokens plus both sides of the take-all / select boundary
+    tok = np.unique(np.concatenate([np.linspace(0, wl.T - 1, 64).astype(np.int64), [0, 1, 2046, 2047, 2048, 16383]]))
     assert_topk(wl, tok, idx[tok], score[tok], exact=False)
 
 
@@ -177,7 +208,7 @@ def test_prefill16k_full_size_sampled():
 def test_ragged_fp8_full_size_sampled():
     wl = W.preset("ragged", with_kv=False)
     idx, score = run_indexer(wl)
-    tok = np.array([0, 1, 7, 14, 15])
+    tok = np.arange(wl.T)
     assert_topk(wl, tok, idx[tok], score[tok], exact=False)
 
 

@@ -97,6 +97,56 @@ def test_hand_softmax_two_rows():
     assert abs(lse[0, 0] - g["lse"]) < 1e-14
 
 
+def test_hand_score_pairs():
+    # the pair scorer on the hand-worked cases above
+    g = GOLD["indexer_relu_tie"]
+    wl = manual_workload(g["q"], g["w"], g["keys"], K=1)
+    got = oracle.score_pairs(wl, np.zeros(4, np.int32), np.array([0, 1, 2, 3]))
+    np.testing.assert_array_equal(got[:3], np.array(g["scores"]))
+    assert np.isnan(got[3])                       # position 3 is past the token's own position
+    g = GOLD["fp8_scale_groups"]
+    q = np.zeros((1, 128), np.float32)
+    q[0, 0] = 1.0
+    q[0, 64] = 1.0
+    codes = np.zeros((1, 128), np.uint8)
+    codes[0, 0] = g["code0"]
+    codes[0, 64] = g["code64"]
+    wl = manual_workload(q, [1.0], None, K=1, key_dtype="fp8", k_codes=codes,
+                         k_scale=np.array([g["scales"]], np.float32))
+    assert oracle.score_pairs(wl, np.zeros(1, np.int32), np.zeros(1, np.int64))[0] == g["score"]
+
+
+@pytest.mark.parametrize("kw", [dict(key_dtype="bf16"), dict(key_dtype="fp8"),
+                                dict(key_dtype="bf16", w_dist="signed")], ids=["bf16", "fp8", "signed"])
+def test_score_pairs_match_full_score_rows(kw):
+    # the pair scorer is a second implementation of the score (it judges near-ties in
+    # the GPU parity tests); at sampled pairs it must equal the full rows pinned above:
+    # paged and shuffled, several tokens per sequence, both causal edges
+    wl = W.make_workload("sp", seq_lens=[300, 900, 70], nq=[1, 3, 2], H_I=16, D_I=128, H=1, K=64, seed=17,
+                         with_kv=False, **kw)
+    r = oracle.indexer_topk(wl, want_all_scores=True)
+    pos = wl.token_pos()
+    rng = np.random.default_rng(5)
+    for t in range(wl.T):
+        p = int(pos[t])
+        ps = np.concatenate([[0, p, max(p - 1, 0)], rng.integers(0, p + 1, 40)]).astype(np.int64)
+        got = oracle.score_pairs(wl, np.full(len(ps), t, np.int32), ps)
+        np.testing.assert_array_equal(got, r["all"][t, ps])
+    assert np.all(np.isnan(oracle.score_pairs(wl, np.arange(wl.T, dtype=np.int32), pos + 1)))
+
+
+def test_signed_weights_give_negative_scores_and_rank_them():
+    # weights of either sign: scores below zero exist and are ranked like any other
+    wl = W.make_workload("neg", seq_lens=[500], nq=1, H_I=8, D_I=64, H=1, K=450, seed=19, w_dist="signed",
+                         with_kv=False)
+    assert (wl.w < 0).any() and (wl.w > 0).any()
+    r = oracle.indexer_topk(wl, want_all_scores=True)
+    s = r["all"][0]
+    assert (s < 0).sum() > 50
+    order = np.lexsort((np.arange(len(s)), -s))
+    np.testing.assert_array_equal(r["idx"][0], np.sort(order[:wl.K]))
+
+
 # ----------------------------------------------------------------------------- library routines
 
 def test_e4m3_decode_all_codes_vs_torch():

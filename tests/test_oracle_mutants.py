@@ -30,11 +30,18 @@ MUTANTS = [
      "out_idx[o] = j < nk ? (int32_t)keep[j] : 0;"),
     ("e4m3_bias_8", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
      "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("pair_score_without_relu", "acc += (double)a->w[(int64_t)t * a->H_I + h] * (dot > 0.0 ? dot : 0.0);",
+     "acc += (double)a->w[(int64_t)t * a->H_I + h] * dot;"),
+    ("pair_score_weight_transposed", "acc += (double)a->w[(int64_t)t * a->H_I + h] * (dot > 0.0 ? dot : 0.0);",
+     "acc += (double)a->w[(int64_t)t * a->H_I + (a->H_I - 1 - h)] * (dot > 0.0 ? dot : 0.0);"),
+    ("pair_score_causal_edge", "if (s < 0 || s > pos) { out[i] = NAN; continue; }",
+     "if (s < 0 || s >= pos) { out[i] = NAN; continue; }"),
     ("softmax_value_from_rope", "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d]);",
      "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d + 64]);"),
 ]
 
 PINS = [pins.test_hand_indexer_relu_gate_weights_and_tie, pins.test_hand_fp8_scale_groups,
+        pins.test_hand_score_pairs, lambda: pins.test_score_pairs_match_full_score_rows(dict(key_dtype="bf16")),
         pins.test_hand_softmax_two_rows, pins.test_e4m3_decode_all_codes_vs_torch,
         pins.test_single_head_unit_weight_is_relu_dot_lexsort,
         pins.test_k_at_least_context_equals_dense_causal_attention]
@@ -55,5 +62,5 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new):
             try:
                 pin()
             except AssertionError:
-                caught.append(pin.__name__)
+                caught.append(getattr(pin, "__name__", "pin"))
     assert caught, f"no pin caught the planted mistake {name}"
