@@ -110,17 +110,24 @@ typedef struct {
 /*
  * Bytes of workspace needed for this batch shape by indexer_topk (ix given),
  * sparse_mla_attn (at given) or both / dsa_decode (both given).  The
- * layout is [256-byte status word area][1 KB of split arrival counters]
- * [indexer group region, a fixed size per device][attention split
- * partials]; one buffer sized with both serves all three entry points, for
- * any mix of shapes.
+ * layout is [256-byte status area][indexer group region and published-key
+ * slots, a fixed size per device][attention split counters, a fixed size per
+ * device][attention partial slots, sized for the largest Top-K]; one buffer
+ * sized with both serves all three entry points, for any mix of shapes.
  * The workspace must be 256-byte aligned and ZERO-FILLED before its first
  * use.  After that the library keeps it consistent by itself (a call that
  * completes without a device error leaves its histograms zero and its
- * barrier counters at rest), so it can be reused by later calls on the same
- * stream; the caller must not modify it.  After a device error
+ * barrier and split counters at rest), so it can be reused by later calls on
+ * the same stream; the caller must not modify it.  After a device error
  * (dsa_get_status != OK) zero-fill it again.  Calls sharing one workspace
  * must not overlap in time.
+ * Status area: int32 word 0 is the device status read by dsa_get_status.
+ * Words 1 and 2 are test hooks of the library's own failure tests and must
+ * stay zero in normal use: word 1 shortens every bounded device wait to that
+ * many microseconds (0 = the default of one second), word 2 injects a wait
+ * that runs out (bit 0: an indexer group barrier waits for one CTA more than
+ * its group has; bit 1: in the attention kernel the second CTA of each pair
+ * never reports its first rows).
  * Returns 0 if the shape is invalid.
  */
 DSA_API size_t dsa_workspace_size(const dsa_batch* batch, const dsa_indexer_inputs* ix,
@@ -144,6 +151,9 @@ DSA_API dsa_status indexer_topk(const dsa_batch* batch, const dsa_indexer_inputs
  * logical positions; negative entries are skipped).
  * out device [T, H, 512] bf16; lse device [T, H] fp32 natural-log
  * log-sum-exp of the scaled logits (-inf if a token selects nothing) or NULL.
+ * The launch is a programmatic dependent of the preceding kernel on the
+ * stream: its prologue may overlap that kernel's end, and it reads nothing
+ * (inputs, index list, workspace counters) before that kernel has completed.
  */
 DSA_API dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs* at,
                            const int32_t* idx, int32_t K,
@@ -156,12 +166,16 @@ DSA_API dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs
  * device memory for the workspace -- code that must not allocate on the
  * device, or that has no device allocator at hand.  The function itself
  * allocates nothing: it uses a fixed 20 MiB scratch array inside the library
- * module (status word, split counters, split partials), zero when the module
- * loads and left zeroed by every call that completes without a device error.
+ * module (status area, split counters, partial slots), which every GPU that
+ * loads the library holds until the process exits.
  * Arguments, layouts and results are those of sparse_mla_attn.
- *  - The first call on a device looks up that device's scratch address (with
- *    the device current); make it before any latency-critical use.
- *  - Shapes whose split plan needs more scratch than 20 MiB are rejected with
+ *  - The first call on a device (and the first after that device's context
+ *    changes) looks up the scratch address with the device current; make it
+ *    before any latency-critical use.
+ *  - Each call first clears the scratch's status area and split counters on
+ *    the stream (one memset), so a call that ended in a device error leaves
+ *    nothing behind for later calls.
+ *  - Shapes whose plan needs more scratch than 20 MiB are rejected with
  *    DSA_ERR_WORKSPACE (dsa_last_error() gives both sizes); on a 148-SM B200
  *    every shape fits.
  *  - All calls on a device share the one scratch: calls whose device work
@@ -179,7 +193,9 @@ DSA_API dsa_status sparse_mla_attn_static(const dsa_batch* batch, const dsa_attn
  * The whole decode step: indexer_topk then sparse_mla_attn on one stream,
  * without a host synchronization in between.  out_idx [T, K] is required
  * (it carries the index list between the stages); out_score and lse may be
- * NULL.
+ * NULL.  The attention launch depends programmatically on the indexer
+ * launch: its prologue and the first token's query load overlap the end of
+ * the indexer, and it reads the index list only after the indexer completed.
  */
 DSA_API dsa_status dsa_decode(const dsa_batch* batch, const dsa_indexer_inputs* ix,
                       const dsa_attn_inputs* at,

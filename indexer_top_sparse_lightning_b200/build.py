@@ -2,9 +2,10 @@
 
     python -m indexer_top_sparse_lightning_b200.build [--force] [--verbose]
 
-nvcc cross-compiles for sm_100a without a GPU.  The CUDA runtime is linked
-statically and the driver entry point for TMA descriptors is fetched at run
-time, so the library loads on machines without a GPU driver.
+nvcc cross-compiles for sm_100a without a GPU, one process per translation
+unit in parallel.  The CUDA runtime is linked statically and the driver entry
+points (TMA descriptor encoding, current context) are fetched at run time, so
+the library loads on machines without a GPU driver.
 """
 from __future__ import annotations
 
@@ -46,15 +47,46 @@ def nvcc() -> str:
     return "nvcc"
 
 
+def units():
+    """Translation units: the C ABI and attention kernel, the host helpers, and one
+    unit per indexer key type and head count (compiled in parallel)."""
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not stale():
         return LIB
+    import concurrent.futures
+    import tempfile
+    tmpdir = tempfile.mkdtemp(prefix="dsa_build_")
+    objs = []
+
+    def compile_one(src):
+        obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *NVCC_FLAGS, *extra, "-c", "-o", obj, src]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if verbose or r.returncode:
+            sys.stdout.write(r.stdout)
+            sys.stderr.write(r.stderr)
+        if r.returncode:
+            raise subprocess.CalledProcessError(r.returncode, cmd)
+        return obj
+
+    srcs = units()
+    workers = max(1, min(len(srcs), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+        objs = list(ex.map(compile_one, srcs))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-shared", "-o", tmp, os.path.join(CSRC, "api.cu")]
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
     os.replace(tmp, LIB)
+    for o in objs:
+        os.remove(o)
+    os.rmdir(tmpdir)
     return LIB
 
 

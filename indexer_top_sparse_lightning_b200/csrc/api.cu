@@ -11,80 +11,24 @@
 
 #include "../../include/dsa.h"
 #include "common.h"
+#include "host.h"
 #include "indexer.cuh"
 #include "sfa.cuh"
 
 using namespace dsa;
+using namespace dsa::host;
 
 static_assert(sizeof(IdxMisc) <= 1024, "indexer misc block exceeds its slot");
 static_assert(sizeof(SfaMisc) <= SfaCfg::MISC_BYTES, "attention misc block exceeds its slot");
 
 namespace {
 
+// Status area at the start of every workspace: word 0 = device status, word 1 =
+// bounded-wait limit in microseconds (0: the 1 s default), word 2 = fault
+// injection bits (test hooks; zero in normal use).
 constexpr size_t kStatusBytes = 256;
-constexpr int kMaxSplitTokens = 128;      // row splits are only used for fewer tokens than this
-constexpr size_t kCounterBytes = kMaxSplitTokens * 2 * 2 * 4;   // split arrivals and ready counts
-constexpr size_t kHeaderBytes = kStatusBytes + kCounterBytes;
+constexpr size_t kHeaderBytes = kStatusBytes;
 
-// ------------------------------------------------------------------ last failure text (per host thread)
-thread_local char g_last_error[256] = "";
-
-dsa_status fail(dsa_status st, const char* what, cudaError_t e = cudaSuccess) {
-    if (e != cudaSuccess)
-        snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
-    else
-        snprintf(g_last_error, sizeof g_last_error, "%s", what);
-    return st;
-}
-
-// ------------------------------------------------------------------ driver entry point (no libcuda link)
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
-              CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t d[5], s[4];
-    cuuint32_t b[5], e[5];
-    for (int i = 0; i < rank; ++i) {
-        d[i] = dims[i];
-        b[i] = box[i];
-        e[i] = 1;
-        if (i + 1 < rank) s[i] = strides_bytes[i];
-    }
-    return fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-              promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-struct DevInfo {
-    int sms = 0;
-    int max_smem = 0;
-};
-
-DevInfo dev_info() {
-    int dev = 0;
-    DevInfo di;
-    if (cudaGetDevice(&dev) != cudaSuccess) return di;
-    cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaDeviceGetAttribute(&di.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    return di;
-}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -117,26 +61,8 @@ dsa_status check_attn(const dsa_attn_inputs* at) {
     return DSA_OK;
 }
 
-size_t align256(size_t v);
-size_t group_region_bytes(int sms);
 
 // ------------------------------------------------------------------ indexer planning
-struct IdxPlan {
-    int mode = 0;        // 0 grouped decode, 1 per-token
-    int nq = 1;          // kernel NQ
-    int grid = 0;        // CTAs per launch
-    int seqs_per_launch = 0;
-    int score_cap = 0;
-    int smem = 0;
-    size_t group_ws = 0; // bytes of group workspace per launch
-};
-
-template <bool FP8, int HI, int DI, int NQ>
-struct IdxKernel {
-    using Cfg = IdxCfg<FP8, HI, DI, NQ>;
-    static void* fn() { return reinterpret_cast<void*>(&indexer_topk_kernel<FP8, HI, DI, NQ>); }
-};
-
 // Fill the fields that depend on the kernel instantiation.
 template <bool FP8, int HI, int DI, int NQ>
 bool plan_for(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl) {
@@ -169,96 +95,6 @@ bool plan_for(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl) {
     // between calls; everything else is)
     pl.group_ws = (size_t)bp * (size_t)group_ws_bytes(2, pl.grid);
     return true;
-}
-
-using LaunchFn = dsa_status (*)(const dsa_batch*, const dsa_indexer_inputs*, int32_t*, float*, uint32_t*,
-                                uint8_t*, const IdxPlan&, cudaStream_t);
-
-template <bool FP8, int HI, int DI, int NQ>
-dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int32_t* out_idx, float* out_score,
-                          uint32_t* status, uint8_t* group_ws, const IdxPlan& pl, cudaStream_t stream) {
-    using Cfg = IdxCfg<FP8, HI, DI, NQ>;
-    CUtensorMap tm_q, tm_k;
-    {
-        const uint64_t dims[3] = {(uint64_t)DI, (uint64_t)HI, (uint64_t)bt->num_tokens};
-        const uint64_t strides[2] = {(uint64_t)DI * 2, (uint64_t)HI * DI * 2};
-        const uint32_t box[3] = {64, (uint32_t)HI, (uint32_t)NQ};
-        if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ix->q_idx, dims, strides, box,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-            return fail(DSA_ERR_CUDA, "indexer query tensor map encoding failed");
-    }
-    {
-        const uint64_t dims[2] = {(uint64_t)DI, (uint64_t)bt->num_blocks * kPage};
-        if (FP8) {
-            const uint64_t strides[1] = {(uint64_t)DI};
-            const uint32_t box[2] = {(uint32_t)DI, (uint32_t)kPage};
-            if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ix->k_cache, dims, strides, box,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
-                return fail(DSA_ERR_CUDA, "indexer key tensor map encoding failed");
-        } else {
-            const uint64_t strides[1] = {(uint64_t)DI * 2};
-            const uint32_t box[2] = {64, (uint32_t)kPage};
-            if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ix->k_cache, dims, strides, box,
-                          CU_TENSOR_MAP_SWIZZLE_128B))
-                return fail(DSA_ERR_CUDA, "indexer key tensor map encoding failed");
-        }
-    }
-    auto kern = &indexer_topk_kernel<FP8, HI, DI, NQ>;
-    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem))
-        return fail(DSA_ERR_CUDA, "indexer shared memory attribute", e);
-
-    IndexerParams p;
-    memset(&p, 0, sizeof p);
-    p.seq_lens = bt->seq_lens;
-    p.cu_q = bt->cu_q;
-    p.block_table = bt->block_table;
-    p.w = ix->w;
-    p.k_scale = ix->k_scale;
-    p.out_idx = out_idx;
-    p.out_score = out_score;
-    p.status = status;
-    p.group_ws = group_ws;
-    p.group_ws_stride = group_ws_bytes(2, pl.grid);
-    p.cand = reinterpret_cast<uint32_t*>(group_ws + group_region_bytes(pl.grid));
-    p.cand_slot = kCandSlotKeys;
-    p.B = bt->batch;
-    p.T = bt->num_tokens;
-    p.max_blocks = bt->max_blocks_per_seq;
-    p.num_blocks = bt->num_blocks;
-    p.mode = pl.mode;
-    p.K = ix->K;
-    p.score_cap = pl.score_cap;
-
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof cfg);
-    cudaLaunchAttribute attr[1];
-    cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)pl.smem;
-    cfg.stream = stream;
-    if (pl.mode == 1) {
-        int grid = pl.grid;
-        if (grid > bt->num_tokens) grid = bt->num_tokens;
-        cfg.gridDim = dim3(grid, 1, 1);
-        cfg.attrs = nullptr;
-        cfg.numAttrs = 0;
-        p.t_begin = 0;
-        p.t_end = bt->num_tokens;
-        if (cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, tm_q, tm_k)) return fail(DSA_ERR_CUDA, "indexer launch", e);
-        return DSA_OK;
-    }
-    // grouped mode: the CTAs of a group wait for one another, so they must be
-    // co-resident -- a cooperative launch guarantees it (or fails)
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cfg.gridDim = dim3(pl.grid, 1, 1);
-    for (int b0 = 0; b0 < bt->batch; b0 += pl.seqs_per_launch) {
-        p.b_begin = b0;
-        p.b_end = b0 + pl.seqs_per_launch < bt->batch ? b0 + pl.seqs_per_launch : bt->batch;
-        if (cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, tm_q, tm_k)) return fail(DSA_ERR_CUDA, "indexer launch", e);
-    }
-    return DSA_OK;
 }
 
 template <bool FP8, int HI, int DI, int NQ>
@@ -306,27 +142,33 @@ dsa_status plan_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, const
 }
 
 // ------------------------------------------------------------------ attention planning
+// The selected rows of all tokens form T * ceil(K/64) blocks of 64 rows; each
+// two-CTA cluster ("pair") of the grid takes a contiguous range of them.  All
+// SM pairs are used once there are at least two blocks per pair.
 struct AttnPlan {
-    int splits = 1;
-    int rows_per_split = 0;
-    size_t part_bytes = 0;
+    int pairs = 1;
+    int64_t total_blocks = 0;
+    size_t counter_bytes = 0;   // split arrival counters, [SM pairs][2], the same for every shape
+    size_t slot_bytes = 0;      // partial slots, [pairs][2 sides][2 CTAs]
 };
 
 AttnPlan plan_attn(const dsa_batch* bt, int K, const DevInfo& di) {
     AttnPlan ap;
-    const int max_splits = (K + SfaCfg::ROWS - 1) / SfaCfg::ROWS;
-    int s = di.sms / (2 * bt->num_tokens);
-    if (s < 1 || bt->num_tokens > kMaxSplitTokens) s = 1;
-    if (s > max_splits) s = max_splits;
-    const int per = (K + s - 1) / s;
-    ap.rows_per_split = ((per + SfaCfg::ROWS - 1) / SfaCfg::ROWS) * SfaCfg::ROWS;
-    ap.splits = (K + ap.rows_per_split - 1) / ap.rows_per_split;
-    if (ap.splits > 1)
-        ap.part_bytes = (size_t)bt->num_tokens * ap.splits * (128 * kDv * 4 + 2 * 256 * 4);
+    const int nb = (K + SfaCfg::ROWS - 1) / SfaCfg::ROWS;
+    ap.total_blocks = (int64_t)bt->num_tokens * nb;
+    // at least kMinBlocks blocks per pair: fewer pairs share a token when there are few
+    // blocks, which keeps the merge of their partials short
+    constexpr int64_t kMinBlocks = 8;
+    const int pmax = di.sms / 2 > 0 ? di.sms / 2 : 1;
+    int64_t np = ap.total_blocks / kMinBlocks;
+    if (np > pmax) np = pmax;
+    if (np < 1) np = 1;
+    ap.pairs = (int)np;
+    ap.counter_bytes = ((size_t)pmax * 2 * 4 + 255) & ~size_t(255);
+    ap.slot_bytes = (size_t)ap.pairs * 2 * 2 * (size_t)SfaCfg::SLOT_BYTES;
     return ap;
 }
 
-size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace layout, the same for every shape on a given device:
 //   [status 256 B][split arrival counters 1 KB][indexer group region, fixed
@@ -334,13 +176,13 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // The indexer regions are sized for the largest grouped launch (one group per
 // SM, two tokens per group), so calls of any shape sharing one workspace
 // never write attention partials over the indexer's barrier words.
-size_t group_region_bytes(int sms) { return align256((size_t)sms * (size_t)group_ws_bytes(2, sms)); }
 size_t idx_region_bytes(const DevInfo& di) {
     return group_region_bytes(di.sms) + align256((size_t)di.sms * (size_t)kCandSlotKeys * 4);
 }
 
 dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int32_t* idx, int K, void* out,
-                       float* lse, uint32_t* status, uint8_t* part, const AttnPlan& ap, cudaStream_t stream) {
+                       float* lse, uint32_t* status, uint8_t* attn_ws, const AttnPlan& ap, cudaStream_t stream,
+                       bool dependent, bool early_q) {
     CUtensorMap tm_q;
     const uint64_t dims[3] = {(uint64_t)kDqk, (uint64_t)at->H, (uint64_t)bt->num_tokens};
     const uint64_t strides[2] = {(uint64_t)kDqk * 2, (uint64_t)at->H * kDqk * 2};
@@ -348,8 +190,18 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     const uint32_t box[3] = {64, (uint32_t)(at->H < 64 ? at->H : 64), 1};
     if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, at->q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return fail(DSA_ERR_CUDA, "attention query tensor map encoding failed");
-    if (cudaError_t e = cudaFuncSetAttribute(&sfa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SfaCfg::SMEM))
+    // latent cache as [rows, 576] with one-row boxes of 64 columns, 128-byte swizzle: the
+    // kernel's row gathers (tile::gather4) fetch four rows of one box each
+    CUtensorMap tm_kv;
+    {
+        const uint64_t kdims[2] = {(uint64_t)kDqk, (uint64_t)bt->num_blocks * kPage};
+        const uint64_t kstrides[1] = {(uint64_t)kDqk * 2};
+        const uint32_t kbox[2] = {64, 1};
+        if (!make_map(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, at->kv_cache, kdims, kstrides, kbox,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return fail(DSA_ERR_CUDA, "latent cache tensor map encoding failed");
+    }
+    if (cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(&sfa_decode_kernel), SfaCfg::SMEM))
         return fail(DSA_ERR_CUDA, "attention shared memory attribute", e);
     SfaParams p;
     memset(&p, 0, sizeof p);
@@ -367,65 +219,92 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     p.K = K;
     p.max_blocks = bt->max_blocks_per_seq;
     p.num_blocks = bt->num_blocks;
-    p.n_splits = ap.splits;
-    p.rows_per_split = ap.rows_per_split;
     p.scale_log2 = at->sm_scale * 1.4426950408889634f;
-    if (ap.splits > 1) {
-        p.part_o = reinterpret_cast<float*>(part);
-        p.part_ml = reinterpret_cast<float*>(part + (size_t)bt->num_tokens * ap.splits * 128 * kDv * 4);
-        p.split_count = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(status) + kStatusBytes);
-        p.split_ready = p.split_count + kMaxSplitTokens * 2;
-    }
+    p.early_q = early_q ? 1 : 0;
+    p.split_count = reinterpret_cast<uint32_t*>(attn_ws);
+    p.part = attn_ws + ap.counter_bytes;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof cfg);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * bt->num_tokens * ap.splits, 1, 1);
+    // a programmatic dependent of the preceding launch (the indexer, in
+    // dsa_decode): the kernel waits for it with griddepcontrol.wait before
+    // reading the index list, and runs its prologue while it finishes
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(2 * ap.pairs, 1, 1);
     cfg.blockDim = dim3(SfaCfg::THREADS, 1, 1);
     cfg.dynamicSmemBytes = SfaCfg::SMEM;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaError_t e = cudaLaunchKernelEx(&cfg, &sfa_decode_kernel, p, tm_q))
+    cfg.numAttrs = dependent ? 2 : 1;
+    if (cudaError_t e = cudaLaunchKernelEx(&cfg, &sfa_decode_kernel, p, tm_q, tm_kv))
         return fail(DSA_ERR_CUDA, "attention launch", e);
     return DSA_OK;
 }
 
 // ------------------------------------------------------------------ allocation-free attention
-// Scratch of sparse_mla_attn_static: the status word, the split counters and
-// the split partials, in module memory (zero when the module loads).  20 MiB
-// holds every split plan on a 148-SM B200 (at most 74 token-splits of 258 KB).
+// Scratch of sparse_mla_attn_static, in module memory: the status area, the
+// split counters and the partial slots of tokens shared by several CTA pairs.
+// 20 MiB holds the largest plan of a 148-SM B200 (74 pairs x 2 sides x 2 CTAs
+// x 66 KB of slots = 19.5 MB, plus 768 bytes of counters), for any token
+// count.  Every GPU that loads the library holds it until exit.
 constexpr size_t kStaticScratchBytes = size_t(20) << 20;
 __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-// Device address of the scratch for the current device, looked up once per
-// device (the first call on a device does the lookup).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// Device address of the scratch for the current device and context.  The
+// lookup (cudaGetSymbolAddress, with the device current) is made by the first
+// call on a device and made again only if that device's context changed
+// (e.g. after cudaDeviceReset the module is loaded at a new address).
 uint8_t* static_scratch(dsa_status* st) {
     static std::mutex mu;
-    static uint8_t* addr[64] = {};
+    static uint8_t* addr[kMaxDevices] = {};
+    static CUcontext ctx_of[kMaxDevices] = {};
+    static CtxGetCurrentFn ctx_fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* fp = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fp, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            ctx_fn = reinterpret_cast<CtxGetCurrentFn>(fp);
+    });
     int dev = 0;
     if (cudaError_t e = cudaGetDevice(&dev)) {
         *st = fail(DSA_ERR_CUDA, "current device query", e);
         return nullptr;
     }
-    if (dev < 0 || dev >= 64) {
+    if (dev < 0 || dev >= kMaxDevices) {
         *st = fail(DSA_ERR_UNSUPPORTED, "device ordinal above 63");
         return nullptr;
     }
+    // the runtime makes the device's primary context current on first use
+    if (cudaError_t e = cudaFree(nullptr)) {
+        *st = fail(DSA_ERR_CUDA, "context initialisation", e);
+        return nullptr;
+    }
+    CUcontext ctx = nullptr;
+    if (ctx_fn) ctx_fn(&ctx);
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || ctx_of[dev] != ctx) {
         void* ptr = nullptr;
         if (cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch)) {
             *st = fail(DSA_ERR_CUDA, "static scratch address lookup", e);
             return nullptr;
         }
         addr[dev] = reinterpret_cast<uint8_t*>(ptr);
+        ctx_of[dev] = ctx;
     }
     return addr[dev];
 }
+
+// Attention part of a workspace: [split counters][partial slots].
+size_t attn_region_bytes(const AttnPlan& ap) { return ap.counter_bytes + align256(ap.slot_bytes); }
 
 }  // namespace
 
@@ -447,7 +326,8 @@ size_t dsa_workspace_size(const dsa_batch* batch, const dsa_indexer_inputs* ix, 
     }
     if (at) {
         if (check_attn(at) != DSA_OK) return 0;
-        need += align256(plan_attn(batch, kMaxTopK, di).part_bytes);
+        // sized for the largest Top-K, so one workspace serves any K
+        need += attn_region_bytes(plan_attn(batch, kMaxTopK, di));
     }
     return need;
 }
@@ -484,10 +364,10 @@ dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs* at, co
     if (di.max_smem < SfaCfg::SMEM) return fail(DSA_ERR_UNSUPPORTED, "device shared memory per block too small");
     const AttnPlan ap = plan_attn(batch, K, di);
     const size_t off = kHeaderBytes + idx_region_bytes(di);
-    if (workspace_bytes < off + ap.part_bytes) return DSA_ERR_WORKSPACE;
+    if (workspace_bytes < off + attn_region_bytes(ap)) return DSA_ERR_WORKSPACE;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + off, ap,
-                       reinterpret_cast<cudaStream_t>(stream));
+                       reinterpret_cast<cudaStream_t>(stream), true, false);
 }
 
 dsa_status sparse_mla_attn_static(const dsa_batch* batch, const dsa_attn_inputs* at, const int32_t* idx, int32_t K,
@@ -501,17 +381,24 @@ dsa_status sparse_mla_attn_static(const dsa_batch* batch, const dsa_attn_inputs*
     if (di.sms <= 0) return fail(DSA_ERR_CUDA, "device query failed");
     if (di.max_smem < SfaCfg::SMEM) return fail(DSA_ERR_UNSUPPORTED, "device shared memory per block too small");
     const AttnPlan ap = plan_attn(batch, K, di);
-    const size_t need = kHeaderBytes + ap.part_bytes;
+    const size_t need = kHeaderBytes + attn_region_bytes(ap);
     if (need > kStaticScratchBytes) {
-        snprintf(g_last_error, sizeof g_last_error,
+        char msg[160];
+        snprintf(msg, sizeof msg,
                  "sparse_mla_attn_static: this shape needs %zu bytes of scratch, the static scratch holds %zu", need,
                  kStaticScratchBytes);
+        set_last_error(msg);
         return DSA_ERR_WORKSPACE;
     }
     uint8_t* ws = static_scratch(&st);
     if (!ws) return st;
-    return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, ap,
-                       reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // every call starts from a clean status area and clean split counters, so a
+    // call that ended in a device error cannot leave stale state to later calls
+    if (cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes + ap.counter_bytes, s))
+        return fail(DSA_ERR_CUDA, "static scratch clear", e);
+    return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, ap, s,
+                       false, false);
 }
 
 dsa_status dsa_decode(const dsa_batch* batch, const dsa_indexer_inputs* ix, const dsa_attn_inputs* at,
@@ -522,12 +409,26 @@ dsa_status dsa_decode(const dsa_batch* batch, const dsa_indexer_inputs* ix, cons
     if ((st = check_indexer(ix)) != DSA_OK) return st;
     if ((st = check_attn(at)) != DSA_OK) return st;
     if (!out_idx || !out) return DSA_ERR_INVALID_ARG;
-    const size_t need = dsa_workspace_size(batch, ix, at);
-    if (need == 0) return DSA_ERR_UNSUPPORTED;
-    if (workspace_bytes < need) return DSA_ERR_WORKSPACE;
-    st = indexer_topk(batch, ix, out_idx, out_score, workspace, workspace_bytes, stream);
+    if (!aligned16(out)) return DSA_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+    const DevInfo di = dev_info();
+    if (di.sms <= 0) return fail(DSA_ERR_CUDA, "device query failed");
+    if (di.max_smem < SfaCfg::SMEM) return fail(DSA_ERR_UNSUPPORTED, "device shared memory per block too small");
+    // one plan for each stage, one workspace layout
+    IdxPlan pl;
+    LaunchFn fn = nullptr;
+    if ((st = plan_indexer(batch, ix, di, pl, fn)) != DSA_OK) return st;
+    if (pl.group_ws > group_region_bytes(di.sms)) return DSA_ERR_UNSUPPORTED;
+    const AttnPlan ap = plan_attn(batch, ix->K, di);
+    const size_t off = kHeaderBytes + idx_region_bytes(di);
+    if (workspace_bytes < off + attn_region_bytes(ap)) return DSA_ERR_WORKSPACE;
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = fn(batch, ix, out_idx, out_score, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, pl, s);
     if (st != DSA_OK) return st;
-    return sparse_mla_attn(batch, at, out_idx, ix->K, out, lse, workspace, workspace_bytes, stream);
+    // the attention launch depends programmatically on the indexer launch just made
+    return launch_attn(batch, at, out_idx, ix->K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + off, ap, s, true,
+                       true);
 }
 
 dsa_status dsa_get_status(void* workspace, void* stream, int32_t* device_status) {
@@ -553,9 +454,7 @@ int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexer_inputs
     LaunchFn fn = nullptr;
     if (plan_indexer(batch, ix, di, pl, fn) != DSA_OK) return -1;
     const int idx_launches = pl.mode == 1 ? 1 : (batch->batch + pl.seqs_per_launch - 1) / pl.seqs_per_launch;
-    const AttnPlan ap = plan_attn(batch, ix->K, di);
-    (void)ap;   // the split merge runs inside the attention kernel
-    return idx_launches + 1;
+    return idx_launches + 1;   // the split merge runs inside the attention kernel
 }
 
 const char* dsa_status_str(int32_t s) {
@@ -572,20 +471,10 @@ const char* dsa_status_str(int32_t s) {
     }
 }
 
-const char* dsa_last_error(void) { return g_last_error; }
+const char* dsa_last_error(void) { return last_error_text(); }
 
 const char* dsa_version(void) { return "dsa-b200 0.1.0 (sm_100a)"; }
 
-#ifdef DSA_TRACE
-// Tracing builds only: copy the per-CTA %globaltimer table ([2048][16] u64).
-DSA_API int32_t dsa_trace_read(void* host_dst, size_t bytes) {
-    if (bytes > sizeof(g_dsa_trace)) bytes = sizeof(g_dsa_trace);
-    return cudaMemcpyFromSymbol(host_dst, g_dsa_trace, bytes) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
-}
-DSA_API int32_t dsa_trace_blk_read(void* host_dst, size_t bytes) {
-    if (bytes > sizeof(g_dsa_trace_blk)) bytes = sizeof(g_dsa_trace_blk);
-    return cudaMemcpyFromSymbol(host_dst, g_dsa_trace_blk, bytes) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
-}
-#endif
+
 
 }  // extern "C"

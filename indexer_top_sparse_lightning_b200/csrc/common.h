@@ -77,13 +77,11 @@ struct SfaParams {
     const int32_t* idx;       // [T, K]
     uint16_t* out;            // [T, H, 512] bf16 bits
     float* lse;               // [T, H] or null
-    float* part_o;            // split partials: [T, S, 2 head halves, 512 columns, 64 heads] (un-normalised)
-    float* part_ml;           // [T, S, 2 head halves, 64 heads, 2] (m in log2 domain, l)
-    uint32_t* split_count;    // [T, 2 halves] arrivals; zero between calls
-    uint32_t* split_ready;    // [T, 2 halves] partials written; zero between calls
-    uint32_t* status;
+    uint8_t* part;            // partials of tokens shared by several pairs: [pairs][2 sides][2 CTAs] slots
+    uint32_t* split_count;    // [pairs, 2 CTAs] arrivals at a split token, by its first pair; zero between calls
+    uint32_t* status;         // status word; words 1-2 of the same area hold the test hooks
     int32_t B, T, H, K, max_blocks, num_blocks;
-    int32_t n_splits, rows_per_split;
+    int32_t early_q;          // Q may be loaded before the preceding launch completes
     float scale_log2;         // sm_scale * log2(e)
 };
 

@@ -94,6 +94,8 @@ struct IdxMisc {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    uint32_t inject;          // test hook: fault injection bits (workspace status area, word 2)
+    uint64_t wait_ns;         // bounded-wait limit of this launch
     // mode-0 assignment of this CTA
     int g_valid, g_b, g_rank, g_size, g_tile_begin, g_tile_count, g_group;
     SelectSmem sel;
@@ -158,7 +160,7 @@ __device__ __forceinline__ bool get_item(const IndexerParams& p, const IdxMisc* 
 
 // Mode-0 partition: every CTA computes the same split of CTAs over the
 // sequences [b_begin, b_end), proportional to their key tiles.
-__device__ void assign_groups(const IndexerParams& p, IdxMisc* m, int nq_max, int score_cap) {
+static __device__ void assign_groups(const IndexerParams& p, IdxMisc* m, int nq_max, int score_cap) {
     const int Bp = p.b_end - p.b_begin;
     const int C = gridDim.x;
     int64_t total = 0;
@@ -234,6 +236,11 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
         mbar_init(&m->q_empty, 1);
         mbar_init(&m->drain, 1);
         m->abort = 0;
+        // test hooks in the status area: word 1 = wait limit in microseconds
+        // (0: the default), word 2 = fault injection bits
+        const uint32_t us = __ldcg(p.status + 1);
+        m->wait_ns = us ? (uint64_t)us * 1000u : kWaitTimeoutNs;
+        m->inject = __ldcg(p.status + 2);
         fence_mbar_init();
         if (p.mode == 0) assign_groups(p, m, NQ, p.score_cap);
     }
@@ -255,7 +262,10 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = m->tmem_base;
-    if (threadIdx.x == 0) DSA_TRACE_MARK(0);
+    const uint64_t wlim = m->wait_ns;
+    // the attention launch that follows may be scheduled now: its CTAs take the SMs
+    // this grid leaves and run their prologue before waiting for the index list
+    griddep_launch_dependents();
 
     if (warp == Cfg::PRODUCER_WARP) {
         // ---------------------------------------------------------------- TMA producer
@@ -285,7 +295,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             __syncwarp();
             int ok = 1;
             if (lane == 0) {
-                if (!mbar_wait(&m->q_empty, (k & 1) ^ 1, abort)) ok = 0;
+                if (!mbar_wait(&m->q_empty, (k & 1) ^ 1, abort, wlim)) ok = 0;
                 if (ok) {
                     mbar_arrive_expect_tx(&m->q_full, Cfg::Q_TX);
                     for (int kb = 0; kb < Cfg::KB; ++kb)
@@ -293,7 +303,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 }
                 for (int li = 0; ok && li < item.tile_count; ++li, ++it) {
                     const int s = it % Cfg::NSTAGE;
-                    if (!mbar_wait(&m->empty[s], ((it / Cfg::NSTAGE) & 1) ^ 1, abort)) { ok = 0; break; }
+                    if (!mbar_wait(&m->empty[s], ((it / Cfg::NSTAGE) & 1) ^ 1, abort, wlim)) { ok = 0; break; }
                     int blk[2];
                     int nvalid = 0;
                     for (int pp = 0; pp < 2; ++pp) {
@@ -318,13 +328,12 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
         }
-        if (lane == 0) DSA_TRACE_MARK(8);
         // drain: no TMA write may still be in flight when the CTA exits
         if (lane == 0) {
             const uint32_t first = it > (uint32_t)Cfg::NSTAGE ? it - Cfg::NSTAGE : 0u;
             volatile int no_abort = 0;
             for (uint32_t d = first; d < it; ++d)
-                mbar_wait(&m->full[d % Cfg::NSTAGE], (d / Cfg::NSTAGE) & 1, &no_abort);
+                mbar_wait(&m->full[d % Cfg::NSTAGE], (d / Cfg::NSTAGE) & 1, &no_abort, wlim);
         }
     } else if (warp == Cfg::MMA_WARP) {
         // ---------------------------------------------------------------- MMA issuer
@@ -333,21 +342,21 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             IdxItem item;
             bool ok = true;
             for (int k = 0; ok && get_item<NQ>(p, m, k, item); ++k) {
-                if (!mbar_wait(&m->q_full, k & 1, abort)) break;
+                if (!mbar_wait(&m->q_full, k & 1, abort, wlim)) break;
                 tc_fence_after();
                 for (int li = 0; li < item.tile_count; ++li, ++it) {
                     const int buf = it & 1;
                     const uint8_t* a_base;
                     if (FP8) {
                         const int cb = it % Cfg::NCV;
-                        if (!mbar_wait(&m->conv_full[cb], (it / Cfg::NCV) & 1, abort)) { ok = false; break; }
+                        if (!mbar_wait(&m->conv_full[cb], (it / Cfg::NCV) & 1, abort, wlim)) { ok = false; break; }
                         a_base = s_conv + cb * Cfg::CONV_BYTES;
                     } else {
                         const int s = it % Cfg::NSTAGE;
-                        if (!mbar_wait(&m->full[s], (it / Cfg::NSTAGE) & 1, abort)) { ok = false; break; }
+                        if (!mbar_wait(&m->full[s], (it / Cfg::NSTAGE) & 1, abort, wlim)) { ok = false; break; }
                         a_base = s_stage + s * Cfg::STAGE_BYTES;
                     }
-                    if (!mbar_wait(&m->tempty[buf], ((it >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+                    if (!mbar_wait(&m->tempty[buf], ((it >> 1) & 1) ^ 1, abort, wlim)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(a_base);
                     const uint32_t b_addr = smem_u32(s_q);
@@ -371,7 +380,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             // drain: every issued MMA completes before TMEM is released
             umma_commit(&m->drain);
             volatile int no_abort = 0;
-            mbar_wait(&m->drain, 0, &no_abort);
+            mbar_wait(&m->drain, 0, &no_abort, wlim);
         }
     } else if (FP8 && warp >= 6) {
         // ---------------------------------------------------------------- fp8 -> bf16 widening
@@ -384,8 +393,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             for (int li = 0; li < item.tile_count; ++li, ++it) {
                 const int s = it % Cfg::NSTAGE;
                 const int cb = it % Cfg::NCV;
-                if (!mbar_wait(&m->full[s], (it / Cfg::NSTAGE) & 1, abort)) { ok = false; break; }
-                if (!mbar_wait(&m->conv_empty[cb], ((it / Cfg::NCV) & 1) ^ 1, abort)) { ok = false; break; }
+                if (!mbar_wait(&m->full[s], (it / Cfg::NSTAGE) & 1, abort, wlim)) { ok = false; break; }
+                if (!mbar_wait(&m->conv_empty[cb], ((it / Cfg::NCV) & 1) ^ 1, abort, wlim)) { ok = false; break; }
                 const uint8_t* raw = s_stage + s * Cfg::STAGE_BYTES;
                 uint8_t* dst = s_conv + cb * Cfg::CONV_BYTES;
 #pragma unroll 4
@@ -469,8 +478,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         }
                     }
                 }
-                if (!mbar_wait(&m->tfull[buf], (it >> 1) & 1, abort)) { ok = false; break; }
-                if (li == 0 && threadIdx.x == 0) DSA_TRACE_MARK(1);
+                if (!mbar_wait(&m->tfull[buf], (it >> 1) & 1, abort, wlim)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * Cfg::COLS_BUF;
                 float score[NQ];
@@ -537,7 +545,6 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 }
             }
             named_bar_sync(1, kEpiThreads);
-            if (threadIdx.x == 0) DSA_TRACE_MARK(2);
 
             // ------------------------------------------------------------ Top-K select
             int nloc[NQ];
@@ -573,11 +580,10 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             if (any_active &&
                 !topk_select<NQ>(p, gv, gen, s_score, stride, nloc, active, chunk0, item.t0, s_hist, s_list,
                                  smem + Cfg::OFF_STAGE, Cfg::SCRATCH_BYTES, &m->sel,
-                                 abort)) {
+                                 abort, wlim, m->inject)) {
                 ok = false;
                 break;
             }
-            if (threadIdx.x == 0) DSA_TRACE_MARK(7);
         }
     }
 
@@ -589,7 +595,6 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
     if (threadIdx.x == 0 && m->abort) set_status(p.status, kStTimeout);
-    if (threadIdx.x == 0) DSA_TRACE_MARK(9);
 }
 
 }  // namespace dsa

@@ -10,7 +10,8 @@
 namespace dsa {
 
 // A wait that lasts longer than this is treated as a failure: the kernel
-// records DSA_ERR_TIMEOUT and returns instead of hanging.
+// records DSA_ERR_TIMEOUT and returns instead of hanging.  The limit a
+// launch uses is read from the workspace header (0 there means this default).
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -22,29 +23,6 @@ __device__ __forceinline__ uint64_t globaltimer() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-
-// ------------------------------------------------------------------ phase tracing (debug builds only)
-// Built with -DDSA_TRACE, kernels record %globaltimer at fixed points of
-// each CTA's life into a device table read back by dsa_trace_read().
-#ifdef DSA_TRACE
-__device__ uint64_t g_dsa_trace[2048][16];
-__device__ uint64_t g_dsa_trace_blk[64][32];  // CTAs 0 and 1: per-block events
-#define DSA_TRACE_MARK(slot)                                                     \
-    do {                                                                         \
-        if (blockIdx.x < 2048) g_dsa_trace[blockIdx.x][(slot)] = globaltimer(); \
-    } while (0)
-#define DSA_TRACE_BLK(jb, ev)                                                          \
-    do {                                                                               \
-        if (blockIdx.x < 2 && (jb) < 64) g_dsa_trace_blk[(jb)][(ev) + 16 * blockIdx.x] = globaltimer(); \
-    } while (0)
-#else
-#define DSA_TRACE_MARK(slot) \
-    do {                     \
-    } while (0)
-#define DSA_TRACE_BLK(jb, ev) \
-    do {                      \
-    } while (0)
-#endif
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -114,7 +92,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t addr, uint32_t pa
 __device__ __forceinline__ void wait_backoff(uint64_t waited_ns) {
     if (waited_ns > 2000) __nanosleep(waited_ns > 20000 ? 1000u : 200u);
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
@@ -124,23 +103,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
             if (mbar_try_wait(a, parity)) return true;
         if (*abort) return false;
         const uint64_t dt = globaltimer() - t0;
-        if (dt > kWaitTimeoutNs) return false;
+        if (dt > limit_ns) return false;
         wait_backoff(dt);
     }
 }
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    const uint32_t a = smem_u32(bar);
-    if (mbar_try_wait_cluster(a, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait_cluster(a, parity)) return true;
-        if (*abort) return false;
-        const uint64_t dt = globaltimer() - t0;
-        if (dt > kWaitTimeoutNs) return false;
-        wait_backoff(dt);
-    }
+
+// ------------------------------------------------------------------ grid dependencies (programmatic launch)
+// Waits until the grids this one depends on have completed and their memory
+// operations are visible (returns at once when launched without a dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets a dependent grid be scheduled before this one has finished.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// Drops a 128-byte L2 line without writing it back (its contents become
+// undefined): for scratch that has been consumed and is not read again.
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 
 // ------------------------------------------------------------------ TMA
@@ -163,6 +141,23 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
+}
+// Row gather: four rows (y0..y3) of one box of a 2-D tensor map whose box is one
+// row high, written as four consecutive box rows at dst (the map's swizzle applies).
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y0, int y1,
+                                            int y2, int y3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
+        "r"(y2), "r"(y3)
+        : "memory");
+}
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;

@@ -60,19 +60,22 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) {
 // threads).  Sense-reversing: the last arriver resets the count and bumps
 // the generation.  `gen` is thread 0's copy of the generation, read once per
 // work item and advanced here, so a barrier costs one atomic and the wait.
-__device__ bool group_barrier(uint32_t* sync, int G, uint32_t& gen, uint32_t* status, volatile int* abort) {
+// `extra` (a test hook, normally 0) makes the barrier wait for arrivals that
+// never come, so that the bounded wait runs out.
+static __device__ bool group_barrier(uint32_t* sync, int G, uint32_t& gen, uint32_t* status, volatile int* abort,
+                              uint64_t limit_ns, uint32_t extra) {
     named_bar_sync(1, kEpiThreads);
     if (threadIdx.x == 0 && !*abort) {
         uint32_t* count = sync;
         uint32_t* genp = sync + 1;
         const uint32_t old = atom_add_acq_rel_gpu(count, 1u);
-        if (old == (uint32_t)G - 1u) {
+        if (old == (uint32_t)G - 1u + extra) {
             *reinterpret_cast<volatile uint32_t*>(count) = 0u;
             st_release_gpu(genp, gen + 1u);
         } else {
             const uint64_t t0 = globaltimer();
             while (ld_acquire_gpu(genp) == gen) {
-                if (globaltimer() - t0 > kWaitTimeoutNs) {
+                if (globaltimer() - t0 > limit_ns) {
                     set_status(status, kStTimeout);
                     *abort = 1;
                     break;
@@ -230,7 +233,7 @@ struct GlobalKeyStream {
 // Exact kk-th largest key among the n keys in `list`.  Short lists: every
 // element counts the larger and equal ones (broadcast reads, one barrier);
 // longer ones: radix select with 8-bit digits in hist[0..255].
-__device__ uint32_t list_select(const uint32_t* list, int n, uint32_t kk, uint32_t* hist, SelectSmem* sm) {
+static __device__ uint32_t list_select(const uint32_t* list, int n, uint32_t kk, uint32_t* hist, SelectSmem* sm) {
     if (n <= 2 * kEpiThreads) {
         uint32_t mine[2];
         uint32_t gt[2] = {0u, 0u}, eq[2] = {0u, 0u};
@@ -404,7 +407,7 @@ template <int NQ>
 __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_t& gen, float* s_score,
                             int stride, const int (&nloc)[NQ], const bool (&active)[NQ], int64_t chunk0,
                             int64_t t0, uint32_t* s_hist, uint32_t* s_list, uint8_t* scratch, int scratch_bytes,
-                            SelectSmem* sm, volatile int* abort) {
+                            SelectSmem* sm, volatile int* abort, uint64_t wlim, uint32_t inject) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lt_mask = (1u << lane) - 1u;
     const uint32_t K = (uint32_t)p.K;
@@ -680,9 +683,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
             }
             publish(j, edge);
         }
-        if (threadIdx.x == 0) DSA_TRACE_MARK(3);
-        if (!group_barrier(gv.sync, G, gen, p.status, abort)) return false;
-        if (threadIdx.x == 0) DSA_TRACE_MARK(4);
+        if (!group_barrier(gv.sync, G, gen, p.status, abort, wlim, inject & 1u)) return false;
     }
 
 #pragma unroll
@@ -696,19 +697,16 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         } else {
             // ---- 2. threshold over the published keys
             gather(j);
-            if (threadIdx.x == 0) DSA_TRACE_MARK(13);
             T = group_T(j);
-            if (threadIdx.x == 0) DSA_TRACE_MARK(14);
             if (sm->g_max_edge > T) {
                 // some CTA held more than it published (every CTA sees the same
                 // keys, so all take this branch): once every CTA has read the
                 // first publication, the CTAs whose edge is above T publish all
                 // their keys >= T, and the threshold of the enlarged set is exact
                 const uint32_t t1 = T;
-                if (threadIdx.x == 0) DSA_TRACE_MARK(12);
-                if (!group_barrier(gv.sync, G, gen, p.status, abort)) return false;
+                if (!group_barrier(gv.sync, G, gen, p.status, abort, wlim, inject & 1u)) return false;
                 if (sm->edge[j] > t1) publish(j, t1);
-                if (!group_barrier(gv.sync, G, gen, p.status, abort)) return false;
+                if (!group_barrier(gv.sync, G, gen, p.status, abort, wlim, inject & 1u)) return false;
                 gather(j);
                 T = group_T(j);
             }
@@ -763,7 +761,6 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
             base = gtb + min(need_eq, eqb);
             take = need_eq > eqb ? need_eq - eqb : 0u;
         }
-        if (threadIdx.x == 0) DSA_TRACE_MARK(5);
 
         // ---- per-warp counts of this CTA's elements above / equal to T, over
         // the warp's position-ordered sequence (list or quarter)
@@ -809,7 +806,6 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         }
         if (G == 1) take = K - cgt;          // this CTA holds every element
         take = min(take, ceq);
-        if (threadIdx.x == 0) DSA_TRACE_MARK(6);
         // ---- this warp's share of the tied elements, output offsets
         const uint32_t allow = take > eq_before ? min(take - eq_before, weq) : 0u;
         named_bar_sync(1, kEpiThreads);

@@ -60,3 +60,27 @@ def test_peaked_logits_rescale_path():
     idx = _oracle_idx(wl)
     o, lse = run_attention(wl, idx)
     assert_attention(wl, idx, np.arange(wl.T), o, lse)
+
+
+def test_workspace_reuse_across_token_counts():
+    # one workspace serves calls of different shapes: a call with many tokens after one
+    # with few must find its split counters at rest (not inside the other's partials)
+    import torch
+    import indexer_top_sparse_lightning_b200 as dsa
+    from tests.gpu_helpers import device_batch
+    small = W.make_workload("few", seq_lens=[9000, 3000, 5000], nq=1, H_I=8, D_I=64, H=128, K=2048, seed=25)
+    big = W.make_workload("many", seq_lens=[3000] * 40, nq=1, H_I=8, D_I=64, H=64, K=2048, seed=26)
+    ws = dsa.Workspace()
+    outs = {}
+    for wl in (small, big, small, big):
+        d = W.to_device(wl)
+        idx = torch.from_numpy(_oracle_idx(wl)).cuda()
+        o, l = dsa.sparse_mla_attn(device_batch(wl, d), d["q"], d["kv"], idx, wl.sm_scale, workspace=ws)
+        fresh = dsa.Workspace()
+        o2, l2 = dsa.sparse_mla_attn(device_batch(wl, d), d["q"], d["kv"], idx, wl.sm_scale, workspace=fresh)
+        torch.cuda.synchronize()
+        assert dsa.get_status(ws) == 0 and dsa.get_status(fresh) == 0
+        assert torch.equal(o, o2) and torch.equal(l, l2)
+        if wl.name in outs:
+            assert torch.equal(o, outs[wl.name])
+        outs[wl.name] = o
