@@ -9,9 +9,14 @@ batched decode at 32K context (64 indexer heads x 128, bf16 keys, K = 2048,
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
-Under torchrun each rank runs its own replica of the batch (weak scaling, no
-data-path collective); the step time is the maximum over ranks.  Prints one
-JSON line on rank 0.
+A step is one dsa_decode call (the attention launch overlaps the end of the
+indexer); per-kernel times come from separate launches with events between
+them.  On one GPU the line also carries the other four workloads (tiny
+decode, ragged verify with fp8 keys, million-token decode, 16K causal
+prefill) under "workloads", each with its step time, per-kernel times and
+roofline fractions.  Under torchrun each rank runs its own replica of the
+batch (weak scaling, no data-path collective); the step time is the maximum
+over ranks.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
@@ -45,6 +50,8 @@ def parse_args():
     ap.add_argument("--workload", default="batch32", choices=["batch32", "tiny", "prefill16k", "ragged", "1m"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="time only the named workload (by default one GPU also times the other four)")
     return ap.parse_args()
 
 
@@ -183,6 +190,122 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def measure(dsa, W, wl, dev, steps, warmup, graph=True):
+    """Time one workload on `dev`: the fused step (dsa_decode, the attention launch overlapping the end of
+    the indexer), each kernel alone (events between the two launches), and a CUDA-graph replay of the step.
+    Inputs smaller than twice the L2 are scrubbed from it between steps (outside the per-step events) and
+    each step is timed on its own."""
+    import torch
+    d = W.to_device(wl, dev)
+    batch = dsa.Batch(d["seq_lens"], d["cu_q"], d["block_table"], wl.num_blocks, int(wl.seq_lens.max()),
+                      int(wl.nq.max()))
+    ws = dsa.Workspace(dev)
+    out_idx = torch.empty((wl.T, wl.K), dtype=torch.int32, device=dev)
+    out = torch.empty((wl.T, wl.H, 512), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    step_bytes = wl.key_bytes() + wl.kv_bytes()
+    flush = step_bytes < 2 * L2_BYTES
+    scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
+
+    def fused():
+        dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], wl.K, wl.sm_scale,
+                       k_scale=d["k_scale"], out_idx=out_idx, out=out, workspace=ws)
+
+    def indexer():
+        dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], wl.K, k_scale=d["k_scale"], out_idx=out_idx,
+                         want_score=False, workspace=ws)
+
+    def attention():
+        dsa.sparse_mla_attn(batch, d["q"], d["kv"], out_idx, wl.sm_scale, out=out, want_lse=False, workspace=ws)
+
+    for _ in range(max(3, warmup)):
+        if flush:
+            scrub.zero_()
+        fused()
+    torch.cuda.synchronize()
+    if dsa.get_status(ws) != 0:
+        raise RuntimeError(f"{wl.name}: device reported an error during warm-up")
+    # fused steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t_start = time.time()
+    e0.record(stream)
+    for a, b in ev:
+        if flush:
+            scrub.zero_()
+        a.record(stream)
+        fused()
+        b.record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_end = time.time()
+    per_step = [a.elapsed_time(b) for a, b in ev]
+    ms_total = sum(per_step) if flush else e0.elapsed_time(e1)
+    q = statistics.quantiles(per_step, n=10) if len(per_step) > 1 else per_step * 9
+    # each kernel on its own
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for a, b, c in kev:
+        if flush:
+            scrub.zero_()
+        a.record(stream)
+        indexer()
+        b.record(stream)
+        attention()
+        c.record(stream)
+    torch.cuda.synchronize()
+    if dsa.get_status(ws) != 0:
+        raise RuntimeError(f"{wl.name}: device status after the timed region")
+    idx_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in kev)
+    sfa_ms = statistics.mean(b.elapsed_time(c) for _, b, c in kev)
+    graph_ms = None
+    if graph and not flush:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fused()
+        stream.wait_stream(side)
+        with torch.cuda.graph(g):
+            fused()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        ga = torch.cuda.Event(enable_timing=True)
+        gb = torch.cuda.Event(enable_timing=True)
+        ga.record(stream)
+        for _ in range(steps):
+            g.replay()
+        gb.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = ga.elapsed_time(gb) / steps
+        del g
+        if dsa.get_status(ws) != 0:
+            raise RuntimeError(f"{wl.name}: device reported an error in the graph replays")
+    return dict(d=d, batch=batch, ws=ws, out=out, out_idx=out_idx, flush=flush, scrub=scrub, fused=fused,
+                ms_total=ms_total, ms_step=ms_total / steps, idx_ms=idx_ms, sfa_ms=sfa_ms, graph_ms=graph_ms,
+                pct={"p10": q[0], "p50": statistics.median(per_step), "p90": q[-1]}, t_start=t_start, t_end=t_end)
+
+
+def kernel_entry(wl, r, peak):
+    """Per-kernel times and roofline fractions of one measured workload."""
+    key_bytes, kv_bytes = wl.key_bytes(), wl.kv_bytes()
+    idx_gbs = key_bytes / (r["idx_ms"] * 1e-3) / 1e9
+    sfa_gbs = kv_bytes / (r["sfa_ms"] * 1e-3) / 1e9
+    e = {"indexer_topk_kernel": {"ms_per_launch": r["idx_ms"], "gbs": idx_gbs, "frac_of_measured_hbm": idx_gbs / peak,
+                                 "algorithmic_bytes": key_bytes},
+         "sfa_decode_kernel": {"ms_per_launch": r["sfa_ms"], "gbs": sfa_gbs, "frac_of_measured_hbm": sfa_gbs / peak,
+                               "algorithmic_bytes": kv_bytes}}
+    if wl.T > 64:
+        tf_peak, _ = peaks_tensor()
+        flops = wl.indexer_flops()
+        e["indexer_topk_kernel"]["tflops"] = flops / (r["idx_ms"] * 1e-3) / 1e12
+        e["indexer_topk_kernel"]["frac_of_measured_bf16"] = flops / (r["idx_ms"] * 1e-3) / 1e12 / tf_peak
+        e["indexer_topk_kernel"]["frac_of_2250_tflops"] = flops / (r["idx_ms"] * 1e-3) / 1e15 / 2.25
+        e["indexer_topk_kernel"]["algorithmic_flops"] = flops
+    return e
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -195,112 +318,36 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     dsa.load_library()
     wl = W.preset(args.workload)
-    d = W.to_device(wl, dev)
-    batch = dsa.Batch(d["seq_lens"], d["cu_q"], d["block_table"], wl.num_blocks, int(wl.seq_lens.max()),
-                      int(wl.nq.max()))
-    ws = dsa.Workspace(dev)
     T, K = wl.T, wl.K
-    out_idx = torch.empty((T, K), dtype=torch.int32, device=dev)
-    out = torch.empty((T, wl.H, 512), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
-
     key_bytes = wl.key_bytes()
     kv_bytes = wl.kv_bytes()
     step_bytes = key_bytes + kv_bytes
-    # Inputs smaller than twice the L2 would be partly served from L2 on the next step: flush between steps
-    # (outside the per-step events) and time each step on its own.
-    flush = step_bytes < 2 * L2_BYTES
-    scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-
-    def step(i=None):
-        if i is not None:
-            ev[i][0].record(stream)
-        dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], K, k_scale=d["k_scale"], out_idx=out_idx,
-                         want_score=False, workspace=ws)
-        if i is not None:
-            ev[i][1].record(stream)
-        dsa.sparse_mla_attn(batch, d["q"], d["kv"], out_idx, wl.sm_scale, out=out, want_lse=False, workspace=ws)
-        if i is not None:
-            ev[i][2].record(stream)
 
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     t_warm = time.time()
-    for _ in range(max(3, args.warmup)):
-        if flush:
-            scrub.zero_()
-        step()
-    torch.cuda.synchronize()
-    if dsa.get_status(ws) != 0:
-        raise RuntimeError("device reported an error during warm-up")
-
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    t_start = time.time()
-    e0.record(stream)
-    for i in range(args.steps):
-        if flush:
-            scrub.zero_()
-        step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t_end = time.time()
+    r = measure(dsa, W, wl, dev, args.steps, args.warmup)
+    d, batch, ws, out, out_idx, flush, scrub = (r[k] for k in ("d", "batch", "ws", "out", "out_idx", "flush", "scrub"))
+    t_start, t_end = r["t_start"], r["t_end"]
     if world > 1:
         dist.barrier()
-    per_step = [a.elapsed_time(c) for a, _, c in ev]
-    idx_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
-    sfa_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
-    ms_total = sum(per_step) if flush else e0.elapsed_time(e1)
-    q = statistics.quantiles(per_step, n=10) if len(per_step) > 1 else per_step * 9
-    pct = {"p10": q[0], "p50": statistics.median(per_step), "p90": q[-1]}
     # keep the GPU busy long enough for the clock sampler if the timed region was short
     soak_end = t_end
     if t_end - t_start < 1.0:
         while time.time() - t_start < 1.2:
             for _ in range(20):
-                step()
+                r["fused"]()
             torch.cuda.synchronize()
         soak_end = time.time()
-    status = dsa.get_status(ws)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
-
-    # the same step captured once in a CUDA graph and replayed (launch overhead removed)
-    graph_ms = None
-    if not flush:
-        g = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            step()
-        stream.wait_stream(side)
-        with torch.cuda.graph(g):
-            step()
-        for _ in range(3):
-            g.replay()
-        torch.cuda.synchronize()
-        ga = torch.cuda.Event(enable_timing=True)
-        gb = torch.cuda.Event(enable_timing=True)
-        ga.record(stream)
-        for _ in range(args.steps):
-            g.replay()
-        gb.record(stream)
-        torch.cuda.synchronize()
-        graph_ms = ga.elapsed_time(gb) / args.steps
-        del g
-        if dsa.get_status(ws) != 0:
-            raise RuntimeError("device reported an error in the graph replays")
-
-    t = torch.tensor([ms_total, idx_ms, sfa_ms, graph_ms or 0.0], dtype=torch.float64, device=dev)
+    t = torch.tensor([r["ms_total"], r["idx_ms"], r["sfa_ms"], r["graph_ms"] or 0.0], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_total, idx_ms, sfa_ms, graph_ms = float(t[0]), float(t[1]), float(t[2]), (float(t[3]) or None)
     ms_step = ms_total / args.steps
+    pct = r["pct"]
 
     # ------------------------------------------------------------ end to end through the public API
     pin = lambda x: x.cpu().pin_memory()
@@ -340,9 +387,30 @@ def run_ours(args, rank, world, local_rank):
 
     launches = dsa.decode_launch_count(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], K, wl.sm_scale,
                                        k_scale=d["k_scale"])
+    peak, peak_kind = peaks()
+    # ------------------------------------------------------------ the other workloads (one GPU): fused step,
+    # each kernel, roofline fractions; fewer steps (each input set is generated on the host first)
+    extra = {}
+    if world == 1 and not args.no_extra_workloads:
+        del r, d, out, out_idx
+        torch.cuda.empty_cache()
+        for name in ("tiny", "ragged", "1m", "prefill16k"):
+            if name == args.workload:
+                continue
+            xw = W.preset(name)
+            nsteps = max(3, min(args.steps, 10 if name == "prefill16k" else 50))
+            xr = measure(dsa, W, xw, dev, nsteps, 3, graph=False)
+            entry = {"workload": describe(xw), "steps": nsteps, "ms_per_step": xr["ms_step"],
+                     "tokens_per_s": xw.T / (xr["ms_step"] * 1e-3), "step_ms_percentiles": xr["pct"],
+                     "bytes_per_step": xw.key_bytes() + xw.kv_bytes(),
+                     "step_gbs": (xw.key_bytes() + xw.kv_bytes()) / (xr["ms_step"] * 1e-3) / 1e9,
+                     "l2": "flushed between steps" if xr["flush"] else "inputs larger than L2",
+                     "kernels": kernel_entry(xw, xr, peak)}
+            extra[name] = entry
+            del xr, xw
+            torch.cuda.empty_cache()
     if rank != 0:
         return
-    peak, peak_kind = peaks()
     idx_gbs = key_bytes / (idx_ms * 1e-3) / 1e9
     sfa_gbs = kv_bytes / (sfa_ms * 1e-3) / 1e9
     step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
@@ -376,13 +444,7 @@ def run_ours(args, rank, world, local_rank):
                 "step_gbs": step_gbs, "frac_of_8tbs": step_gbs / SPEC_HBM_GBS,
                 "frac_of_measured": step_gbs / peak},
         "roofline": roof,
-        "kernels": {
-            "indexer_topk_kernel": {"ms_per_launch": idx_ms, "gbs": idx_gbs, "frac_of_measured_hbm": idx_gbs / peak,
-                                    "algorithmic_bytes": key_bytes},
-            "sfa_decode_kernel": {"ms_per_launch": sfa_ms, "gbs": sfa_gbs, "frac_of_measured_hbm": sfa_gbs / peak,
-                                  "algorithmic_bytes": kv_bytes,
-                                  "traffic": ncu_traffic("sfa_decode_kernel") if args.workload == "batch32" else None},
-        },
+        "kernels": kernel_entry(wl, dict(idx_ms=idx_ms, sfa_ms=sfa_ms), peak),
         "step_ms_percentiles": pct,
         "graph": {"ms_per_step": graph_ms, "value": tokens_total / (graph_ms * 1e-3) if graph_ms else None,
                   "note": "the same step captured once in a CUDA graph and replayed back to back"
@@ -392,6 +454,9 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches * args.steps,
         "clocks": dict(clocks or {}, window=window),
     }
+    line["kernels"]["sfa_decode_kernel"]["traffic"] = ncu_traffic("sfa_decode_kernel") if args.workload == "batch32" else None
+    if extra:
+        line["workloads"] = extra
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         value, dt = cpu_baseline(wl, np.arange(wl.T) if wl.T <= 64 else np.linspace(0, wl.T - 1, 32).astype(np.int64))

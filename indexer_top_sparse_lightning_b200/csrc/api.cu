@@ -147,32 +147,42 @@ dsa_status plan_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, const
 // SM pairs are used once there are at least two blocks per pair.
 struct AttnPlan {
     int pairs = 1;
+    int align_tokens = 0;       // pairs take whole tokens (no token is shared, nothing to merge)
     int64_t total_blocks = 0;
     size_t counter_bytes = 0;   // split arrival counters, [SM pairs][2], the same for every shape
     size_t slot_bytes = 0;      // partial slots, [pairs][2 sides][2 CTAs]
 };
 
+// With at least as many tokens as SM pairs, every pair takes whole tokens.  With
+// fewer, each token is split evenly over s pairs (s * T <= SM pairs, at least
+// kMinBlocks blocks per split): the contiguous block ranges then coincide with the
+// splits, every pair works on one token, and a token's s partials are merged once.
 AttnPlan plan_attn(const dsa_batch* bt, int K, const DevInfo& di) {
+    constexpr int64_t kMinBlocks = 4;
     AttnPlan ap;
     const int nb = (K + SfaCfg::ROWS - 1) / SfaCfg::ROWS;
-    ap.total_blocks = (int64_t)bt->num_tokens * nb;
-    // at least kMinBlocks blocks per pair: fewer pairs share a token when there are few
-    // blocks, which keeps the merge of their partials short
-    constexpr int64_t kMinBlocks = 8;
+    const int64_t T = bt->num_tokens;
+    ap.total_blocks = T * nb;
     const int pmax = di.sms / 2 > 0 ? di.sms / 2 : 1;
-    int64_t np = ap.total_blocks / kMinBlocks;
-    if (np > pmax) np = pmax;
-    if (np < 1) np = 1;
-    ap.pairs = (int)np;
+    if (T >= pmax) {
+        ap.pairs = pmax;
+        ap.align_tokens = 1;
+    } else {
+        int64_t sp = pmax / T;
+        const int64_t by_len = (nb + kMinBlocks - 1) / kMinBlocks;
+        if (sp > by_len) sp = by_len;
+        if (sp > nb) sp = nb;
+        if (sp < 1) sp = 1;
+        ap.pairs = (int)(T * sp);
+    }
     ap.counter_bytes = ((size_t)pmax * 2 * 4 + 255) & ~size_t(255);
-    ap.slot_bytes = (size_t)ap.pairs * 2 * 2 * (size_t)SfaCfg::SLOT_BYTES;
+    ap.slot_bytes = (size_t)pmax * 2 * 2 * (size_t)SfaCfg::SLOT_BYTES;
     return ap;
 }
 
-
 // Workspace layout, the same for every shape on a given device:
-//   [status 256 B][split arrival counters 1 KB][indexer group region, fixed
-//   size][indexer published-key slots, one per SM][attention partials]
+//   [status 256 B][indexer group region, fixed size][indexer published-key
+//   slots, one per SM][attention split counters][attention partial slots]
 // The indexer regions are sized for the largest grouped launch (one group per
 // SM, two tokens per group), so calls of any shape sharing one workspace
 // never write attention partials over the indexer's barrier words.
@@ -221,6 +231,7 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     p.num_blocks = bt->num_blocks;
     p.scale_log2 = at->sm_scale * 1.4426950408889634f;
     p.early_q = early_q ? 1 : 0;
+    p.align_tokens = ap.align_tokens;
     p.split_count = reinterpret_cast<uint32_t*>(attn_ws);
     p.part = attn_ws + ap.counter_bytes;
     cudaLaunchConfig_t cfg;

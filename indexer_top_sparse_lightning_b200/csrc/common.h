@@ -82,6 +82,7 @@ struct SfaParams {
     uint32_t* status;         // status word; words 1-2 of the same area hold the test hooks
     int32_t B, T, H, K, max_blocks, num_blocks;
     int32_t early_q;          // Q may be loaded before the preceding launch completes
+    int32_t align_tokens;     // pairs take whole tokens (ranges start at token boundaries)
     float scale_log2;         // sm_scale * log2(e)
 };
 

@@ -92,6 +92,7 @@ struct IdxMisc {
     uint64_t q_full;
     uint64_t q_empty;
     uint64_t drain;
+    uint64_t gbar;            // grouped select: all published keys of a token landed
     uint32_t tmem_base;
     int abort;
     uint32_t inject;          // test hook: fault injection bits (workspace status area, word 2)
@@ -235,6 +236,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
         mbar_init(&m->q_full, 1);
         mbar_init(&m->q_empty, 1);
         mbar_init(&m->drain, 1);
+        mbar_init(&m->gbar, 1);
+        m->sel.gphase = 0;
         m->abort = 0;
         // test hooks in the status area: word 1 = wait limit in microseconds
         // (0: the default), word 2 = fault injection bits
@@ -580,7 +583,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             if (any_active &&
                 !topk_select<NQ>(p, gv, gen, s_score, stride, nloc, active, chunk0, item.t0, s_hist, s_list,
                                  smem + Cfg::OFF_STAGE, Cfg::SCRATCH_BYTES, &m->sel,
-                                 abort, wlim, m->inject)) {
+                                 abort, wlim, m->inject, &m->gbar)) {
                 ok = false;
                 break;
             }

@@ -50,6 +50,7 @@ struct SelectSmem {
     uint32_t edge[4];            // this CTA's publication edge, per token
     uint32_t wpub[4][4];         // [token][warp] published elements
     uint32_t g_lo, g_hi, g_total, g_resident, g_max_edge;
+    uint32_t gphase;             // phase of the published-key load barrier
 };
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) {
@@ -407,7 +408,7 @@ template <int NQ>
 __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_t& gen, float* s_score,
                             int stride, const int (&nloc)[NQ], const bool (&active)[NQ], int64_t chunk0,
                             int64_t t0, uint32_t* s_hist, uint32_t* s_list, uint8_t* scratch, int scratch_bytes,
-                            SelectSmem* sm, volatile int* abort, uint64_t wlim, uint32_t inject) {
+                            SelectSmem* sm, volatile int* abort, uint64_t wlim, uint32_t inject, uint64_t* gbar) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lt_mask = (1u << lane) - 1u;
     const uint32_t K = (uint32_t)p.K;
@@ -470,7 +471,16 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         }
         if (lane == 0) sm->wpub[j][warp] = n;
     };
-    // publish token j's elements >= edge (after build): keys in warp order, header
+    // rank table and (if they fit) all published keys of token j in shared memory
+    uint32_t* rt = reinterpret_cast<uint32_t*>(gscratch);
+    uint32_t* keys = rt + ((2 * G + 3) & ~3);
+    const int keys_cap = (gscratch_bytes - ((2 * G + 3) & ~3) * 4) / 4;   // u32 keys that fit after the rank table
+
+    // publish token j's elements >= edge (after build): keys in warp order, padded with
+    // zero keys to a multiple of four (the readers' bulk loads move whole 16-byte
+    // units), then the header.  The keys are staged in shared memory and leave with
+    // one bulk store (small global stores from this CTA are slow next to a copy
+    // engine transfer); if they do not fit there, they are stored directly.
     auto publish = [&](int j, uint32_t edge) {
         build(j, edge);
         if (threadIdx.x == 0) sm->cmin = 0xFFFFFFFFu;
@@ -482,7 +492,15 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
             if (w < warp) off += sm->wpub[j][w];
             tot += sm->wpub[j][w];
         }
-        uint32_t* slot = my_slot(j) + off;
+        const uint32_t tot_pad = (tot + 3u) & ~3u;
+        const bool staged = (int)tot_pad <= keys_cap;
+        uint32_t* slot = staged ? keys + off : my_slot(j) + off;
+        if (staged) {
+            fence_proxy_async_smem();   // the scratch last held copy-engine data
+            for (uint32_t i = tot + threadIdx.x; i < tot_pad; i += kEpiThreads) keys[i] = 0u;
+        } else {
+            for (uint32_t i = tot + threadIdx.x; i < tot_pad; i += kEpiThreads) __stcg(my_slot(j) + i, 0u);
+        }
         uint32_t kmn = 0xFFFFFFFFu;
         if (lists) {
             const uint16_t* lw = s_lists + list_off[j] + warp * qlen[j];
@@ -497,7 +515,10 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
 #pragma unroll
                 for (int u = 0; u < kU; ++u) {
                     const int t = q0 + u * 32 + lane;
-                    if (t < n) __stcg(slot + t, k[u]);
+                    if (t < n) {
+                        if (staged) slot[t] = k[u];
+                        else __stcg(slot + t, k[u]);
+                    }
                     kmn = min(kmn, k[u]);
                 }
             }
@@ -511,7 +532,8 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
                 const bool in = i < end && key >= edge;
                 const uint32_t m = __ballot_sync(0xffffffffu, in);
                 if (in) {
-                    __stcg(slot + o + __popc(m & lt_mask), key);
+                    if (staged) slot[o + __popc(m & lt_mask)] = key;
+                    else __stcg(slot + o + __popc(m & lt_mask), key);
                     kmn = min(kmn, key);
                 }
                 o += __popc(m);
@@ -522,6 +544,12 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         if (lane == 0) red_min_shared(&sm->cmin, kmn);
         named_bar_sync(1, kEpiThreads);
         if (threadIdx.x == 0) {
+            if (staged && tot_pad > 0) {
+                fence_proxy_async_smem();   // the staged keys -> the copy engine
+                bulk_store(my_slot(j), keys, tot_pad * 4u);
+                bulk_store_wait();          // written before the group is told (barrier below)
+            }
+            __threadfence();
             sm->edge[j] = edge;
             uint32_t* h = gv.hdr + ((int64_t)gv.rank * NQ + j) * 4;
             __stcg(reinterpret_cast<uint4*>(h), make_uint4(tot, sm->cmin, sm->kmax[j], edge));
@@ -529,9 +557,6 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         named_bar_sync(1, kEpiThreads);
     };
 
-    // rank table and (if they fit) all published keys of token j in shared memory
-    uint32_t* rt = reinterpret_cast<uint32_t*>(gscratch);
-    uint32_t* keys = rt + ((2 * G + 3) & ~3);
     auto gather = [&](int j) {
         // headers of ranks tid and tid + 128 (G <= 256), read together; flat offsets
         // of the (4-padded) ranks by a prefix over rank order
@@ -583,59 +608,39 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         }
         named_bar_sync(1, kEpiThreads);
         if (sm->g_resident) {
-            // the first range histogram of the threshold search is built while loading
+            // every rank's (padded) keys by one bulk load each, counted on an mbarrier,
+            // then the first range histogram of the threshold search
             const uint32_t glo = sm->g_lo, ghi = sm->g_hi;
             const int shift0 = glo < ghi ? range_shift(glo, ghi) : 0;
             for (int i = threadIdx.x; i < kBins; i += kEpiThreads) s_hist[i] = 0u;
-            // the scratch last held TMA-written key tiles
-            fence_proxy_async_smem();
+            const uint32_t ph = sm->gphase;
+            if (warp == 0) {
+                // the scratch was last read by these threads and written by copy engines
+                fence_proxy_async_smem();
+                if (lane == 0) mbar_arrive_expect_tx(gbar, sm->g_total * 4u);
+                __syncwarp();
+                for (int r = lane; r < G; r += 32) {
+                    const uint32_t n4 = (rt[2 * r] + 3u) & ~3u;
+                    if (n4) bulk_load(keys + rt[2 * r + 1], gv.cand + (int64_t)r * p.cand_slot + j * slot_keys, n4 * 4u, gbar);
+                }
+            }
+            const bool landed = mbar_wait(gbar, ph, abort, wlim);
             named_bar_sync(1, kEpiThreads);
-            // 16-byte vectors of the concatenated (padded) ranks, eight loads in
-            // flight per thread; vector v belongs to the rank whose offset range holds 4v
-            const int nv = (int)(sm->g_total >> 2);
-            for (int v0 = 0; v0 < nv; v0 += kEpiThreads * 8) {
-                uint4 x[8];
-                uint32_t cnt[8], e4[8];
+            if (threadIdx.x == 0) sm->gphase = ph ^ 1u;
+            if (!landed) *abort = 1;
+            const int n = (int)sm->g_total;
+            for (int i0 = 0; i0 < n; i0 += kEpiThreads * kU) {
+                uint32_t k[kU];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int v = v0 + u * kEpiThreads + (int)threadIdx.x;
-                    x[u] = make_uint4(0, 0, 0, 0);
-                    cnt[u] = 0;
-                    e4[u] = 0;
-                    if (v < nv) {
-                        int lo = 0, hi = G - 1;
-                        while (lo < hi) {
-                            const int mid = (lo + hi + 1) >> 1;
-                            if (rt[2 * mid + 1] <= 4u * (uint32_t)v) lo = mid; else hi = mid - 1;
-                        }
-                        cnt[u] = rt[2 * lo];
-                        e4[u] = 4u * (uint32_t)v - rt[2 * lo + 1];
-                        const uint32_t* src = gv.cand + (int64_t)lo * p.cand_slot + j * slot_keys;
-                        x[u] = __ldcg(reinterpret_cast<const uint4*>(src + e4[u]));
-                    }
+                for (int u = 0; u < kU; ++u) {
+                    const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+                    k[u] = i < n ? keys[i] : 0u;
                 }
+                // padding keys 0 are below glo and not counted
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int v = v0 + u * kEpiThreads + (int)threadIdx.x;
-                    if (v < nv) {
-                        const uint32_t e = e4[u], n = cnt[u];   // keys past the count read as 0
-                        uint4 y = x[u];
-                        if (e + 1u > n) y.x = 0u;
-                        if (e + 2u > n) y.y = 0u;
-                        if (e + 3u > n) y.z = 0u;
-                        if (e + 4u > n) y.w = 0u;
-                        *reinterpret_cast<uint4*>(keys + 4 * v) = y;
-                        x[u] = y;
-                    }
-                }
-                // histogram adds by all lanes (padding keys 0 are below glo and not counted)
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int v = v0 + u * kEpiThreads + (int)threadIdx.x;
-                    const uint32_t w4[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        hist_add(s_hist, v < nv && w4[q] >= glo && w4[q] <= ghi, (w4[q] - glo) >> shift0);
+                for (int u = 0; u < kU; ++u) {
+                    const int i = i0 + u * kEpiThreads + (int)threadIdx.x;
+                    hist_add(s_hist, i < n && k[u] >= glo && k[u] <= ghi, (k[u] - glo) >> shift0);
                 }
             }
             named_bar_sync(1, kEpiThreads);

@@ -11,10 +11,11 @@
 //
 // Work split.  The selected rows of all tokens form one list of 64-row blocks
 // (token-major, ceil(K/64) blocks per token).  A cluster of two CTAs (one
-// "pair") owns a contiguous range of that list, so every pair of the grid
-// gets the same number of blocks whatever the token count; a range may start
-// or end inside a token, and the pairs that share a token merge their
-// partial (m, l, O) at the end (the last to finish does it).
+// "pair") owns a contiguous range of that list: whole tokens when there are at
+// least as many tokens as pairs, otherwise an even share of one token (the
+// launcher sizes the grid so the ranges split tokens evenly); the pairs that
+// share a token merge their partial (m, l, O) at the end (the last to finish
+// does it).
 //
 // Per block the pair runs two-CTA tensor-core MMAs (tcgen05 cta_group::2,
 // issued by CTA 0):
@@ -201,7 +202,9 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     const int pair = (int)(blockIdx.x >> 1);
     const int nb = (p.K + Cfg::ROWS - 1) / Cfg::ROWS;       // blocks per token
     const int64_t total = (int64_t)p.T * nb;
-    const int64_t g0 = pair_start(total, pair, np), g1 = pair_start(total, pair + 1, np);
+    // contiguous block ranges; with align_tokens they start at token boundaries
+    const int64_t g0 = p.align_tokens ? (int64_t)nb * ((int64_t)p.T * pair / np) : pair_start(total, pair, np);
+    const int64_t g1 = p.align_tokens ? (int64_t)nb * ((int64_t)p.T * (pair + 1) / np) : pair_start(total, pair + 1, np);
     const int nblk = (int)(g1 - g0);
     const int head0 = 64 * (int)crank;
 
