@@ -111,14 +111,14 @@ typedef struct {
  * Bytes of workspace needed for this batch shape by indexer_topk (ix given),
  * sparse_mla_attn (at given) or both / dsa_decode (both given).  The
  * layout is [256-byte status area][indexer group region and published-key
- * slots, a fixed size per device][attention split counters, a fixed size per
- * device][attention partial slots, sized for the largest Top-K]; one buffer
- * sized with both serves all three entry points, for any mix of shapes.
+ * slots, a fixed size per device][attention partial slots of tokens shared
+ * by several SM pairs, a fixed size per device]; one buffer sized with both
+ * serves all three entry points, for any mix of shapes.
  * The workspace must be 256-byte aligned and ZERO-FILLED before its first
  * use.  After that the library keeps it consistent by itself (a call that
  * completes without a device error leaves its histograms zero and its
- * barrier and split counters at rest), so it can be reused by later calls on
- * the same stream; the caller must not modify it.  After a device error
+ * barrier words at rest), so it can be reused by later calls on the same
+ * stream; the caller must not modify it.  After a device error
  * (dsa_get_status != OK) zero-fill it again.  Calls sharing one workspace
  * must not overlap in time.
  * Status area: int32 word 0 is the device status read by dsa_get_status.
@@ -153,7 +153,10 @@ DSA_API dsa_status indexer_topk(const dsa_batch* batch, const dsa_indexer_inputs
  * log-sum-exp of the scaled logits (-inf if a token selects nothing) or NULL.
  * The launch is a programmatic dependent of the preceding kernel on the
  * stream: its prologue may overlap that kernel's end, and it reads nothing
- * (inputs, index list, workspace counters) before that kernel has completed.
+ * (inputs, index list, workspace) before that kernel has completed.  When a
+ * token's rows are spread over several SM pairs (few tokens), a second, small
+ * kernel merges the pairs' partial results (normalised bf16 O and softmax
+ * statistics, kept in the workspace) into out and lse.
  */
 DSA_API dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs* at,
                            const int32_t* idx, int32_t K,
@@ -166,15 +169,15 @@ DSA_API dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs
  * device memory for the workspace -- code that must not allocate on the
  * device, or that has no device allocator at hand.  The function itself
  * allocates nothing: it uses a fixed 20 MiB scratch array inside the library
- * module (status area, split counters, partial slots), which every GPU that
- * loads the library holds until the process exits.
+ * module (status area and partial slots), which every GPU that loads the
+ * library holds until the process exits.
  * Arguments, layouts and results are those of sparse_mla_attn.
  *  - The first call on a device (and the first after that device's context
  *    changes) looks up the scratch address with the device current; make it
  *    before any latency-critical use.
- *  - Each call first clears the scratch's status area and split counters on
- *    the stream (one memset), so a call that ended in a device error leaves
- *    nothing behind for later calls.
+ *  - Each call first clears the scratch's status area on the stream (one
+ *    memset), so a call that ended in a device error leaves nothing behind
+ *    for later calls.
  *  - Shapes whose plan needs more scratch than 20 MiB are rejected with
  *    DSA_ERR_WORKSPACE (dsa_last_error() gives both sizes); on a 148-SM B200
  *    every shape fits.
@@ -212,7 +215,8 @@ DSA_API dsa_status dsa_get_status(void* workspace, void* stream, int32_t* device
 
 /*
  * Number of kernel launches dsa_decode enqueues for this shape (indexer
- * launches + attention launches), or -1 if the shape is invalid.  Useful for
+ * launches + the attention launch + the merge launch when tokens are shared
+ * by several SM pairs), or -1 if the shape is invalid.  Useful for
  * sizing CUDA graphs and for launch accounting; performs no launch.
  */
 DSA_API int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexer_inputs* ix,

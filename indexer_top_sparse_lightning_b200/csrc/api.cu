@@ -143,46 +143,43 @@ dsa_status plan_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, const
 
 // ------------------------------------------------------------------ attention planning
 // The selected rows of all tokens form T * ceil(K/64) blocks of 64 rows; each
-// two-CTA cluster ("pair") of the grid takes a contiguous range of them.  All
-// SM pairs are used once there are at least two blocks per pair.
+// two-CTA cluster ("pair") of the grid takes a contiguous range of them.
 struct AttnPlan {
     int pairs = 1;
     int align_tokens = 0;       // pairs take whole tokens (no token is shared, nothing to merge)
     int64_t total_blocks = 0;
-    size_t counter_bytes = 0;   // split arrival counters, [SM pairs][2], the same for every shape
-    size_t slot_bytes = 0;      // partial slots, [pairs][2 sides][2 CTAs]
+    bool combine = false;       // some token is shared by several pairs: the merge kernel runs
+    size_t slot_bytes = 0;      // partial slots, [SM pairs][2 sides][2 CTAs], the same for every shape
 };
 
-// With at least as many tokens as SM pairs, every pair takes whole tokens.  With
-// fewer, each token is split evenly over s pairs (s * T <= SM pairs, at least
-// kMinBlocks blocks per split): the contiguous block ranges then coincide with the
-// splits, every pair works on one token, and a token's s partials are merged once.
+// With many more tokens than SM pairs (at least kAlignTokens per pair), every
+// pair takes whole tokens: the ranges differ by at most one token, and nothing
+// is merged.  Otherwise the blocks are shared evenly by min(SM pairs, blocks)
+// pairs, so every pair streams the same number of rows, and the tokens cut by
+// a range boundary are merged by the second kernel.
 AttnPlan plan_attn(const dsa_batch* bt, int K, const DevInfo& di) {
-    constexpr int64_t kMinBlocks = 4;
+    constexpr int64_t kAlignTokens = 8;
     AttnPlan ap;
     const int nb = (K + SfaCfg::ROWS - 1) / SfaCfg::ROWS;
     const int64_t T = bt->num_tokens;
     ap.total_blocks = T * nb;
     const int pmax = di.sms / 2 > 0 ? di.sms / 2 : 1;
-    if (T >= pmax) {
+    if (T >= kAlignTokens * pmax) {
         ap.pairs = pmax;
         ap.align_tokens = 1;
     } else {
-        int64_t sp = pmax / T;
-        const int64_t by_len = (nb + kMinBlocks - 1) / kMinBlocks;
-        if (sp > by_len) sp = by_len;
-        if (sp > nb) sp = nb;
-        if (sp < 1) sp = 1;
-        ap.pairs = (int)(T * sp);
+        ap.pairs = (int)(ap.total_blocks < pmax ? ap.total_blocks : pmax);
+        // a token is shared when a range boundary falls inside it
+        for (int pr = 1; pr < ap.pairs && !ap.combine; ++pr)
+            ap.combine = (ap.total_blocks * pr / ap.pairs) % nb != 0;
     }
-    ap.counter_bytes = ((size_t)pmax * 2 * 4 + 255) & ~size_t(255);
     ap.slot_bytes = (size_t)pmax * 2 * 2 * (size_t)SfaCfg::SLOT_BYTES;
     return ap;
 }
 
 // Workspace layout, the same for every shape on a given device:
 //   [status 256 B][indexer group region, fixed size][indexer published-key
-//   slots, one per SM][attention split counters][attention partial slots]
+//   slots, one per SM][attention partial slots]
 // The indexer regions are sized for the largest grouped launch (one group per
 // SM, two tokens per group), so calls of any shape sharing one workspace
 // never write attention partials over the indexer's barrier words.
@@ -232,8 +229,7 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     p.scale_log2 = at->sm_scale * 1.4426950408889634f;
     p.early_q = early_q ? 1 : 0;
     p.align_tokens = ap.align_tokens;
-    p.split_count = reinterpret_cast<uint32_t*>(attn_ws);
-    p.part = attn_ws + ap.counter_bytes;
+    p.part = attn_ws;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof cfg);
     cudaLaunchAttribute attr[2];
@@ -254,15 +250,27 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     cfg.numAttrs = dependent ? 2 : 1;
     if (cudaError_t e = cudaLaunchKernelEx(&cfg, &sfa_decode_kernel, p, tm_q, tm_kv))
         return fail(DSA_ERR_CUDA, "attention launch", e);
+    if (!ap.combine) return DSA_OK;
+    // the merge of shared tokens: a programmatic dependent of the attention launch
+    // (scheduled early, it waits for that grid before reading the partials)
+    cudaLaunchConfig_t ccfg;
+    memset(&ccfg, 0, sizeof ccfg);
+    ccfg.gridDim = dim3((unsigned)bt->num_tokens, (unsigned)((at->H + 7) / 8), 1);
+    ccfg.blockDim = dim3(SfaCfg::COMBINE_THREADS, 1, 1);
+    ccfg.stream = stream;
+    ccfg.attrs = &attr[1];
+    ccfg.numAttrs = 1;
+    if (cudaError_t e = cudaLaunchKernelEx(&ccfg, &sfa_combine_kernel, p, ap.pairs))
+        return fail(DSA_ERR_CUDA, "attention merge launch", e);
     return DSA_OK;
 }
 
 // ------------------------------------------------------------------ allocation-free attention
-// Scratch of sparse_mla_attn_static, in module memory: the status area, the
-// split counters and the partial slots of tokens shared by several CTA pairs.
-// 20 MiB holds the largest plan of a 148-SM B200 (74 pairs x 2 sides x 2 CTAs
-// x 66 KB of slots = 19.5 MB, plus 768 bytes of counters), for any token
-// count.  Every GPU that loads the library holds it until exit.
+// Scratch of sparse_mla_attn_static, in module memory: the status area and the
+// partial slots of tokens shared by several CTA pairs.  20 MiB holds the
+// largest plan of a 148-SM B200 (74 pairs x 2 sides x 2 CTAs x 66 KB of slots
+// = 19.5 MB), for any token count.  Every GPU that loads the library holds it
+// until exit.
 constexpr size_t kStaticScratchBytes = size_t(20) << 20;
 __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
@@ -314,8 +322,8 @@ uint8_t* static_scratch(dsa_status* st) {
     return addr[dev];
 }
 
-// Attention part of a workspace: [split counters][partial slots].
-size_t attn_region_bytes(const AttnPlan& ap) { return ap.counter_bytes + align256(ap.slot_bytes); }
+// Attention part of a workspace: the partial slots.
+size_t attn_region_bytes(const AttnPlan& ap) { return align256(ap.slot_bytes); }
 
 }  // namespace
 
@@ -404,9 +412,9 @@ dsa_status sparse_mla_attn_static(const dsa_batch* batch, const dsa_attn_inputs*
     uint8_t* ws = static_scratch(&st);
     if (!ws) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // every call starts from a clean status area and clean split counters, so a
+    // every call starts from a clean status area (the test-hook words included), so a
     // call that ended in a device error cannot leave stale state to later calls
-    if (cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes + ap.counter_bytes, s))
+    if (cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, s))
         return fail(DSA_ERR_CUDA, "static scratch clear", e);
     return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, ap, s,
                        false, false);
@@ -465,7 +473,7 @@ int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexer_inputs
     LaunchFn fn = nullptr;
     if (plan_indexer(batch, ix, di, pl, fn) != DSA_OK) return -1;
     const int idx_launches = pl.mode == 1 ? 1 : (batch->batch + pl.seqs_per_launch - 1) / pl.seqs_per_launch;
-    return idx_launches + 1;   // the split merge runs inside the attention kernel
+    return idx_launches + 1 + (plan_attn(batch, ix->K, di).combine ? 1 : 0);   // attention (+ merge)
 }
 
 const char* dsa_status_str(int32_t s) {

@@ -78,7 +78,6 @@ struct SfaParams {
     uint16_t* out;            // [T, H, 512] bf16 bits
     float* lse;               // [T, H] or null
     uint8_t* part;            // partials of tokens shared by several pairs: [pairs][2 sides][2 CTAs] slots
-    uint32_t* split_count;    // [pairs, 2 CTAs] arrivals at a split token, by its first pair; zero between calls
     uint32_t* status;         // status word; words 1-2 of the same area hold the test hooks
     int32_t B, T, H, K, max_blocks, num_blocks;
     int32_t early_q;          // Q may be loaded before the preceding launch completes

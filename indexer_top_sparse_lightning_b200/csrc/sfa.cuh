@@ -11,11 +11,12 @@
 //
 // Work split.  The selected rows of all tokens form one list of 64-row blocks
 // (token-major, ceil(K/64) blocks per token).  A cluster of two CTAs (one
-// "pair") owns a contiguous range of that list: whole tokens when there are at
-// least as many tokens as pairs, otherwise an even share of one token (the
-// launcher sizes the grid so the ranges split tokens evenly); the pairs that
-// share a token merge their partial (m, l, O) at the end (the last to finish
-// does it).
+// "pair") owns a contiguous range of that list: whole tokens when there are
+// many more tokens than pairs, otherwise an even share of the list, so that
+// every SM pair streams the same number of rows.  A token whose blocks are
+// spread over several pairs gets one partial result per pair (normalised O in
+// bf16 and the softmax statistics (m, l)), and a second, light kernel
+// (sfa_combine_kernel, a programmatic dependent of this one) merges them.
 //
 // Per block the pair runs two-CTA tensor-core MMAs (tcgen05 cta_group::2,
 // issued by CTA 0):
@@ -31,12 +32,15 @@
 // operand layout, completion counted in bytes on an mbarrier).  The copies
 // bypass L1, whose share of the unified on-chip memory is small next to the
 // 227 KB of stages, so the bytes in flight are bounded by the stages alone.
+// One warp issues a row gather only every ~100 cycles per lane, so the
+// gathers of a stage are spread over six warps (the rate grows with the number
+// of issuing warps, not of lanes).
 // The logit part of a stage (own rows, all 576 columns) is refilled as soon as
 // its QK has completed, the value part (this CTA's value columns of all 64
 // rows) once its P.V has.  The online softmax keeps a lazy reference max (O
 // and l are rescaled only when the max grows by more than 2^8).
 //
-// Roles per CTA (256 threads):
+// Roles per CTA (384 threads):
 //   warps 0-3   softmax and epilogue (thread L <-> TMEM lane L: head 64c+L%64,
 //               block rows 32*(L/64).. of the logits, value columns of half
 //               L/64 of each 256-column MMA)
@@ -44,7 +48,8 @@
 //               landed" and "my Q landed" to CTA 0
 //   warp 5      row ids: selected position -> block table -> cache row, one
 //               ring slot per block; loads Q of each token with TMA
-//   warps 6, 7  TMA row gathers of the logit and value parts of each stage
+//   warps 6-8   TMA row gathers of the logit part of each stage
+//   warps 9-11  TMA row gathers of the value part of each stage
 //
 // The kernel is launched as a programmatic dependent of the launch before it:
 // every thread waits for that launch with griddepcontrol.wait after its
@@ -79,11 +84,14 @@ struct SfaCfg {
     static constexpr int OFF_MISC = OFF_XM + 128 * 4;
     static constexpr int MISC_BYTES = 768;
     static constexpr int SMEM = 1024 + OFF_MISC + MISC_BYTES;
-    static constexpr int THREADS = 256;
+    static constexpr int THREADS = 384;
     static constexpr int MMA_WARP = 4;
     static constexpr int ROW_WARP = 5;
-    static constexpr int QK_WARP = 6;                   // issues the row gathers of the logit part
-    static constexpr int V_WARP = 7;                    // issues the row gathers of the value part
+    static constexpr int QK_WARP0 = 6;                  // warps 6-8: row gathers of the logit part
+    static constexpr int V_WARP0 = 9;                   // warps 9-11: row gathers of the value part
+    static constexpr int GATHER_WARPS = 3;              // issuing warps per part
+    static constexpr int QK_OPS = (HROWS / 4) * KBQ;    // 72 four-row gathers per logit part
+    static constexpr int V_OPS = (ROWS / 4) * 4;        // 64 four-row gathers per value part
     static constexpr int S_COLS = HROWS;                // TMEM columns of one logit buffer
     static constexpr int TMEM_COLS = 512;               // O: [0, 256), logit buffers from column 256
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, ROWS, false, false);
@@ -93,13 +101,17 @@ struct SfaCfg {
     static constexpr int64_t SLOT_O = 64 * 512 * 2;
     static constexpr int64_t SLOT_BYTES = SLOT_O + 64 * 8;
     static constexpr int MAX_SPLITS = (kMaxTopK + ROWS - 1) / ROWS;   // a token meets at most this many pairs
+    static constexpr int COMBINE_THREADS = 256;         // merge kernel: one warp per (token, head)
 };
 
 static_assert(SfaCfg::SMEM <= 232448, "attention shared memory exceeds the per-CTA limit");
 static_assert(SfaCfg::OFF_QK % 1024 == 0 && SfaCfg::OFF_V % 1024 == 0 && SfaCfg::QK_STAGE % 1024 == 0 &&
                   SfaCfg::V_STAGE % 1024 == 0 && SfaCfg::OFF_P % 1024 == 0,
               "128-byte swizzled operands need 1024-byte alignment");
-static_assert(SfaCfg::MAX_SPLITS * 8 + SfaCfg::MAX_SPLITS * 64 * 4 + 64 * 4 <= SfaCfg::NSB * SfaCfg::P_BYTES, "merge tables fit the P buffers");
+static_assert(SfaCfg::MAX_SPLITS <= 32, "the merge kernel keeps one split per lane");
+static_assert(SfaCfg::QK_OPS <= 32 * SfaCfg::GATHER_WARPS && SfaCfg::V_OPS <= 32 * SfaCfg::GATHER_WARPS &&
+                  SfaCfg::V_OPS >= SfaCfg::GATHER_WARPS,
+              "one gather instruction per issuing warp and stage");
 
 struct SfaMisc {
     uint64_t q_full;            // own Q landed
@@ -120,11 +132,8 @@ struct SfaMisc {
     uint64_t drain;
     uint64_t rows_full[SfaCfg::NRB];
     uint64_t rows_empty[SfaCfg::NRB];
-    uint64_t merge_full[2];     // a partial slot landed in a stage buffer (split merges)
     uint32_t tmem_base;
     int abort;
-    int last;
-    int pending[2];             // tokens this CTA merges at the end of its range (-1: none)
     uint32_t inject;
     uint64_t wait_ns;
 };
@@ -213,10 +222,10 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         mbar_init(&m->q_peer, 1);
         mbar_init(&m->q_empty, 1);
         for (int i = 0; i < Cfg::NS; ++i) {
-            mbar_init(&m->qk_full[i], 1);
+            mbar_init(&m->qk_full[i], Cfg::GATHER_WARPS);   // one byte-counted arrival per issuing warp
             mbar_init(&m->qk_peer[i], 1);
             mbar_init(&m->qk_empty[i], 1);
-            mbar_init(&m->v_full[i], 1);
+            mbar_init(&m->v_full[i], Cfg::GATHER_WARPS);
             mbar_init(&m->v_peer[i], 1);
             mbar_init(&m->v_empty[i], 1);
         }
@@ -231,13 +240,9 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         mbar_init(&m->drain, 1);
         for (int i = 0; i < Cfg::NRB; ++i) {
             mbar_init(&m->rows_full[i], 1);
-            mbar_init(&m->rows_empty[i], 4 + 2);   // softmax warps and the two gather warps
+            mbar_init(&m->rows_empty[i], 4 + 2 * Cfg::GATHER_WARPS);   // softmax and gather warps
         }
-        mbar_init(&m->merge_full[0], 1);
-        mbar_init(&m->merge_full[1], 1);
         m->abort = 0;
-        m->last = 0;
-        m->pending[0] = m->pending[1] = -1;
         // test hooks in the status area: word 1 = wait limit in microseconds
         // (0: the default), word 2 = fault injection bits
         const uint32_t us = __ldcg(p.status + 1);
@@ -268,6 +273,9 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
     const uint64_t wlim = m->wait_ns;
     const uint32_t inject = m->inject;
 
+    // the merge kernel (a programmatic dependent) may be scheduled on SMs this grid
+    // leaves idle; it waits for the whole grid before reading the partials
+    griddep_launch_dependents();
     // Q of the first token does not depend on the index list: when the preceding
     // launch is known not to write it, it is loaded before waiting
     if (!p.early_q) griddep_wait();
@@ -489,19 +497,41 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             volatile int no_abort = 0;
             mbar_wait(&m->q_full, sfa_block(g0, g1, nb, nblk - 1).seg & 1, &no_abort, wlim);
         }
-    } else if (warp == Cfg::QK_WARP || warp == Cfg::V_WARP) {
+    } else if (warp >= Cfg::QK_WARP0 && warp < Cfg::V_WARP0 + Cfg::GATHER_WARPS) {
         // ---------------------------------------------------------------- TMA row gathers
-        // warp 6: the logit part of each stage -- own rows 32c..32c+31, all nine 64-column
-        // chunks (lane kb issues the eight four-row gathers of chunk kb); warp 7: the
-        // value part -- this CTA's four value chunks of all 64 rows (lane i issues the
-        // four gathers of rows 4i..4i+3).  Skipped selections (row -1) fetch row 0;
-        // their logits are masked.
-        const bool vpart = warp == Cfg::V_WARP;
+        // Logit part (warps 6-8): own rows 32c..32c+31, all nine 64-column chunks, as 72
+        // four-row gathers; value part (warps 9-11): this CTA's four value chunks of all 64
+        // rows, 64 gathers.  Gather o of a part goes to lane o / 3 of issuing warp o % 3, so
+        // each warp issues one instruction per stage (21 to 24 active lanes) and counts its
+        // own bytes on the stage barrier.  Skipped selections (row -1) fetch row 0; their
+        // logits are masked.
+        const bool vpart = warp >= Cfg::V_WARP0;
+        const int gw = warp - (vpart ? Cfg::V_WARP0 : Cfg::QK_WARP0);
         const int c = (int)crank;
+        const int nops = vpart ? Cfg::V_OPS : Cfg::QK_OPS;
+        const int o = lane * Cfg::GATHER_WARPS + gw;           // this lane's gather of the stage
+        const int my_ops = (nops - gw + Cfg::GATHER_WARPS - 1) / Cfg::GATHER_WARPS;   // <= 32
         uint64_t* full = vpart ? m->v_full : m->qk_full;
         uint64_t* empty = vpart ? m->v_empty : m->qk_empty;
         uint8_t* stage0 = vpart ? s_v : s_qk;
         const int stage_bytes = vpart ? Cfg::V_STAGE : Cfg::QK_STAGE;
+        // destination and source of gather o: logit part -- row group o / 9, chunk o % 9;
+        // value part -- row group o / 4, value chunk slot o % 4
+        int dst_off = 0, x = 0, g4 = 0;
+        if (o < nops) {
+            if (!vpart) {
+                g4 = o / Cfg::KBQ;
+                const int kb = o % Cfg::KBQ;
+                dst_off = kb * Cfg::KOWN_KB + g4 * 512;
+                x = kb * 64;
+                g4 = 32 * c + 4 * g4;                          // first block row of the group
+            } else {
+                const int i = o >> 2, vch = o & 3;
+                dst_off = vch * Cfg::VALL_KB + i * 512;
+                x = (4 * (vch >> 1) + 2 * c + (vch & 1)) * 64;   // value chunk of the row
+                g4 = 4 * i;
+            }
+        }
         bool ok = true;
         int issued = 0;
         for (int jj = 0; ok && jj < nblk; ++jj) {
@@ -511,31 +541,12 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                 ok = false;
                 break;
             }
-            if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(my_ops * 512));
             __syncwarp();
-            uint8_t* st = stage0 + s * stage_bytes;
-            const int32_t* rows = s_rows + r * Cfg::ROWS;
-            if (!vpart) {
-                if (lane < Cfg::KBQ) {
-                    const int kb = lane;
-#pragma unroll
-                    for (int i = 0; i < Cfg::HROWS / 4; ++i) {
-                        const int4 rr = *reinterpret_cast<const int4*>(rows + 32 * c + 4 * i);
-                        tma_gather4(st + kb * Cfg::KOWN_KB + i * 512, &tm_kv, &full[s], kb * 64, rr.x < 0 ? 0 : rr.x,
-                                    rr.y < 0 ? 0 : rr.y, rr.z < 0 ? 0 : rr.z, rr.w < 0 ? 0 : rr.w);
-                    }
-                }
-            } else {
-                if (lane < Cfg::ROWS / 4) {
-                    const int i = lane;
-                    const int4 rr = *reinterpret_cast<const int4*>(rows + 4 * i);
-#pragma unroll
-                    for (int vch = 0; vch < 4; ++vch) {
-                        const int vc = 4 * (vch >> 1) + 2 * c + (vch & 1);          // value chunk of the row
-                        tma_gather4(st + vch * Cfg::VALL_KB + i * 512, &tm_kv, &full[s], vc * 64, rr.x < 0 ? 0 : rr.x,
-                                    rr.y < 0 ? 0 : rr.y, rr.z < 0 ? 0 : rr.z, rr.w < 0 ? 0 : rr.w);
-                    }
-                }
+            if (o < nops) {
+                const int4 rr = *reinterpret_cast<const int4*>(s_rows + r * Cfg::ROWS + g4);
+                tma_gather4(stage0 + s * stage_bytes + dst_off, &tm_kv, &full[s], x, rr.x < 0 ? 0 : rr.x,
+                            rr.y < 0 ? 0 : rr.y, rr.z < 0 ? 0 : rr.z, rr.w < 0 ? 0 : rr.w);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&m->rows_empty[r]);
@@ -704,12 +715,9 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                 if (half == 0 && head < p.H && p.lse)
                     p.lse[(int64_t)t * p.H + head] = empty ? -INFINITY : (mrun + log2f(ltot)) * 0.69314718055994531f;
             } else {
-                // The token is shared with other pairs: every pair writes its normalised
-                // partial (bf16) and (m, l), then counts itself in; the one that arrives
-                // last merges (no pair waits for another), at the end of its range with
-                // all its threads, so the next token's blocks are not held up.
+                // The token is shared with other pairs: this pair writes its normalised
+                // partial O (bf16) and (m, l) to its slot; the merge kernel combines them.
                 const int pf = pair_of_block(total, (int64_t)t * nb, np);
-                const int S = pair_of_block(total, (int64_t)(t + 1) * nb - 1, np) - pf + 1;
                 uint8_t* sl = slot(t, pf, pair - pf);
                 uint16_t* od = reinterpret_cast<uint16_t*>(sl) + hl * 512;
                 for (int c0 = 0; c0 < 256; c0 += 32) {
@@ -726,18 +734,6 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
                 }
                 if (half == 0)
                     __stcg(reinterpret_cast<float2*>(sl + Cfg::SLOT_O) + hl, make_float2(mrun, empty ? 0.0f : ltot));
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (L == 0) {
-                    // a token shared by several pairs is the only split token whose first
-                    // pair is pf, so the counter is keyed by pf
-                    uint32_t* arrive = p.split_count + (int64_t)pf * 2 + crank;
-                    const bool last = atom_add_acq_rel_gpu(arrive, 1u) == (uint32_t)S - 1u;
-                    if (last) *arrive = 0u;   // at rest for the next call
-                    m->last = last;
-                }
-                named_bar_sync(1, 128);
-                if (m->last && L == 0) m->pending[m->pending[0] >= 0 ? 1 : 0] = t;
             }
             // O has been read: the next token's first P.V may overwrite it
             tc_fence_before();
@@ -745,118 +741,6 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
             if (L % 32 == 0) arrive_leader(&m->o_empty, crank);
         }
         if (!ok) *abort = 1;
-    }
-
-    // ---------------------------------------------------------------- split merges
-    // Merges of the tokens this CTA arrived at last, by all 256 threads: thread i takes
-    // head i/4 and value columns 128*(i%4).. of this CTA's 64 heads.  Each split's
-    // partial (64 KB of bf16) is brought into the idle stages by a 1-D bulk copy, two
-    // splits in flight; weights 2^(m_s - M) * l_s go to the P buffers (idle: every P.V
-    // has completed); splits are folded in index order, so the result has the same
-    // bits whichever pair merges; the consumed slots' L2 lines are dropped without
-    // being written back.
-    __syncthreads();
-    {
-        uint32_t mphase[2] = {0u, 0u};
-        for (int pi = 0; pi < 2; ++pi) {
-            const int t = m->pending[pi];
-            if (t < 0 || m->abort) break;
-            const int pf = pair_of_block(total, (int64_t)t * nb, np);
-            const int S = pair_of_block(total, (int64_t)(t + 1) * nb - 1, np) - pf + 1;
-            const uint8_t** sptr = reinterpret_cast<const uint8_t**>(s_p);                   // [MAX_SPLITS]
-            float* wts = reinterpret_cast<float*>(s_p + Cfg::MAX_SPLITS * 8);               // [S][64 heads]
-            float* red = wts + Cfg::MAX_SPLITS * 64;                                         // [64 heads]: 1 / sum
-            uint8_t* buf[2] = {s_qk, s_v};
-            if (threadIdx.x < S) {
-                const int s_idx = threadIdx.x;
-                const int side = (s_idx == 0 && pair_start(total, pf, np) < (int64_t)t * nb) ? 1 : 0;
-                sptr[s_idx] = p.part + ((int64_t)(2 * (pf + s_idx) + side) * 2 + crank) * Cfg::SLOT_BYTES;
-            }
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                fence_proxy_async_smem();   // the stages were last read by the MMAs and written by TMA
-                for (int s2 = 0; s2 < 2 && s2 < S; ++s2) {
-                    mbar_arrive_expect_tx(&m->merge_full[s2], (uint32_t)Cfg::SLOT_O);
-                    bulk_load(buf[s2], sptr[s2], (uint32_t)Cfg::SLOT_O, &m->merge_full[s2]);
-                }
-            }
-            const int hl = threadIdx.x >> 2, part = threadIdx.x & 3, rot = lane & 15;
-            const int head = head0 + hl;
-            if (part == 0) {
-                // (m, l) of every split, all loads in flight together
-                float2 ml[Cfg::MAX_SPLITS];
-#pragma unroll
-                for (int s2 = 0; s2 < Cfg::MAX_SPLITS; ++s2)
-                    ml[s2] = s2 < S ? __ldcg(reinterpret_cast<const float2*>(sptr[s2] + Cfg::SLOT_O) + hl)
-                                    : make_float2(-INFINITY, 0.0f);
-                float M = -INFINITY;
-#pragma unroll
-                for (int s2 = 0; s2 < Cfg::MAX_SPLITS; ++s2) M = fmaxf(M, ml[s2].x);
-                float Lsum = 0.0f;
-#pragma unroll
-                for (int s2 = 0; s2 < Cfg::MAX_SPLITS; ++s2) {
-                    const float2 v = ml[s2];
-                    const float w = (M == -INFINITY || v.x == -INFINITY || !(v.y > 0.0f)) ? 0.0f : exp2f(v.x - M) * v.y;
-                    if (s2 < S) wts[s2 * 64 + hl] = w;
-                    Lsum += w;
-                }
-                red[hl] = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
-                if (head < p.H && p.lse)
-                    p.lse[(int64_t)t * p.H + head] = Lsum > 0.0f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
-            }
-            __syncthreads();
-            const float inv = red[hl];
-            float acc[128];
-#pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-            bool ok = true;
-            for (int s2 = 0; s2 < S; ++s2) {
-                const int bi = s2 & 1;
-                ok = ok && mbar_wait(&m->merge_full[bi], mphase[bi], abort, wlim);
-                mphase[bi] ^= 1u;
-                const float w = wts[s2 * 64 + hl];
-                // head hl's row of the split (1 KB), this thread's 128 columns as sixteen
-                // 16-byte chunks, visited from chunk rot on (the lanes of a quarter-warp
-                // then read distinct bank groups); acc[8*v0..] holds chunk (v0+rot)%16
-                const uint4* row = reinterpret_cast<const uint4*>(buf[bi] + hl * 1024 + part * 256);
-                if (ok && w != 0.0f) {
-#pragma unroll
-                    for (int v0 = 0; v0 < 16; ++v0) {
-                        const uint4 x = row[(v0 + rot) & 15];
-                        const uint32_t xs4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            acc[8 * v0 + 2 * e] = fmaf(w, __uint_as_float(xs4[e] << 16), acc[8 * v0 + 2 * e]);
-                            acc[8 * v0 + 2 * e + 1] = fmaf(w, __uint_as_float(xs4[e] & 0xFFFF0000u), acc[8 * v0 + 2 * e + 1]);
-                        }
-                    }
-                }
-                __syncthreads();   // every thread is done with buffer bi
-                if (threadIdx.x == 0 && s2 + 2 < S && ok) {
-                    fence_proxy_async_smem();
-                    mbar_arrive_expect_tx(&m->merge_full[bi], (uint32_t)Cfg::SLOT_O);
-                    bulk_load(buf[bi], sptr[s2 + 2], (uint32_t)Cfg::SLOT_O, &m->merge_full[bi]);
-                }
-            }
-            if (ok && head < p.H) {
-                uint16_t* dstp = p.out + ((int64_t)t * p.H + head) * kDv + part * 128;
-#pragma unroll
-                for (int v0 = 0; v0 < 16; ++v0) {
-                    const float* a = acc + 8 * v0;
-                    *reinterpret_cast<uint4*>(dstp + 8 * ((v0 + rot) & 15)) =
-                        make_uint4(pack_bf16(a[0] * inv, a[1] * inv), pack_bf16(a[2] * inv, a[3] * inv),
-                                   pack_bf16(a[4] * inv, a[5] * inv), pack_bf16(a[6] * inv, a[7] * inv));
-                }
-            }
-            if (!ok) *abort = 1;
-            __syncthreads();
-            for (int s2 = 0; s2 < S; ++s2) {
-                const uint8_t* sl = sptr[s2];
-                for (int64_t off = (int64_t)threadIdx.x * 128; off <= Cfg::SLOT_BYTES - 128; off += 128 * Cfg::THREADS)
-                    discard_l2_line(sl + off);
-            }
-            __syncthreads();
-        }
     }
 
     // ---------------------------------------------------------------- teardown
@@ -868,6 +752,74 @@ __global__ void __launch_bounds__(SfaCfg::THREADS, 1)
         tmem_dealloc_2cta(tmem_base, Cfg::TMEM_COLS);
     }
     if (threadIdx.x == 0 && m->abort) atomicCAS(p.status, 0u, (uint32_t)kStTimeout);
+}
+
+// Merge of the tokens whose blocks were spread over several pairs (the launcher
+// starts it only when some token is).  One warp per (token, head): lane s reads
+// the statistics (m_s, l_s) of split s (log2 units: m is the running maximum of
+// the scaled logits, l the sum of 2^(logit - m) over the split's rows), the
+// weights are 2^(m_s - M) * l_s with M the largest m_s, and each lane merges 16
+// value columns of the splits' normalised outputs in split order:
+//   O = sum_s w_s O_s / sum_s w_s,   lse = (M + log2(sum_s w_s)) * ln 2.
+// A split that selected nothing has l_s = 0 and weight 0; a token with no row
+// at all gets O = 0 and lse = -inf, as in the attention kernel.  The L2 lines
+// of a consumed partial row are dropped without being written back.
+__global__ void __launch_bounds__(SfaCfg::COMBINE_THREADS)
+    sfa_combine_kernel(const __grid_constant__ SfaParams p, int np) {
+    using Cfg = SfaCfg;
+    // the partials are written by the attention launch this one depends on
+    griddep_wait();
+    const int t = (int)blockIdx.x;
+    const int head = (int)blockIdx.y * (Cfg::COMBINE_THREADS / 32) + (int)(threadIdx.x >> 5);
+    const int lane = (int)(threadIdx.x & 31);
+    const int nb = (p.K + Cfg::ROWS - 1) / Cfg::ROWS;
+    const int64_t total = (int64_t)p.T * nb;
+    const int pf = pair_of_block(total, (int64_t)t * nb, np);
+    const int pl = pair_of_block(total, (int64_t)(t + 1) * nb - 1, np);
+    if (pf == pl || head >= p.H) return;     // a whole token is finished by its pair
+    const int S = pl - pf + 1;
+    const int crank = head >> 6, hl = head & 63;
+    // slot of split si: its pair's first segment (side 0) unless that pair started in
+    // an earlier token (then token t is its last segment, side 1)
+    auto slot = [&](int si) -> const uint8_t* {
+        const int side = (si == 0 && pair_start(total, pf, np) < (int64_t)t * nb) ? 1 : 0;
+        return p.part + ((int64_t)(2 * (pf + si) + side) * 2 + crank) * Cfg::SLOT_BYTES;
+    };
+    float2 ml = make_float2(-INFINITY, 0.0f);
+    if (lane < S) ml = __ldcg(reinterpret_cast<const float2*>(slot(lane) + Cfg::SLOT_O) + hl);
+    float M = ml.x;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+    const float w = (M == -INFINITY || ml.x == -INFINITY || !(ml.y > 0.0f)) ? 0.0f : exp2f(ml.x - M) * ml.y;
+    float Lsum = w;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, d);
+    float acc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+#pragma unroll 4
+    for (int si = 0; si < S; ++si) {
+        const float ws = __shfl_sync(0xffffffffu, w, si);
+        const uint4* row = reinterpret_cast<const uint4*>(slot(si) + (int64_t)hl * 1024) + 2 * lane;
+        const uint4 x0 = __ldcs(row), x1 = __ldcs(row + 1);
+        const uint32_t xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            acc[2 * e] = fmaf(ws, __uint_as_float(xs[e] << 16), acc[2 * e]);
+            acc[2 * e + 1] = fmaf(ws, __uint_as_float(xs[e] & 0xFFFF0000u), acc[2 * e + 1]);
+        }
+    }
+    const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+    uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)t * p.H + head) * kDv) + 2 * lane;
+    dst[0] = make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
+                        pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
+    dst[1] = make_uint4(pack_bf16(acc[8] * inv, acc[9] * inv), pack_bf16(acc[10] * inv, acc[11] * inv),
+                        pack_bf16(acc[12] * inv, acc[13] * inv), pack_bf16(acc[14] * inv, acc[15] * inv));
+    if (lane == 0 && p.lse)
+        p.lse[(int64_t)t * p.H + head] = Lsum > 0.0f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+    // every lane's loads have returned (their values are in the output): drop the rows
+    __syncwarp();
+    for (int li = lane; li < S * 8; li += 32) discard_l2_line(slot(li >> 3) + (int64_t)hl * 1024 + (li & 7) * 128);
 }
 
 }  // namespace dsa

@@ -61,8 +61,8 @@ def test_group_barrier_timeout_is_reported_and_recoverable():
 
 
 def test_attention_pipeline_timeout_is_reported_and_recoverable():
-    # two tokens of 2048 selected rows: each token is shared by several CTA pairs, the
-    # last of which merges the others' partials
+    # two tokens of 2048 selected rows: each token is shared by several CTA pairs whose
+    # partials the merge kernel combines
     wl = W.make_workload("fail_attn", seq_lens=[9000, 12000], nq=1, H_I=8, D_I=64, H=128, K=2048, seed=52)
     d = W.to_device(wl)
     b = device_batch(wl, d)
@@ -86,7 +86,7 @@ def test_attention_pipeline_timeout_is_reported_and_recoverable():
     torch.cuda.synchronize()
     assert dsa.get_status(ws) == 0
     assert torch.equal(out1, out0) and torch.equal(lse1, lse0)
-    # the allocation-free entry point clears its own counters on every call: it is
+    # the allocation-free entry point clears its own status area on every call: it is
     # unaffected by what happened in a workspace, and equal to the workspace path
     out2, lse2 = dsa.sparse_mla_attn_static(b, d["q"], d["kv"], idx, wl.sm_scale)
     torch.cuda.synchronize()

@@ -29,11 +29,22 @@ def test_sixteen_heads_tiny_preset():
     assert_attention(wl, idx, np.arange(wl.T), o, lse)
 
 
-def test_single_split_many_tokens():
-    # enough tokens that every (token) pair of CTAs takes all its rows: no partials
+def test_even_split_many_tokens():
+    # a few more tokens than SM pairs: the blocks are shared evenly, most pairs cut a
+    # token at each end of their range (partials on both sides of a pair)
     rng = np.random.default_rng(3)
     lens = rng.integers(50, 900, size=80)
     wl = W.make_workload("many", seq_lens=lens, nq=1, H_I=8, D_I=64, H=128, K=256, seed=22)
+    idx = _oracle_idx(wl)
+    o, lse = run_attention(wl, idx)
+    assert_attention(wl, idx, np.arange(wl.T), o, lse)
+
+
+def test_whole_tokens_per_pair():
+    # many more tokens than SM pairs: every pair takes whole tokens, nothing is merged
+    rng = np.random.default_rng(5)
+    lens = rng.integers(20, 300, size=700)
+    wl = W.make_workload("whole", seq_lens=lens, nq=1, H_I=8, D_I=64, H=16, K=100, seed=27)
     idx = _oracle_idx(wl)
     o, lse = run_attention(wl, idx)
     assert_attention(wl, idx, np.arange(wl.T), o, lse)
@@ -63,8 +74,8 @@ def test_peaked_logits_rescale_path():
 
 
 def test_workspace_reuse_across_token_counts():
-    # one workspace serves calls of different shapes: a call with many tokens after one
-    # with few must find its split counters at rest (not inside the other's partials)
+    # one workspace serves calls of different shapes: the partial slots of a call with
+    # few tokens and those of a call with more tokens share the region without harm
     import torch
     import indexer_top_sparse_lightning_b200 as dsa
     from tests.gpu_helpers import device_batch
