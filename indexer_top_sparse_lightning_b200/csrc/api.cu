@@ -75,21 +75,23 @@ bool plan_for(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl) {
     // one CTA per SM (shared memory use allows no more); a group's select reads
     // at most 256 publication headers
     pl.grid = di.sms < 256 ? di.sms : 256;
+    // a work item's page ids are staged in shared memory (MAX_PAGES of them)
+    constexpr int64_t kMaxItemKeys = (int64_t)Cfg::MAX_PAGES * kPage;
     if (pl.mode == 1) {
-        if (bt->max_seq_len > pl.score_cap) return false;
-        pl.seqs_per_launch = bt->batch;
+        if (bt->max_seq_len > pl.score_cap || bt->max_seq_len > kMaxItemKeys) return false;
         pl.group_ws = 0;
         return true;
     }
-    const int64_t mt = (bt->max_seq_len + kTileKeys - 1) / kTileKeys;   // tiles of the longest sequence
-    const int64_t cap_tiles = pl.score_cap / (kTileKeys * NQ);
-    // B' sequences per launch so that ceil(total/(C-B')) <= cap_tiles even if all are longest
+    const int64_t mt = (bt->max_seq_len + kTileKeys - 1) / kTileKeys;   // tiles of the longest window
+    int64_t cap_tiles = pl.score_cap / (kTileKeys * NQ);
+    if (cap_tiles > kMaxItemKeys / kTileKeys) cap_tiles = kMaxItemKeys / kTileKeys;
+    // W' windows per launch so that ceil(total/(C-W')) <= cap_tiles even if all are longest
     int64_t bp = ((int64_t)pl.grid * cap_tiles) / (mt + cap_tiles);
     if (bp > pl.grid) bp = pl.grid;
-    if (bp > bt->batch) bp = bt->batch;
+    if (bp > pl.windows) bp = pl.windows;
     while (bp >= 1 && (bp * mt + (pl.grid - bp) - 1) / (pl.grid - bp > 0 ? pl.grid - bp : 1) > cap_tiles) --bp;
     if (bp < 1) return false;
-    pl.seqs_per_launch = (int)bp;
+    pl.windows_per_launch = (int)bp;
     // one stride for every NQ: the barrier words of group g sit at the same
     // offset whichever kernel used the workspace last (they are not zero
     // between calls; everything else is)
@@ -126,19 +128,36 @@ bool select_hi(int H_I, int D_I, const dsa_batch* bt, const DevInfo& di, IdxPlan
     }
 }
 
+// Up to two query tokens per sequence (decode, speculative verify): grouped mode,
+// one window per sequence.  More (chunked prefill, longer verify): one CTA per
+// token when a token's whole score row fits one CTA's shared memory; otherwise
+// grouped mode over windows of two tokens, each window split over enough CTAs.
 dsa_status plan_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, const DevInfo& di, IdxPlan& pl,
                         LaunchFn& fn) {
-    int nq = bt->max_q_per_seq < bt->num_tokens ? bt->max_q_per_seq : bt->num_tokens;
+    const int nq = bt->max_q_per_seq < bt->num_tokens ? bt->max_q_per_seq : bt->num_tokens;
+    const bool fp8 = ix->key_dtype == DSA_KEY_FP8_E4M3;
+    auto select = [&]() {
+        return fp8 ? select_hi<true>(ix->H_I, ix->D_I, bt, di, pl, fn) : select_hi<false>(ix->H_I, ix->D_I, bt, di, pl, fn);
+    };
     if (nq <= 2) {
         pl.mode = 0;
         pl.nq = nq;
-    } else {
-        pl.mode = 1;   // many tokens per sequence (chunked prefill): one CTA per token
-        pl.nq = 1;
+        pl.seq_windows = 1;
+        pl.windows = bt->batch;
+        return select() ? DSA_OK : DSA_ERR_UNSUPPORTED;
     }
-    const bool fp8 = ix->key_dtype == DSA_KEY_FP8_E4M3;
-    bool ok = fp8 ? select_hi<true>(ix->H_I, ix->D_I, bt, di, pl, fn) : select_hi<false>(ix->H_I, ix->D_I, bt, di, pl, fn);
-    return ok ? DSA_OK : DSA_ERR_UNSUPPORTED;
+    pl.mode = 1;
+    pl.nq = 1;
+    if (select()) return DSA_OK;
+    // sum_b ceil(nq_b / 2) <= min(B * ceil(max_q / 2), T / 2 + B): launches past the
+    // last window find no work
+    pl.mode = 0;
+    pl.nq = 2;
+    pl.seq_windows = 0;
+    const int64_t by_max = (int64_t)bt->batch * ((nq + 1) / 2);
+    const int64_t by_total = (int64_t)(bt->num_tokens + 1) / 2 + bt->batch;
+    pl.windows = by_max < by_total ? by_max : by_total;
+    return select() ? DSA_OK : DSA_ERR_UNSUPPORTED;
 }
 
 // ------------------------------------------------------------------ attention planning
@@ -472,8 +491,8 @@ int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexer_inputs
     IdxPlan pl;
     LaunchFn fn = nullptr;
     if (plan_indexer(batch, ix, di, pl, fn) != DSA_OK) return -1;
-    const int idx_launches = pl.mode == 1 ? 1 : (batch->batch + pl.seqs_per_launch - 1) / pl.seqs_per_launch;
-    return idx_launches + 1 + (plan_attn(batch, ix->K, di).combine ? 1 : 0);   // attention (+ merge)
+    const int64_t n_idx = pl.mode == 1 ? 1 : idx_launches(pl.windows, pl.windows_per_launch);
+    return (int32_t)n_idx + 1 + (plan_attn(batch, ix->K, di).combine ? 1 : 0);   // attention (+ merge)
 }
 
 const char* dsa_status_str(int32_t s) {

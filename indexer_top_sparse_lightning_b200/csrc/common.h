@@ -26,9 +26,13 @@ struct WsHeader {
 
 // ------------------------------------------------------------------ indexer
 // Work decomposition:
-//  mode 0 (decode): one group per sequence of the launch range [b_begin,
-//    b_end); each group gets g_b CTAs, each CTA scores a contiguous chunk of
-//    key tiles, and the group agrees on its Top-K through global histograms.
+//  mode 0 (grouped): one group per query window of the launch range
+//    [w_begin, w_end).  A window is up to NQ consecutive query tokens of one
+//    sequence (a sequence with nq_b tokens has ceil(nq_b / NQ) windows, in
+//    token order; with seq_windows every sequence is exactly one window).  A
+//    window's keys are the positions its last token sees.  Each group gets g
+//    CTAs, each CTA scores a contiguous chunk of key tiles, and the group
+//    agrees on its Top-K through published candidate keys.
 //  mode 1 (independent): every query token is its own group with one CTA;
 //    CTAs loop over tokens in zig-zag order (head-tail pairing).
 struct IndexerParams {
@@ -45,7 +49,8 @@ struct IndexerParams {
     uint32_t* cand;           // mode 0: published keys, cand_slot per CTA
     int64_t cand_slot;        // keys per CTA slot (NQ tokens share it equally)
     int32_t B, T, max_blocks, num_blocks;
-    int32_t b_begin, b_end;   // mode 0 launch range
+    int32_t w_begin, w_end;   // mode 0 launch range (window indices)
+    int32_t seq_windows;      // mode 0: every sequence has at most NQ tokens (window index = sequence)
     int32_t t_begin, t_end;   // mode 1 token range
     int32_t mode;
     int32_t K;

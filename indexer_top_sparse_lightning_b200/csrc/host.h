@@ -40,14 +40,18 @@ constexpr int kMaxDevices = 64;
 DevInfo dev_info();
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+// Mode-0 launches of a plan.
+inline int64_t idx_launches(int64_t windows, int per_launch) { return (windows + per_launch - 1) / per_launch; }
 // Bytes of the indexer's group region (sync words and publication headers).
 inline size_t group_region_bytes(int sms) { return align256((size_t)sms * (size_t)group_ws_bytes(2, sms)); }
 
 struct IdxPlan {
-    int mode = 0;        // 0 grouped decode, 1 per-token
-    int nq = 1;          // kernel NQ
+    int mode = 0;        // 0 grouped (query windows), 1 per-token
+    int nq = 1;          // kernel NQ (tokens per window in mode 0)
     int grid = 0;        // CTAs per launch
-    int seqs_per_launch = 0;
+    int seq_windows = 1; // mode 0: every sequence is one window
+    int64_t windows = 0; // mode 0: windows of the batch (an upper bound unless seq_windows)
+    int windows_per_launch = 0;
     int score_cap = 0;
     int smem = 0;
     size_t group_ws = 0; // bytes of group workspace per launch

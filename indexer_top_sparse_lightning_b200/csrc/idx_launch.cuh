@@ -91,9 +91,10 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cfg.gridDim = dim3(pl.grid, 1, 1);
-    for (int b0 = 0; b0 < bt->batch; b0 += pl.seqs_per_launch) {
-        p.b_begin = b0;
-        p.b_end = b0 + pl.seqs_per_launch < bt->batch ? b0 + pl.seqs_per_launch : bt->batch;
+    p.seq_windows = pl.seq_windows;
+    for (int64_t w0 = 0; w0 < pl.windows; w0 += pl.windows_per_launch) {
+        p.w_begin = (int32_t)w0;
+        p.w_end = (int32_t)(w0 + pl.windows_per_launch < pl.windows ? w0 + pl.windows_per_launch : pl.windows);
         if (cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p, tm_q, tm_k)) return fail(DSA_ERR_CUDA, "indexer launch", e);
     }
     return DSA_OK;

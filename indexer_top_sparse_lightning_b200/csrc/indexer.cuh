@@ -98,7 +98,8 @@ struct IdxMisc {
     uint32_t inject;          // test hook: fault injection bits (workspace status area, word 2)
     uint64_t wait_ns;         // bounded-wait limit of this launch
     // mode-0 assignment of this CTA
-    int g_valid, g_b, g_rank, g_size, g_tile_begin, g_tile_count, g_group;
+    int g_valid, g_b, g_rank, g_size, g_tile_begin, g_tile_count, g_group, g_t0, g_nq;
+    int64_t g_L;
     SelectSmem sel;
 };
 
@@ -121,9 +122,9 @@ __device__ __forceinline__ bool get_item(const IndexerParams& p, const IdxMisc* 
         it.group = m->g_group;
         it.tile_begin = m->g_tile_begin;
         it.tile_count = m->g_tile_count;
-        it.t0 = __ldg(p.cu_q + it.b);
-        it.nq = __ldg(p.cu_q + it.b + 1) - it.t0;
-        it.L = __ldg(p.seq_lens + it.b);
+        it.t0 = m->g_t0;
+        it.nq = m->g_nq;
+        it.L = m->g_L;      // keys visible to the window's last token
         for (int j = 0; j < NQ; ++j) it.pos[j] = it.L - it.nq + j;
         return true;
     }
@@ -159,27 +160,61 @@ __device__ __forceinline__ bool get_item(const IndexerParams& p, const IdxMisc* 
     return true;
 }
 
-// Mode-0 partition: every CTA computes the same split of CTAs over the
-// sequences [b_begin, b_end), proportional to their key tiles.
+// Calls f(b, t0, n, L) for the query windows [w_begin, w_end) of a mode-0 launch, in
+// order: sequence b, its tokens t0 .. t0+n-1, and L = the number of positions the
+// window's last token sees.  Window w of sequence b holds its tokens w*nq_max ..; a
+// sequence without tokens counts as one window with n = 0 (reported by the caller).
+template <typename F>
+static __device__ void for_windows(const IndexerParams& p, int nq_max, F&& f) {
+    if (p.seq_windows) {
+        for (int b = p.w_begin; b < p.w_end; ++b) {
+            const int t0 = __ldg(p.cu_q + b);
+            f(b, t0, __ldg(p.cu_q + b + 1) - t0, (int64_t)__ldg(p.seq_lens + b));
+        }
+        return;
+    }
+    int gi = 0;
+    for (int b = 0; b < p.B && gi < p.w_end; ++b) {
+        const int t0 = __ldg(p.cu_q + b), nq = __ldg(p.cu_q + b + 1) - t0;
+        const int nw = nq >= 1 ? (nq + nq_max - 1) / nq_max : 1;
+        if (gi + nw <= p.w_begin) {
+            gi += nw;
+            continue;
+        }
+        const int64_t L = __ldg(p.seq_lens + b);
+        for (int w = 0; w < nw && gi < p.w_end; ++w, ++gi) {
+            if (gi < p.w_begin) continue;
+            const int j0 = w * nq_max;
+            const int n = nq >= 1 ? (nq - j0 < nq_max ? nq - j0 : nq_max) : 0;
+            f(b, t0 + j0, n, L - nq + j0 + n);
+        }
+    }
+}
+
+// Mode-0 partition: every CTA computes the same split of CTAs over the windows
+// of the launch, proportional to their key tiles.
 static __device__ void assign_groups(const IndexerParams& p, IdxMisc* m, int nq_max, int score_cap) {
-    const int Bp = p.b_end - p.b_begin;
     const int C = gridDim.x;
     int64_t total = 0;
-    for (int b = p.b_begin; b < p.b_end; ++b) total += (__ldg(p.seq_lens + b) + kTileKeys - 1) / kTileKeys;
+    int Wn = 0;
+    for_windows(p, nq_max, [&](int, int, int, int64_t L) {
+        total += (L + kTileKeys - 1) / kTileKeys;
+        ++Wn;
+    });
     m->g_valid = 0;
-    if (total <= 0 || C < Bp) return;
-    int acc = 0;
-    for (int b = p.b_begin; b < p.b_end; ++b) {
-        const int64_t L = __ldg(p.seq_lens + b);
+    if (total <= 0 || C < Wn) return;
+    int acc = 0, gidx = 0;
+    bool done = false;
+    for_windows(p, nq_max, [&](int b, int t0, int nq, int64_t L) {
+        if (done) return;
         const int tiles = (int)((L + kTileKeys - 1) / kTileKeys);
-        int g = 1 + (int)(((int64_t)(C - Bp) * tiles) / total);
+        int g = 1 + (int)(((int64_t)(C - Wn) * tiles) / total);
         if (g > tiles) g = tiles;
         if (g < 1) g = 1;
         if ((int)blockIdx.x >= acc && (int)blockIdx.x < acc + g) {
+            done = true;
             const int r = (int)blockIdx.x - acc;
             const int base = tiles / g, rem = tiles % g;
-            const int t0 = __ldg(p.cu_q + b);
-            const int nq = __ldg(p.cu_q + b + 1) - t0;
             const int max_chunk = (base + (rem ? 1 : 0)) * kTileKeys;
             if (nq < 1 || nq > nq_max || nq > L || t0 < 0 || t0 + nq > p.T || L > (int64_t)p.max_blocks * kPage) {
                 set_status(p.status, kStBounds);
@@ -191,15 +226,18 @@ static __device__ void assign_groups(const IndexerParams& p, IdxMisc* m, int nq_
             }
             m->g_valid = 1;
             m->g_b = b;
+            m->g_t0 = t0;
+            m->g_nq = nq;
+            m->g_L = L;
             m->g_rank = r;
             m->g_size = g;
-            m->g_group = b - p.b_begin;
+            m->g_group = gidx;
             m->g_tile_begin = r * base + (r < rem ? r : rem);
             m->g_tile_count = base + (r < rem ? 1 : 0);
-            return;
         }
         acc += g;
-    }
+        ++gidx;
+    });
 }
 
 template <bool FP8, int HI, int DI, int NQ>

@@ -158,6 +158,35 @@ def test_prefill_after_cached_prefix():
     assert_topk(wl, tok, idx[tok], score[tok], exact=False)
 
 
+@pytest.mark.parametrize("key_dtype", ["bf16", "fp8"])
+def test_long_chunk_on_long_prefix(key_dtype):
+    # 700 new tokens on a 40,000-token cached prefix: a token's score row does not fit
+    # one CTA, so the tokens go in windows of two, each window split over several CTAs
+    wl = W.make_workload("chunk40k", seq_lens=[40700], nq=700, H_I=64, D_I=128, H=1, K=2048, seed=12,
+                         key_dtype=key_dtype, with_kv=False)
+    idx, score = run_indexer(wl)
+    tok = np.concatenate([np.arange(0, 700, 53), [1, 698, 699]])
+    assert_topk(wl, tok, idx[tok], score[tok], exact=False)
+
+
+def test_three_token_verify_at_64k():
+    # speculative verify with three tokens per sequence at 64K context: two windows per
+    # sequence (tokens 0-1, token 2), both sequences in one grouped launch
+    wl = W.make_workload("verify3", seq_lens=[65536, 50000], nq=3, H_I=64, D_I=128, H=1, K=2048, seed=13,
+                         with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+def test_uneven_windows_integer_inputs_bit_exact():
+    # 5, 1 and 3 tokens per sequence past what one CTA stages (32,768 positions): full and
+    # partial windows, a one-token sequence among them; integer inputs make every score exact
+    wl = W.make_workload("windows", seq_lens=[60000, 40000, 52000], nq=[5, 1, 3], H_I=8, D_I=64, H=1, K=512,
+                         seed=14, int_inputs=True, w_dist="u256", with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
+
+
 def test_score_output_is_optional():
     wl = W.preset("tiny", with_kv=False)
     idx, score = run_indexer(wl, want_score=False)
