@@ -11,7 +11,9 @@ constexpr int kTileKeys = 128;        // keys per indexer MMA tile (two pages)
 constexpr int kMaxTopK = 2048;
 constexpr int kDqk = 576;             // latent 512 + RoPE 64
 constexpr int kDv = 512;
-constexpr int kEpiThreads = 128;      // four epilogue warps, one TMEM lane each
+constexpr int kEpiWarps = 8;          // indexer epilogue / Top-K warps (two per TMEM lane quarter)
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kConvThreads = 128;     // fp8 key widening threads (four warps)
 
 // Device status word values (mirrors dsa_status).
 enum : uint32_t {

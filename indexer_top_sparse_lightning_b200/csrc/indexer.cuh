@@ -60,9 +60,14 @@ struct IdxCfg {
     static constexpr bool Q_PAD = NQ * HI < N;                // rows [NQ*HI, N) stay zero
     static constexpr int HIST_WORDS = kBins;                  // select histograms
     static constexpr int W_FLOATS = NQ * HI;
-    static constexpr int THREADS = FP8 ? 320 : 192;
-    static constexpr int PRODUCER_WARP = 4;
-    static constexpr int MMA_WARP = 5;
+    // warps 0-7 epilogue and Top-K, 8 TMA producer, 9 MMA issuer, 10-13 fp8 widening
+    static constexpr int THREADS = kEpiThreads + 64 + (FP8 ? kConvThreads : 0);
+    static constexpr int PRODUCER_WARP = kEpiWarps;
+    static constexpr int MMA_WARP = kEpiWarps + 1;
+    static constexpr int CONV_WARP0 = kEpiWarps + 2;
+    // heads split between the two warps of a TMEM lane quarter (HI >= 32), else one warp
+    static constexpr bool SPLIT = HI >= 32;
+    static constexpr int HH = SPLIT ? HI / 2 : HI;            // heads per epilogue thread
     static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, false, false);
 
     static constexpr int OFF_STAGE = 0;
@@ -74,7 +79,9 @@ struct IdxCfg {
     static constexpr int MISC_BYTES = 1024;
     static constexpr int MAX_PAGES = 512;                     // page ids of one work item, staged in smem
     static constexpr int OFF_BLK = OFF_MISC + MISC_BYTES;
-    static constexpr int OFF_LIST = OFF_BLK + MAX_PAGES * 4;   // select list, u32 [kListCap]
+    // partial head sums handed between the two warps of a lane quarter, [2][NQ][128]
+    static constexpr int OFF_PART = OFF_BLK + MAX_PAGES * 4;
+    static constexpr int OFF_LIST = OFF_PART + (SPLIT ? 2 * NQ * kTileKeys * 4 : 0);   // select list, u32 [kListCap]
     static constexpr int OFF_SCORE = OFF_LIST + kListCap * 4;
     // shared memory free during grouped select (the key stages and widened keys)
     static constexpr int SCRATCH_BYTES = OFF_Q - OFF_STAGE;
@@ -263,10 +270,10 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < Cfg::NSTAGE; ++i) {
             mbar_init(&m->full[i], 1);
-            mbar_init(&m->empty[i], FP8 ? kEpiThreads : 1);
+            mbar_init(&m->empty[i], FP8 ? kConvThreads : 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&m->conv_full[i], kEpiThreads);
+            mbar_init(&m->conv_full[i], kConvThreads);
             mbar_init(&m->conv_empty[i], 1);
             mbar_init(&m->tfull[i], 1);
             mbar_init(&m->tempty[i], kEpiThreads);
@@ -423,9 +430,9 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             volatile int no_abort = 0;
             mbar_wait(&m->drain, 0, &no_abort, wlim);
         }
-    } else if (FP8 && warp >= 6) {
+    } else if (FP8 && warp >= Cfg::CONV_WARP0) {
         // ---------------------------------------------------------------- fp8 -> bf16 widening
-        const int ct = threadIdx.x - 192;
+        const int ct = threadIdx.x - Cfg::CONV_WARP0 * 32;
         uint32_t it = 0;
         IdxItem item;
         bool ok = true;
@@ -439,7 +446,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 const uint8_t* raw = s_stage + s * Cfg::STAGE_BYTES;
                 uint8_t* dst = s_conv + cb * Cfg::CONV_BYTES;
 #pragma unroll 4
-                for (int u = ct; u < kTileKeys * CH; u += kEpiThreads) {
+                for (int u = ct; u < kTileKeys * CH; u += kConvThreads) {
                     const int r = u / CH, c = u % CH;
                     const uint4 v = *reinterpret_cast<const uint4*>(raw + r * DI + c * 16);
                     uint32_t outw[8];
@@ -468,9 +475,16 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 mbar_arrive(&m->empty[s]);
             }
         }
-    } else if (warp < 4) {
+    } else if (warp < kEpiWarps) {
         // ---------------------------------------------------------------- epilogue + select
-        const int row = threadIdx.x;            // TMEM lane == key row in the tile
+        // Warps w and w+4 read the same TMEM lanes (key rows 32*(w%4)..): with SPLIT each
+        // sums half of the heads and warp w adds warp w+4's partial; otherwise warps 4-7
+        // wait out the epilogue.  All eight warps run the Top-K.
+        const int row = 32 * (warp & 3) + lane;   // TMEM lane == key row in the tile
+        const int half = warp >> 2;
+        const bool scorer = Cfg::SPLIT || half == 0;
+        const bool owner = half == 0;              // writes the final score of its row
+        float* s_part = reinterpret_cast<float*>(smem + Cfg::OFF_PART);
         uint32_t it = 0;
         IdxItem item;
         bool ok = true;
@@ -508,7 +522,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 const int buf = it & 1;
                 const int64_t pos = chunk0 + (int64_t)li * kTileKeys + row;
                 float sc[2] = {1.0f, 1.0f};
-                if (FP8) {
+                if (FP8 && scorer) {
                     const int64_t pg = pos / kPage;
                     if (pg < npages) {
                         const int bid = __ldg(p.block_table + (int64_t)item.b * p.max_blocks + pg);
@@ -519,19 +533,25 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         }
                     }
                 }
-                if (!mbar_wait(&m->tfull[buf], (it >> 1) & 1, abort, wlim)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * Cfg::COLS_BUF;
+                const bool got = mbar_wait(&m->tfull[buf], (it >> 1) & 1, abort, wlim);
                 float score[NQ];
 #pragma unroll
-                for (int j = 0; j < NQ; ++j) {
-                    float acc = 0.0f;
-                    if (j < item.nq) {
-                        constexpr int CW = HI < 32 ? HI : 32;
+                for (int j = 0; j < NQ; ++j) score[j] = 0.0f;
+                if (got) {
+                    tc_fence_after();
+                    const uint32_t tb = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + buf * Cfg::COLS_BUF;
 #pragma unroll
-                        for (int c0 = 0; c0 < HI; c0 += CW) {
+                    for (int j = 0; j < NQ; ++j) {
+                        if (!scorer || j >= item.nq) continue;
+                        // four independent partial sums (head h into sum h % 4), weights
+                        // read four at a time
+                        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                        constexpr int CW = Cfg::HH < 32 ? Cfg::HH : 32;
+#pragma unroll
+                        for (int c0 = 0; c0 < Cfg::HH; c0 += CW) {
                             uint32_t a0[32], a1[32];
-                            const uint32_t col = j * HI + c0;
+                            const int h0 = (Cfg::SPLIT ? half * Cfg::HH : 0) + c0;   // first head of the chunk
+                            const uint32_t col = j * HI + h0;
                             if constexpr (CW == 32) {
                                 tmem_ld32(tb + col, a0);
                                 if (FP8 && Cfg::KB > 1) tmem_ld32(tb + Cfg::N + col, a1);
@@ -543,25 +563,41 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                                 if (FP8 && Cfg::KB > 1) tmem_ld8(tb + Cfg::N + col, *reinterpret_cast<uint32_t(*)[8]>(a1));
                             }
                             tmem_wait_ld();
+                            const float4* w4 = reinterpret_cast<const float4*>(s_w + j * HI + h0);
 #pragma unroll
-                            for (int h = 0; h < CW; ++h) {
-                                float x = __uint_as_float(a0[h]);
-                                if (FP8) {
-                                    x = x * sc[0];
-                                    if (Cfg::KB > 1) x = fmaf(__uint_as_float(a1[h]), sc[1], x);
+                            for (int h = 0; h < CW; h += 4) {
+                                const float4 wv = w4[h >> 2];
+                                const float wq[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    float x = __uint_as_float(a0[h + e]);
+                                    if (FP8) {
+                                        x = x * sc[0];
+                                        if (Cfg::KB > 1) x = fmaf(__uint_as_float(a1[h + e]), sc[1], x);
+                                    }
+                                    part[e] = fmaf(wq[e], fmaxf(x, 0.0f), part[e]);
                                 }
-                                acc = fmaf(s_w[j * HI + c0 + h], fmaxf(x, 0.0f), acc);
                             }
                         }
+                        score[j] = (part[0] + part[1]) + (part[2] + part[3]);
                     }
-                    score[j] = acc;
+                    tc_fence_before();
+                    mbar_arrive(&m->tempty[buf]);
+                    if (Cfg::SPLIT && !owner) {
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) s_part[(buf * NQ + j) * kTileKeys + row] = score[j];
+                    }
                 }
-                tc_fence_before();
-                mbar_arrive(&m->tempty[buf]);
+                // the hand-over barrier carries the exit vote, so every thread leaves together
+                const bool all = Cfg::SPLIT ? named_bar_and(2, kEpiThreads, got) : got;
+                if (!all) { ok = false; break; }
+                if (!owner) continue;
 #pragma unroll
                 for (int j = 0; j < NQ; ++j) {
                     if (j < item.nq) {
-                        const float f = score[j] == 0.0f ? 0.0f : score[j];
+                        float f = score[j];
+                        if (Cfg::SPLIT) f += s_part[(buf * NQ + j) * kTileKeys + row];
+                        f = f == 0.0f ? 0.0f : f;
                         s_score[j * stride + li * kTileKeys + row] = f;
                         // range of the visible keys, for the select's first histogram
                         if (pos <= item.pos[j]) {

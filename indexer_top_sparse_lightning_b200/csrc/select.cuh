@@ -28,7 +28,7 @@
 //      CTA's output offset and its share of the tied elements.
 // Elements above T are selected; elements equal to T are selected lowest
 // position first (CTAs own contiguous position ranges in rank order, and
-// within a CTA warp w owns the w-th quarter).  Indices are written in
+// within a CTA warp w owns the w-th eighth).  Indices are written in
 // ascending position order with ballots and prefix counts.
 #pragma once
 #include "common.h"
@@ -40,15 +40,15 @@ constexpr int kBins = 2048;      // range histogram bins (11 bits)
 constexpr int kListCap = 1024;   // keys of the threshold bin resolved exactly
 
 struct SelectSmem {
-    uint32_t scan[8];
+    uint32_t scan[kEpiWarps];
     uint32_t kmin[4], kmax[4];   // order keys of the visible local scores, per token (from the epilogue)
     uint32_t res_bin, res_kk, res_cnt;
     uint32_t fill;               // list / published-key fill counter
     uint32_t cmin;               // smallest published key
-    uint32_t wcnt[4][2];         // [warp][gt, eq]
-    uint32_t wallow[4];
+    uint32_t wcnt[kEpiWarps][2]; // [warp][gt, eq]
+    uint32_t wallow[kEpiWarps];
     uint32_t edge[4];            // this CTA's publication edge, per token
-    uint32_t wpub[4][4];         // [token][warp] published elements
+    uint32_t wpub[4][kEpiWarps]; // [token][warp] published elements
     uint32_t g_lo, g_hi, g_total, g_resident, g_max_edge;
     uint32_t gphase;             // phase of the published-key load barrier
 };
@@ -57,7 +57,7 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) {
     atomicCAS(status, 0u, code);
 }
 
-// Bounded barrier among the CTAs of one group (called by the 128 select
+// Bounded barrier among the CTAs of one group (called by the select
 // threads).  Sense-reversing: the last arriver resets the count and bumps
 // the generation.  `gen` is thread 0's copy of the generation, read once per
 // work item and advanced here, so a barrier costs one atomic and the wait.
@@ -89,7 +89,7 @@ static __device__ bool group_barrier(uint32_t* sync, int G, uint32_t& gen, uint3
     return !*abort;
 }
 
-// Exclusive prefix over the 128 select threads; *total receives the sum.
+// Exclusive prefix over the select threads; *total receives the sum.
 __device__ __forceinline__ uint32_t epi_exclusive_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t x = v;
@@ -102,7 +102,7 @@ __device__ __forceinline__ uint32_t epi_exclusive_scan(uint32_t v, uint32_t* scr
     named_bar_sync(1, kEpiThreads);
     uint32_t before = 0, all = 0;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < kEpiWarps; ++w) {
         const uint32_t s = scratch[w];
         if (w < warp) before += s;
         all += s;
@@ -231,11 +231,12 @@ struct GlobalKeyStream {
     }
 };
 
-// Exact kk-th largest key among the n keys in `list`.  Short lists: every
-// element counts the larger and equal ones (broadcast reads, one barrier);
-// longer ones: radix select with 8-bit digits in hist[0..255].
+// Exact kk-th largest key among the n keys in `list`.  Short lists (at most
+// 256): every element counts the larger and equal ones (broadcast reads, one
+// barrier); longer ones: radix select with 8-bit digits in hist[0..255].
 static __device__ uint32_t list_select(const uint32_t* list, int n, uint32_t kk, uint32_t* hist, SelectSmem* sm) {
-    if (n <= 2 * kEpiThreads) {
+    static_assert(2 * kEpiThreads >= 256, "short lists: at most two elements per thread");
+    if (n <= 256) {
         uint32_t mine[2];
         uint32_t gt[2] = {0u, 0u}, eq[2] = {0u, 0u};
 #pragma unroll
@@ -380,7 +381,7 @@ __device__ uint32_t sampled_threshold(const Stream& st, uint32_t lo, uint32_t hi
     named_bar_sync(1, kEpiThreads);
     above = inside = 0;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < kEpiWarps; ++w) {
         above += sm->wcnt[w][0];
         inside += sm->wcnt[w][1];
     }
@@ -400,7 +401,7 @@ struct GroupView {
 // Exact Top-K of NQ tokens' score rows held in shared memory (s_score, token
 // j at j*stride, nloc[j] valid entries starting at position chunk0).
 // Writes out_idx/out_score rows [t0 + j] in ascending position order.
-// Called by the 128 select threads; sm->kmin/kmax[j] hold the smallest and
+// Called by the select threads; sm->kmin/kmax[j] hold the smallest and
 // largest key of the visible scores.  s_hist holds kBins words, s_list
 // kListCap; `scratch` (scratch_bytes, 16-byte aligned) is shared memory that
 // is free in grouped work (the key stages).
@@ -415,18 +416,18 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
     const int G = gv.G;
     const int64_t slot_keys = p.cand_slot / NQ;
 
-    // warp w owns the w-th quarter of a token's elements (quarters are multiples of 32)
+    // warp w owns the w-th eighth of a token's elements (eighths are multiples of 32)
     int qlen[NQ], list_off[NQ];
     int list_words = 0;     // u16 entries of all per-warp lists
 #pragma unroll
     for (int j = 0; j < NQ; ++j) {
-        qlen[j] = ((nloc[j] + 4 * 32 - 1) / (4 * 32)) * 32;
+        qlen[j] = ((nloc[j] + kEpiWarps * 32 - 1) / (kEpiWarps * 32)) * 32;
         list_off[j] = list_words;
-        list_words += 4 * qlen[j];
+        list_words += kEpiWarps * qlen[j];
     }
     // Grouped work keeps, per warp, the position-ordered list of its published
     // elements (a superset of its selected ones) when the lists take at most
-    // half of the scratch; otherwise its whole quarter is scanned again.
+    // half of the scratch; otherwise its whole eighth is scanned again.
     const int list_bytes = ((list_words * 2 + 15) / 16) * 16;
     const bool lists = G > 1 && 2 * list_bytes <= scratch_bytes;
     uint16_t* s_lists = reinterpret_cast<uint16_t*>(scratch);
@@ -434,7 +435,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
     const int gscratch_bytes = scratch_bytes - (lists ? list_bytes : 0);
 
     // The n-th element of warp `warp`'s sequence for token j: in list mode the
-    // listed local indices, otherwise its quarter.
+    // listed local indices, otherwise its eighth.
     auto seq_len = [&](int j) -> int {
         if (lists) return (int)sm->wpub[j][warp];
         const int beg = warp * qlen[j];
@@ -488,7 +489,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         const float* sj = s_score + j * stride;
         uint32_t off = 0, tot = 0;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < kEpiWarps; ++w) {
             if (w < warp) off += sm->wpub[j][w];
             tot += sm->wpub[j][w];
         }
@@ -558,12 +559,13 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
     };
 
     auto gather = [&](int j) {
-        // headers of ranks tid and tid + 128 (G <= 256), read together; flat offsets
+        // headers of ranks tid + u * threads (G <= 256), read together; flat offsets
         // of the (4-padded) ranks by a prefix over rank order
-        static_assert(kEpiThreads == 128, "two header slots per thread cover 256 ranks");
-        uint4 h[2];
+        constexpr int HS = 256 / kEpiThreads;
+        static_assert(HS * kEpiThreads == 256, "header slots per thread cover 256 ranks");
+        uint4 h[HS];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < HS; ++u) {
             const int r = (int)threadIdx.x + u * kEpiThreads;
             h[u] = r < G ? __ldcg(reinterpret_cast<const uint4*>(gv.hdr + ((int64_t)r * NQ + j) * 4))
                          : make_uint4(0u, 0xFFFFFFFFu, 0u, 0u);
@@ -573,16 +575,20 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
             sm->g_hi = 0u;
             sm->g_max_edge = 0u;
         }
-        uint32_t tot0, tot1;
-        const uint32_t off0 = epi_exclusive_scan((h[0].x + 3u) & ~3u, sm->scan, &tot0);
-        const uint32_t off1 = tot0 + epi_exclusive_scan((h[1].x + 3u) & ~3u, sm->scan, &tot1);
+        uint32_t offs[HS], totall = 0;
+#pragma unroll
+        for (int u = 0; u < HS; ++u) {
+            uint32_t tu;
+            offs[u] = totall + epi_exclusive_scan((h[u].x + 3u) & ~3u, sm->scan, &tu);
+            totall += tu;
+        }
         uint32_t lo = 0xFFFFFFFFu, hi = 0u, emax = 0u;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < HS; ++u) {
             const int r = (int)threadIdx.x + u * kEpiThreads;
             if (r < G) {
                 rt[2 * r] = h[u].x;
-                rt[2 * r + 1] = u == 0 ? off0 : off1;
+                rt[2 * r + 1] = offs[u];
                 if (h[u].x) {
                     lo = min(lo, h[u].y);
                     hi = max(hi, h[u].z);
@@ -602,7 +608,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
             red_max_shared(&sm->g_max_edge, emax);
         }
         if (threadIdx.x == 0) {
-            const uint32_t off = tot0 + tot1;
+            const uint32_t off = totall;
             sm->g_total = off;
             sm->g_resident = (int64_t)((2 * G + 3) & ~3) * 4 + (int64_t)off * 4 <= (int64_t)gscratch_bytes;
         }
@@ -755,7 +761,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
             named_bar_sync(1, kEpiThreads);
             uint32_t gtb = 0, eqb = 0, gta = 0;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
+            for (int w = 0; w < kEpiWarps; ++w) {
                 gtb += sm->wcnt[w][0];
                 eqb += sm->wcnt[w][1];
                 gta += sm->wallow[w];
@@ -768,7 +774,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         }
 
         // ---- per-warp counts of this CTA's elements above / equal to T, over
-        // the warp's position-ordered sequence (list or quarter)
+        // the warp's position-ordered sequence (list or eighth)
         // (float compares against T's value: the same order as the keys for
         // finite scores, and -0 == +0 like the folded keys)
         const int n = seq_len(j);
@@ -799,7 +805,7 @@ __device__ bool topk_select(const IndexerParams& p, const GroupView& gv, uint32_
         named_bar_sync(1, kEpiThreads);
         uint32_t gt_before = 0, eq_before = 0, cgt = 0, ceq = 0, weq = 0;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < kEpiWarps; ++w) {
             const uint32_t g = sm->wcnt[w][0], e = sm->wcnt[w][1];
             if (w < warp) {
                 gt_before += g;
