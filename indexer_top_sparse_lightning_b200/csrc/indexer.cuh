@@ -50,7 +50,10 @@ struct IdxCfg {
     static constexpr int ACC = FP8 ? KB : 1;                  // fp8: one accumulator per scale group
     static constexpr int COLS_BUF = N * ACC;
     static constexpr int TMEM_COLS = pow2_at_least(2 * COLS_BUF);
-    static constexpr int NSTAGE = FP8 ? 4 : (NQ == 1 ? 4 : 3);
+    // key stages in flight: fp8 keys keep three (their widened copies take two more
+    // buffers), so that a CTA holds 16 K scores and a 128 K-context batch of eight
+    // plans into one grouped launch
+    static constexpr int NSTAGE = FP8 ? 3 : (NQ == 1 ? 4 : 3);
     static constexpr int STAGE_BYTES = kTileKeys * DI * (FP8 ? 1 : 2);
     static constexpr int NCONV = FP8 ? 2 : 0;                 // widened-operand buffers
     static constexpr int NCV = FP8 ? 2 : 1;                   // (modulus for the ring index)
