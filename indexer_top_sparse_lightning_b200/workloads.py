@@ -12,7 +12,9 @@ head weights, paged block tables, sequence lengths, K and latent KV):
 * indexer queries ``q_idx``  [T, H_I, D_I]   bf16 (stored as uint16 bits)
 * head weights    ``w``      [T, H_I]        fp32
 * indexer keys    ``k_idx``  [nblk, 64, D_I] bf16 bits, or e4m3 codes (uint8)
-                  ``k_scale``[nblk, 64, D_I/64] fp32 (fp8 keys only)
+                  ``k_scale``[nblk, 64, D_I/64] fp32 (fp8 keys), or
+                             [nblk, 64, D_I/32] uint8 shared exponents (MXFP8 keys)
+* MXFP8 queries   ``q_idx``  [T, H_I, D_I] e4m3 codes, ``q_scale`` [T, H_I, D_I/32] uint8
 * MLA queries     ``q``      [T, H, 576]     bf16 bits (512 latent + 64 RoPE)
 * latent cache    ``kv``     [nblk, 64, 576] bf16 bits
 * ``block_table`` [B, max_blocks] int32 (-1 past a sequence's last page);
@@ -69,20 +71,21 @@ class Workload:
     D_I: int
     H: int
     K: int
-    key_dtype: str               # "bf16" or "fp8"
+    key_dtype: str               # "bf16", "fp8" or "mxfp8" (MXFP8 queries too)
     seq_lens: np.ndarray         # [B] int32
     cu_q: np.ndarray             # [B+1] int32
     block_table: np.ndarray      # [B, max_blocks] int32
     num_blocks: int
-    q_idx: np.ndarray            # [T, H_I, D_I] uint16 (bf16 bits)
+    q_idx: np.ndarray            # [T, H_I, D_I] uint16 (bf16 bits), or uint8 e4m3 codes (mxfp8)
     w: np.ndarray                # [T, H_I] float32
     k_idx: np.ndarray            # [nblk, 64, D_I] uint16 (bf16) or uint8 (e4m3)
-    k_scale: Optional[np.ndarray]  # [nblk, 64, D_I//64] float32 or None
+    k_scale: Optional[np.ndarray]  # [nblk, 64, D_I//64] float32, [nblk, 64, D_I//32] uint8 (mxfp8) or None
     q: np.ndarray                # [T, H, 576] uint16
     kv: np.ndarray               # [nblk, 64, 576] uint16
     sm_scale: float
     planted: Optional[np.ndarray] = None   # sorted positions of a planted Top-K set
     seed: int = 0
+    q_scale: Optional[np.ndarray] = None   # [T, H_I, D_I//32] uint8 (mxfp8 queries)
 
     @property
     def max_blocks(self) -> int:
@@ -110,6 +113,8 @@ class Workload:
         per = self.D_I * (2 if self.key_dtype == "bf16" else 1)
         if self.key_dtype == "fp8":
             per += 4 * (self.D_I // 64)
+        elif self.key_dtype == "mxfp8":
+            per += self.D_I // 32
         return int(np.sum(self.seq_lens.astype(np.int64))) * per
 
     def indexer_flops(self) -> int:
@@ -178,6 +183,20 @@ def _quantize_fp8_groups(x: np.ndarray, group: int = 64):
     return codes.reshape(x.shape), scale
 
 
+def _quantize_mx(x: np.ndarray):
+    """MXFP8 encoding along the last axis, 32 contiguous elements per group: the
+    shared scale is X = 2^(floor(log2 amax) - 8) (8 = the largest e4m3 exponent),
+    stored as the byte e = log2 X + 127; the elements are e4m3fn(x / X), rounded to
+    nearest even and saturated at +-448.  An all-zero group gets X = 1."""
+    g = x.reshape(*x.shape[:-1], x.shape[-1] // 32, 32).astype(np.float64)
+    amax = np.abs(g).max(axis=-1)
+    safe = np.where(amax > 0, amax, 1.0)
+    ex = np.where(amax > 0, np.floor(np.log2(safe)) - 8, 0).astype(np.int64)
+    ex = np.clip(ex, -127, 127)
+    codes = encode_e4m3((g / np.ldexp(1.0, ex)[..., None]).astype(np.float32))
+    return codes.reshape(x.shape), (ex + 127).astype(np.uint8)
+
+
 def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=128, K=2048,
                   key_dtype="bf16", int_inputs=False, w_dist="u8", shuffle=True,
                   planted_k: int = 0, planted_tail: bool = False, seed: int = 0,
@@ -204,7 +223,15 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
 
     table, num_blocks = _paging(_rng(seed, 1), seq_lens, shuffle)
 
-    if int_inputs:
+    mx = key_dtype == "mxfp8"
+    q_scale = None
+    if mx:
+        # MXFP8 index queries: drawn in float32, then encoded
+        rq = _rng(seed, 2)
+        q_f = (rq.integers(-4, 5, size=(T, H_I, D_I)).astype(np.float32) if int_inputs
+               else rq.standard_normal((T, H_I, D_I), dtype=np.float32))
+        q_idx, q_scale = _quantize_mx(q_f)
+    elif int_inputs:
         q_idx = to_bf16_bits(_rng(seed, 2).integers(-4, 5, size=(T, H_I, D_I)).astype(np.float32))
     else:
         q_idx = _normal_bf16(seed, 2, (T, H_I, D_I))
@@ -231,7 +258,7 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
     plant_rows = plant_vals = None
     if planted_k:
         # keys along the query's head-weighted direction, far above the N(0,1) keys
-        assert B == 1 and T == 1
+        assert B == 1 and T == 1 and not mx
         rp = _rng(seed, 5)
         L = int(seq_lens[0])
         if planted_tail:
@@ -253,6 +280,12 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
         if planted_k:
             k_idx.reshape(n_keys, D_I)[plant_rows] = to_bf16_bits(plant_vals)
         k_scale = None
+    elif mx:
+        k_f = (r.integers(-4, 5, size=(n_keys, D_I)).astype(np.float32) if int_inputs
+               else r.standard_normal((n_keys, D_I), dtype=np.float32))
+        codes, ex = _quantize_mx(k_f)
+        k_idx = codes.reshape(num_blocks, BLOCK, D_I)
+        k_scale = ex.reshape(num_blocks, BLOCK, D_I // 32)
     else:
         k_f = r.standard_normal((n_keys, D_I), dtype=np.float32)
         if planted_k:
@@ -271,7 +304,7 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
     return Workload(name=name, B=B, T=T, H_I=H_I, D_I=D_I, H=H, K=K, key_dtype=key_dtype,
                     seq_lens=seq_lens, cu_q=cu_q, block_table=table, num_blocks=num_blocks,
                     q_idx=q_idx, w=w, k_idx=k_idx, k_scale=k_scale, q=q, kv=kv,
-                    sm_scale=1.0 / math.sqrt(D_QK), planted=planted, seed=seed)
+                    sm_scale=1.0 / math.sqrt(D_QK), planted=planted, seed=seed, q_scale=q_scale)
 
 
 # The five workloads.  Seeds are 1000 + index.
@@ -291,6 +324,9 @@ PRESETS = {
     # batch 1, 1M context, fp8 keys, planted dominant Top-K set, w ~ U(0,1).
     "1m": dict(seq_lens=[1 << 20], nq=1, H_I=64, D_I=128, H=128, K=2048, key_dtype="fp8",
                w_dist="u", planted_k=2048, seed=1004),
+    # batch32 with MXFP8 index queries and keys (e4m3, one power-of-two scale per 32 elements)
+    "batch32_mxfp8": dict(seq_lens=[32768] * 32, nq=1, H_I=64, D_I=128, H=128, K=2048, key_dtype="mxfp8",
+                          w_dist="u8", seed=1005),
 }
 
 
@@ -312,8 +348,10 @@ def to_device(wl: Workload, device="cuda", with_kv: bool = True) -> dict:
             x = x.view(dtype)
         return x.to(device)
 
+    mx = wl.key_dtype == "mxfp8"
     d = dict(seq_lens=t(wl.seq_lens), cu_q=t(wl.cu_q), block_table=t(wl.block_table),
-             q_idx=t(wl.q_idx, torch.bfloat16), w=t(wl.w))
+             q_idx=t(wl.q_idx) if mx else t(wl.q_idx, torch.bfloat16), w=t(wl.w),
+             q_scale=t(wl.q_scale) if mx else None)
     if wl.key_dtype == "bf16":
         d["k_cache"] = t(wl.k_idx, torch.bfloat16)
         d["k_scale"] = None

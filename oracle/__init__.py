@@ -40,7 +40,7 @@ class _IndexerArgs(ctypes.Structure):
                 ("seq_lens", ctypes.c_void_p), ("cu_q", ctypes.c_void_p),
                 ("block_table", ctypes.c_void_p), ("max_blocks", ctypes.c_int32),
                 ("q_idx", ctypes.c_void_p), ("w", ctypes.c_void_p), ("k_idx", ctypes.c_void_p),
-                ("k_scale", ctypes.c_void_p)]
+                ("k_scale", ctypes.c_void_p), ("q_mx", ctypes.c_int32), ("q_scale", ctypes.c_void_p)]
 
 
 class _AttnArgs(ctypes.Structure):
@@ -62,6 +62,8 @@ def _bind(path):
                                        ctypes.c_void_p, ctypes.c_void_p]
     lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
     lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+    lib.oracle_e8m0_to_f64.argtypes = [ctypes.c_uint8]
+    lib.oracle_e8m0_to_f64.restype = ctypes.c_double
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
 
@@ -102,17 +104,22 @@ def _ptr(a):
     return a.ctypes.data if a is not None else None
 
 
+_KEY_FORMAT = {"bf16": 0, "fp8": 1, "mxfp8": 2}
+
+
 def _indexer_args(wl, keep):
+    mx = wl.key_dtype == "mxfp8"
     arrs = dict(seq_lens=_c(wl.seq_lens, np.int32), cu_q=_c(wl.cu_q, np.int32),
-                block_table=_c(wl.block_table, np.int32), q_idx=_c(wl.q_idx, np.uint16),
+                block_table=_c(wl.block_table, np.int32), q_idx=_c(wl.q_idx, np.uint8 if mx else np.uint16),
                 w=_c(wl.w, np.float32),
                 k_idx=_c(wl.k_idx, np.uint16 if wl.key_dtype == "bf16" else np.uint8),
-                k_scale=None if wl.k_scale is None else _c(wl.k_scale, np.float32))
+                k_scale=None if wl.k_scale is None else _c(wl.k_scale, np.uint8 if mx else np.float32),
+                q_scale=_c(wl.q_scale, np.uint8) if mx else None)
     keep.append(arrs)
-    return _IndexerArgs(wl.B, wl.T, wl.H_I, wl.D_I, wl.K, 0 if wl.key_dtype == "bf16" else 1,
+    return _IndexerArgs(wl.B, wl.T, wl.H_I, wl.D_I, wl.K, _KEY_FORMAT[wl.key_dtype],
                         _ptr(arrs["seq_lens"]), _ptr(arrs["cu_q"]), _ptr(arrs["block_table"]),
                         wl.block_table.shape[1], _ptr(arrs["q_idx"]), _ptr(arrs["w"]),
-                        _ptr(arrs["k_idx"]), _ptr(arrs["k_scale"]))
+                        _ptr(arrs["k_idx"]), _ptr(arrs["k_scale"]), 1 if mx else 0, _ptr(arrs["q_scale"]))
 
 
 def indexer_topk(wl, tokens=None, want_all_scores: bool = False):
@@ -184,6 +191,10 @@ def sparse_attn(wl, idx, tokens=None, sm_scale=None):
 
 def e4m3_to_f64(code: int) -> float:
     return float(_load().oracle_e4m3_to_f64(int(code)))
+
+
+def e8m0_to_f64(e: int) -> float:
+    return float(_load().oracle_e8m0_to_f64(int(e)))
 
 
 def num_threads() -> int:

@@ -21,6 +21,11 @@
  *     fp8 keys: k[s,d] = e4m3(code[s,d]) * scale[s, d/64] (one fp32 scale per
  *     64 contiguous elements of a key; "Day0 Adaptation and Performance
  *     Optimization ...", section 4, every N elements share a scaling factor).
+ *     MXFP8 index queries and keys (same page, section 4: full quantization of
+ *     index Q/K in the MXFP8 format, every 32 elements share a scaling factor;
+ *     "Optimizing and Deploying Ultra-Long Sequence Inference Architectures",
+ *     section II item 1): x[d] = e4m3(code[d]) * 2^(e[d/32] - 127), e an
+ *     8-bit power-of-two scale shared by 32 contiguous elements of one vector.
  *
  *  2. Top-K selection.  "Large Model Inference Acceleration: Day-0
  *     Adaptation ...", section 1.1 (a Top-K pass picks the most important
@@ -60,6 +65,13 @@ static double bf16_to_f64(uint16_t b) {
     return (double)f;
 }
 
+/* MX shared scale (8 exponent bits, no mantissa) -> double: 2^(e - 127);
+ * 0xFF is NaN (the generator never produces it). */
+double oracle_e8m0_to_f64(uint8_t e) {
+    if (e == 0xFF) return NAN;
+    return ldexp(1.0, (int)e - 127);
+}
+
 /* OCP e4m3fn code -> double.  Sign bit, 4 exponent bits (bias 7), 3 mantissa
  * bits; exponent 0 is subnormal (2^-6 * m/8); S.1111.111 is NaN (returned as
  * NaN; the generator never produces it). */
@@ -74,7 +86,7 @@ double oracle_e4m3_to_f64(uint8_t c) {
 
 typedef struct {
     int32_t B, T, H_I, D_I, K;
-    int32_t key_fp8;                 /* 0: bf16 keys, 1: e4m3 codes + scales */
+    int32_t key_fp8;                 /* 0: bf16 keys, 1: e4m3 codes + fp32 scales, 2: MXFP8 */
     const int32_t* seq_lens;         /* [B] */
     const int32_t* cu_q;             /* [B+1] */
     const int32_t* block_table;      /* [B, max_blocks] */
@@ -82,7 +94,9 @@ typedef struct {
     const uint16_t* q_idx;           /* [T, H_I, D_I] bf16 bits */
     const float* w;                  /* [T, H_I] */
     const void* k_idx;               /* [nblk, 64, D_I] bf16 bits or u8 codes */
-    const float* k_scale;            /* [nblk, 64, D_I/64] or NULL */
+    const float* k_scale;            /* [nblk, 64, D_I/64] fp32, [nblk, 64, D_I/32] u8 (MXFP8) or NULL */
+    int32_t q_mx;                    /* 1: q_idx holds e4m3 codes [T, H_I, D_I] (MXFP8 queries) */
+    const uint8_t* q_scale;          /* [T, H_I, D_I/32] shared scales of MXFP8 queries, or NULL */
 } oracle_indexer_args;
 
 /* Sequence and absolute position of query token t. */
@@ -105,11 +119,26 @@ static double key_elem(const oracle_indexer_args* a, int64_t row, int d) {
     if (!a->key_fp8) {
         const uint16_t* k = (const uint16_t*)a->k_idx;
         return bf16_to_f64(k[row * a->D_I + d]);
+    } else if (a->key_fp8 == 2) {
+        /* MXFP8: the code times the shared scale of its 32-element group */
+        const uint8_t* k = (const uint8_t*)a->k_idx;
+        const uint8_t* e = (const uint8_t*)a->k_scale;
+        return oracle_e4m3_to_f64(k[row * a->D_I + d]) * oracle_e8m0_to_f64(e[row * (a->D_I / 32) + d / 32]);
     } else {
         const uint8_t* k = (const uint8_t*)a->k_idx;
         double sc = (double)a->k_scale[row * (a->D_I / 64) + d / 64];
         return oracle_e4m3_to_f64(k[row * a->D_I + d]) * sc;
     }
+}
+
+/* Query element d of head h of token t, as a double: bf16 bits, or (MXFP8
+ * queries) the code times the shared scale of its 32-element group. */
+static double query_elem(const oracle_indexer_args* a, int t, int h, int d) {
+    int64_t i = ((int64_t)t * a->H_I + h) * a->D_I + d;
+    if (!a->q_mx) return bf16_to_f64(a->q_idx[i]);
+    const uint8_t* qc = (const uint8_t*)a->q_idx;
+    return oracle_e4m3_to_f64(qc[i]) *
+           oracle_e8m0_to_f64(a->q_scale[((int64_t)t * a->H_I + h) * (a->D_I / 32) + d / 32]);
 }
 
 /* Step 1 for one token: scores of positions 0..pos into out[0..pos]. */
@@ -120,7 +149,8 @@ static void score_token(const oracle_indexer_args* a, int t, double* out, int64_
     int H = a->H_I, D = a->D_I;
     double* q = (double*)malloc(sizeof(double) * (size_t)H * D);
     double* k = (double*)malloc(sizeof(double) * (size_t)D);
-    for (int i = 0; i < H * D; i++) q[i] = bf16_to_f64(a->q_idx[(int64_t)t * H * D + i]);
+    for (int h = 0; h < H; h++)
+        for (int d = 0; d < D; d++) q[h * D + d] = query_elem(a, t, h, d);
     for (int64_t s = 0; s <= pos; s++) {
         int64_t row = phys_row(a, b, s);
         for (int d = 0; d < D; d++) k[d] = key_elem(a, row, d);
@@ -213,7 +243,7 @@ int oracle_indexer_score_pairs(const oracle_indexer_args* a, const int32_t* toke
         for (int h = 0; h < a->H_I; h++) {
             double dot = 0.0;
             for (int d = 0; d < a->D_I; d++)
-                dot += bf16_to_f64(a->q_idx[((int64_t)t * a->H_I + h) * a->D_I + d]) * key_elem(a, row, d);
+                dot += query_elem(a, t, h, d) * key_elem(a, row, d);
             acc += (double)a->w[(int64_t)t * a->H_I + h] * (dot > 0.0 ? dot : 0.0);
         }
         out[i] = acc;

@@ -4,7 +4,8 @@
 * special cases that reduce to library routines: with one head and w=1 the
   indexer is ReLU(q.k) ranked by numpy.lexsort; with K >= context the sparse
   attention is dense causal softmax attention computed by torch in float64;
-* the e4m3 decode of all 256 codes against torch.float8_e4m3fn;
+* the e4m3 decode of all 256 codes against torch.float8_e4m3fn, and the MX
+  shared-scale decode of all 255 exponents against torch.float8_e8m0fnu;
 * invariants: page permutation, positive rescaling of w, convex outputs,
   a dominant logit;
 * the planted million-token workload: its Top-K must be the planted set;
@@ -26,9 +27,12 @@ GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_ca
 
 
 def manual_workload(q_idx_f, w, keys_f, *, K, key_dtype="bf16", k_codes=None, k_scale=None,
-                    q_mla=None, kv=None, H=1, sm_scale=1.0):
-    """One sequence, one query token at the last position; identity paging."""
-    q_idx_f = np.asarray(q_idx_f, np.float32)
+                    q_mla=None, kv=None, H=1, sm_scale=1.0, q_codes=None, q_scale=None):
+    """One sequence, one query token at the last position; identity paging.
+    MXFP8 (key_dtype "mxfp8"): q_codes [H_I, D_I] / q_scale [H_I, D_I/32] and
+    k_codes [L, D_I] / k_scale [L, D_I/32] are given as codes and scale bytes."""
+    mx = key_dtype == "mxfp8"
+    q_idx_f = np.asarray(q_idx_f if not mx else np.zeros(np.shape(q_codes)), np.float32)
     H_I, D_I = q_idx_f.shape
     L = len(keys_f) if keys_f is not None else k_codes.shape[0]
     nblk = (L + W.BLOCK - 1) // W.BLOCK
@@ -38,6 +42,13 @@ def manual_workload(q_idx_f, w, keys_f, *, K, key_dtype="bf16", k_codes=None, k_
         kk[:L] = np.asarray(keys_f, np.float32)
         k_idx = W.to_bf16_bits(kk).reshape(nblk, W.BLOCK, D_I)
         ks = None
+    elif mx:
+        cc = np.zeros((rows, D_I), np.uint8)
+        cc[:L] = k_codes
+        k_idx = cc.reshape(nblk, W.BLOCK, D_I)
+        ss = np.full((rows, D_I // 32), 127, np.uint8)
+        ss[:L] = k_scale
+        ks = ss.reshape(nblk, W.BLOCK, D_I // 32)
     else:
         cc = np.zeros((rows, D_I), np.uint8)
         cc[:L] = k_codes
@@ -51,8 +62,9 @@ def manual_workload(q_idx_f, w, keys_f, *, K, key_dtype="bf16", k_codes=None, k_
     return W.Workload(name="manual", B=1, T=1, H_I=H_I, D_I=D_I, H=H, K=K, key_dtype=key_dtype,
                       seq_lens=np.array([L], np.int32), cu_q=np.array([0, 1], np.int32),
                       block_table=np.arange(nblk, dtype=np.int32)[None, :], num_blocks=nblk,
-                      q_idx=W.to_bf16_bits(q_idx_f)[None], w=np.asarray(w, np.float32)[None],
-                      k_idx=k_idx, k_scale=ks, q=q_mla, kv=kv, sm_scale=sm_scale)
+                      q_idx=(np.asarray(q_codes, np.uint8) if mx else W.to_bf16_bits(q_idx_f))[None],
+                      w=np.asarray(w, np.float32)[None], k_idx=k_idx, k_scale=ks, q=q_mla, kv=kv,
+                      sm_scale=sm_scale, q_scale=np.asarray(q_scale, np.uint8)[None] if mx else None)
 
 
 # ----------------------------------------------------------------------------- hand cases
@@ -78,6 +90,85 @@ def test_hand_fp8_scale_groups():
                          k_scale=np.array([g["scales"]], np.float32))
     r = oracle.indexer_topk(wl, want_all_scores=True)
     assert r["all"][0, 0] == g["score"]
+
+
+def _mx_hand_workload():
+    g = GOLD["mxfp8_groups"]
+
+    def codes(spec, n):
+        c = np.zeros(n, np.uint8)
+        for k, v in spec.items():
+            c[int(k)] = v
+        return c
+    qc = codes(g["q_codes"], 64)[None]
+    kc = np.stack([codes(g["k0_codes"], 64), codes(g["k1_codes"], 64)])
+    ks = np.array([g["k0_scale"], g["k1_scale"]], np.uint8)
+    return g, manual_workload(None, [1.0], None, K=1, key_dtype="mxfp8", k_codes=kc, k_scale=ks,
+                              q_codes=qc, q_scale=np.array([g["q_scale"]], np.uint8))
+
+
+def test_hand_mxfp8_groups():
+    g, wl = _mx_hand_workload()
+    r = oracle.indexer_topk(wl, want_all_scores=True)
+    np.testing.assert_array_equal(r["all"][0, :2], np.array(g["scores"]))
+    assert r["idx"][0, 0] == 0
+    np.testing.assert_array_equal(oracle.score_pairs(wl, np.zeros(2, np.int32), np.array([0, 1])),
+                                  np.array(g["scores"]))
+
+
+def test_e8m0_decode_all_exponents_vs_torch():
+    e = np.arange(255, dtype=np.uint8)
+    ref = torch.from_numpy(e).view(torch.float8_e8m0fnu).to(torch.float32).numpy().astype(np.float64)
+    got = np.array([oracle.e8m0_to_f64(int(x)) for x in e])
+    np.testing.assert_array_equal(got, ref)
+    np.testing.assert_array_equal(got, np.ldexp(1.0, e.astype(np.int64) - 127))
+    assert math.isnan(oracle.e8m0_to_f64(255))
+
+
+def test_mx_encoding_follows_the_shared_scale_rule():
+    # the generator's MXFP8 encoding, decoded by the oracle: the shared exponent is
+    # floor(log2 amax) - 8 of its 32-element group, every element is the nearest e4m3
+    # value of x / 2^e (saturated at 448), so the error is within half an e4m3 step
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal((40, 128)) * np.exp(rng.uniform(-6, 6, size=(40, 1)))).astype(np.float32)
+    x[3, 32:64] = 0.0
+    codes, ex = W._quantize_mx(x)
+    dec = np.vectorize(oracle.e4m3_to_f64)(codes) * np.repeat(
+        np.vectorize(oracle.e8m0_to_f64)(ex), 32, axis=-1)
+    g = x.reshape(40, 4, 32).astype(np.float64)
+    amax = np.abs(g).max(-1)
+    mant, e2 = np.frexp(np.where(amax > 0, amax, 1.0))          # amax = mant * 2^e2, mant in [0.5, 1)
+    want_e = np.where(amax > 0, e2 - 1 - 8, 0) + 127
+    np.testing.assert_array_equal(ex.astype(np.int64), want_e)
+    scale = np.repeat(np.ldexp(1.0, want_e - 127), 32, axis=-1)
+    y = x.astype(np.float64) / scale                              # in units of the shared scale
+    sat = np.abs(y) > 448
+    step = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(y), 2.0 ** -6))).astype(np.int64) - 3)
+    err = np.abs(dec / scale - np.clip(y, -448, 448))
+    assert np.all(err[~sat] <= step[~sat] / 2 + 1e-12)
+    assert np.all(np.abs(dec[sat] / scale[sat]) == 448.0)
+    assert np.all(dec[3, 32:64] == 0.0)
+
+
+def test_mxfp8_integer_inputs_scores_are_exact():
+    # integers in [-4, 4] are encoded exactly (shared scale 2^-6, codes up to 256)
+    wl = W.make_workload("mxint", seq_lens=[300, 130], nq=[1, 2], H_I=8, D_I=64, H=1, K=64, key_dtype="mxfp8",
+                         int_inputs=True, w_dist="u256", seed=31, with_kv=False)
+    r = oracle.indexer_topk(wl, want_all_scores=True)
+    qd = np.vectorize(oracle.e4m3_to_f64)(wl.q_idx) * np.repeat(np.vectorize(oracle.e8m0_to_f64)(wl.q_scale), 32, -1)
+    kd = np.vectorize(oracle.e4m3_to_f64)(wl.k_idx) * np.repeat(np.vectorize(oracle.e8m0_to_f64)(wl.k_scale), 32, -1)
+    assert np.all(qd == np.round(qd)) and np.all(np.abs(qd) <= 4) and np.all(kd == np.round(kd))
+    qi = qd.astype(np.int64)
+    kflat = kd.reshape(-1, wl.D_I).astype(np.int64)
+    w256 = np.round(wl.w.astype(np.float64) * 256).astype(np.int64)
+    pos = wl.token_pos()
+    seq = wl.token_seq()
+    for t in range(wl.T):
+        rows = wl.block_table[seq[t], np.arange(pos[t] + 1) // W.BLOCK].astype(np.int64) * W.BLOCK + \
+            np.arange(pos[t] + 1) % W.BLOCK
+        dots = kflat[rows] @ qi[t].T                                  # [positions, heads] exact
+        want = (np.maximum(dots, 0) * w256[t][None, :]).sum(1) / 256.0
+        np.testing.assert_array_equal(r["all"][t, :pos[t] + 1], want)
 
 
 def test_hand_softmax_two_rows():

@@ -38,13 +38,19 @@ MUTANTS = [
      "if (s < 0 || s >= pos) { out[i] = NAN; continue; }"),
     ("softmax_value_from_rope", "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d]);",
      "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d + 64]);"),
+    ("mx_key_group_of_64", "oracle_e8m0_to_f64(e[row * (a->D_I / 32) + d / 32]);",
+     "oracle_e8m0_to_f64(e[row * (a->D_I / 32) + d / 64]);"),
+    ("mx_query_group_of_64", "oracle_e8m0_to_f64(a->q_scale[((int64_t)t * a->H_I + h) * (a->D_I / 32) + d / 32]);",
+     "oracle_e8m0_to_f64(a->q_scale[((int64_t)t * a->H_I + h) * (a->D_I / 32) + d / 64]);"),
+    ("e8m0_bias_126", "return ldexp(1.0, (int)e - 127);", "return ldexp(1.0, (int)e - 126);"),
 ]
 
 PINS = [pins.test_hand_indexer_relu_gate_weights_and_tie, pins.test_hand_fp8_scale_groups,
         pins.test_hand_score_pairs, lambda: pins.test_score_pairs_match_full_score_rows(dict(key_dtype="bf16")),
         pins.test_hand_softmax_two_rows, pins.test_e4m3_decode_all_codes_vs_torch,
         pins.test_single_head_unit_weight_is_relu_dot_lexsort,
-        pins.test_k_at_least_context_equals_dense_causal_attention]
+        pins.test_k_at_least_context_equals_dense_causal_attention, pins.test_hand_mxfp8_groups,
+        pins.test_e8m0_decode_all_exponents_vs_torch]
 
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
