@@ -209,10 +209,10 @@ def measure(dsa, W, wl, dev, steps, warmup, graph=True):
 
     def fused():
         dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], wl.K, wl.sm_scale,
-                       k_scale=d["k_scale"], out_idx=out_idx, out=out, workspace=ws)
+                       k_scale=d["k_scale"], q_scale=d["q_scale"], out_idx=out_idx, out=out, workspace=ws)
 
     def indexer():
-        dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], wl.K, k_scale=d["k_scale"], out_idx=out_idx,
+        dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], wl.K, k_scale=d["k_scale"], q_scale=d["q_scale"], out_idx=out_idx,
                          want_score=False, workspace=ws)
 
     def attention():
@@ -361,7 +361,7 @@ def run_ours(args, rank, world, local_rank):
         for k, v in host_in.items():
             d[k].copy_(v, non_blocking=True)
         dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], K, wl.sm_scale,
-                       k_scale=d["k_scale"], out_idx=out_idx, out=out, workspace=ws)
+                       k_scale=d["k_scale"], q_scale=d["q_scale"], out_idx=out_idx, out=out, workspace=ws)
         host_out.copy_(out, non_blocking=True)
         host_idx.copy_(out_idx, non_blocking=True)
 
@@ -386,7 +386,7 @@ def run_ours(args, rank, world, local_rank):
     sampler.stop()
 
     launches = dsa.decode_launch_count(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], K, wl.sm_scale,
-                                       k_scale=d["k_scale"])
+                                       k_scale=d["k_scale"], q_scale=d["q_scale"])
     peak, peak_kind = peaks()
     # ------------------------------------------------------------ the other workloads (one GPU): fused step,
     # each kernel, roofline fractions; fewer steps (each input set is generated on the host first)
@@ -394,7 +394,7 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_extra_workloads:
         del r, d, out, out_idx
         torch.cuda.empty_cache()
-        for name in ("tiny", "ragged", "1m", "prefill16k"):
+        for name in ("tiny", "ragged", "1m", "prefill16k", "batch32_mxfp8"):
             if name == args.workload:
                 continue
             xw = W.preset(name)

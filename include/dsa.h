@@ -70,9 +70,21 @@ typedef enum {
 
 typedef enum {
     DSA_KEY_BF16 = 0,           /* indexer keys: bf16 [num_blocks, 64, D_I]                       */
-    DSA_KEY_FP8_E4M3 = 1        /* indexer keys: e4m3fn codes [num_blocks, 64, D_I] (uint8) plus  */
+    DSA_KEY_FP8_E4M3 = 1,       /* indexer keys: e4m3fn codes [num_blocks, 64, D_I] (uint8) plus  */
                                 /* fp32 scales [num_blocks, 64, D_I/64], one per 64 elements      */
+    DSA_KEY_MXFP8 = 2           /* indexer keys in MXFP8: e4m3fn codes [num_blocks, 64, D_I]      */
+                                /* (uint8) plus one shared scale per 32 elements, [num_blocks,   */
+                                /* 64, D_I/32] uint8 exponents e (scale 2^(e-127)); needs MXFP8   */
+                                /* queries.  "Day0 Adaptation and Performance Optimization for   */
+                                /* Novel Long-Sequence Reasoning Models", section 4: full MXFP8   */
+                                /* quantization of index Q/K, every 32 elements share a scale.   */
 } dsa_key_dtype;
+
+typedef enum {
+    DSA_Q_BF16 = 0,             /* indexer queries: bf16 [T, H_I, D_I]                             */
+    DSA_Q_MXFP8 = 1             /* indexer queries in MXFP8: e4m3fn codes [T, H_I, D_I] (uint8) in */
+                                /* q_idx plus q_scale [T, H_I, D_I/32] uint8 exponents            */
+} dsa_query_dtype;
 
 /* Batch and paging description shared by all entry points. */
 typedef struct {
@@ -89,14 +101,18 @@ typedef struct {
 
 /* Indexer inputs (Lightning Indexer + Top-K). */
 typedef struct {
-    const void* q_idx;          /* device [T, H_I, D_I] bf16                                   */
+    const void* q_idx;          /* device [T, H_I, D_I] bf16 (or e4m3 codes, see q_dtype)      */
     const float* w;             /* device [T, H_I] fp32 head weights (any sign)                */
     const void* k_cache;        /* device indexer-key cache, layout per key_dtype              */
-    const float* k_scale;       /* device [num_blocks, 64, D_I/64] (fp8 keys), NULL for bf16   */
+    const float* k_scale;       /* device key scales: [num_blocks, 64, D_I/64] fp32 (fp8 keys, */
+                                /* 4-byte aligned) or [num_blocks, 64, D_I/32] uint8 exponents */
+                                /* (MXFP8 keys, 16-byte aligned); NULL for bf16 keys           */
     int32_t key_dtype;          /* dsa_key_dtype                                               */
     int32_t H_I;                /* indexer heads: 8, 16, 32 or 64                              */
     int32_t D_I;                /* indexer dim: 64 or 128                                      */
     int32_t K;                  /* Top-K, 1..2048                                              */
+    int32_t q_dtype;            /* dsa_query_dtype (MXFP8 exactly when key_dtype is MXFP8)     */
+    const uint8_t* q_scale;     /* device [T, H_I, D_I/32] exponents of MXFP8 queries, or NULL */
 } dsa_indexer_inputs;
 
 /* Sparse MLA attention inputs. */

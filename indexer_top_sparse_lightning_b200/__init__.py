@@ -8,10 +8,15 @@ passes raw device pointers plus the current CUDA stream.  There is no
 fallback: if the library is missing, importing the entry points raises.
 
 Entry points (same names as the C ABI):
-    indexer_topk(batch, q_idx, w, k_cache, K, k_scale=None) -> (idx, score)
+    indexer_topk(batch, q_idx, w, k_cache, K, k_scale=None, q_scale=None) -> (idx, score)
     sparse_mla_attn(batch, q, kv_cache, idx, sm_scale) -> (out, lse)
-    dsa_decode(batch, q_idx, w, k_cache, q, kv_cache, K, sm_scale, k_scale=None)
+    dsa_decode(batch, q_idx, w, k_cache, q, kv_cache, K, sm_scale, k_scale=None, q_scale=None)
         -> (idx, score, out, lse)
+
+Key formats: bf16 keys (k_scale None); e4m3 keys (uint8) with fp32 k_scale
+[nblk, 64, D_I/64]; MXFP8 queries and keys when q_scale is given: q_idx and
+k_cache hold e4m3 codes (uint8), q_scale [T, H_I, D_I/32] and k_scale
+[nblk, 64, D_I/32] hold uint8 exponents (one power-of-two scale per 32 elements).
 """
 from __future__ import annotations
 
@@ -29,6 +34,9 @@ _lib = None
 
 KEY_BF16 = 0
 KEY_FP8_E4M3 = 1
+KEY_MXFP8 = 2
+Q_BF16 = 0
+Q_MXFP8 = 1
 
 
 DSA_ERR_CUDA = 4   # dsa_status code of a failed CUDA runtime / driver call
@@ -53,7 +61,8 @@ class _Batch(ctypes.Structure):
 class _Indexer(ctypes.Structure):
     _fields_ = [("q_idx", ctypes.c_void_p), ("w", ctypes.c_void_p), ("k_cache", ctypes.c_void_p),
                 ("k_scale", ctypes.c_void_p), ("key_dtype", ctypes.c_int32), ("H_I", ctypes.c_int32),
-                ("D_I", ctypes.c_int32), ("K", ctypes.c_int32)]
+                ("D_I", ctypes.c_int32), ("K", ctypes.c_int32), ("q_dtype", ctypes.c_int32),
+                ("q_scale", ctypes.c_void_p)]
 
 
 class _Attn(ctypes.Structure):
@@ -170,19 +179,32 @@ class Batch:
                       int(self.block_table.shape[1]), self.num_blocks, self.max_seq_len, self.max_q_per_seq)
 
 
-def _indexer_struct(q_idx, w, k_cache, k_scale, K):
+def _indexer_struct(q_idx, w, k_cache, k_scale, K, q_scale=None):
     import torch
-    _check(q_idx, "q_idx", torch.bfloat16, 3)
-    T, H_I, D_I = q_idx.shape
-    _check(w, "w", torch.float32, 2, (T, H_I))
-    if k_scale is None:
-        _check(k_cache, "k_cache", torch.bfloat16, 3, (None, 64, D_I))
-        dt = KEY_BF16
-    else:
+    if q_scale is not None:
+        # MXFP8 queries and keys
+        _check(q_idx, "q_idx", torch.uint8, 3)
+        T, H_I, D_I = q_idx.shape
+        _check(q_scale, "q_scale", torch.uint8, 3, (T, H_I, D_I // 32))
         _check(k_cache, "k_cache", torch.uint8, 3, (None, 64, D_I))
-        _check(k_scale, "k_scale", torch.float32, 3, (k_cache.shape[0], 64, D_I // 64))
-        dt = KEY_FP8_E4M3
-    return _Indexer(_ptr(q_idx), _ptr(w), _ptr(k_cache), _ptr(k_scale), dt, H_I, D_I, int(K)), T
+        if k_scale is None:
+            raise ValueError("MXFP8 queries need MXFP8 keys (k_scale)")
+        _check(k_scale, "k_scale", torch.uint8, 3, (k_cache.shape[0], 64, D_I // 32))
+        dt, qt = KEY_MXFP8, Q_MXFP8
+    else:
+        _check(q_idx, "q_idx", torch.bfloat16, 3)
+        T, H_I, D_I = q_idx.shape
+        qt = Q_BF16
+        if k_scale is None:
+            _check(k_cache, "k_cache", torch.bfloat16, 3, (None, 64, D_I))
+            dt = KEY_BF16
+        else:
+            _check(k_cache, "k_cache", torch.uint8, 3, (None, 64, D_I))
+            _check(k_scale, "k_scale", torch.float32, 3, (k_cache.shape[0], 64, D_I // 64))
+            dt = KEY_FP8_E4M3
+    _check(w, "w", torch.float32, 2, (T, H_I))
+    return _Indexer(_ptr(q_idx), _ptr(w), _ptr(k_cache), _ptr(k_scale), dt, H_I, D_I, int(K), qt,
+                    _ptr(q_scale)), T
 
 
 def _attn_struct(q, kv_cache, sm_scale):
@@ -226,12 +248,12 @@ def _workspace(ws, device):
     return _default_ws[key]
 
 
-def indexer_topk(batch: Batch, q_idx, w, k_cache, K: int, k_scale=None, *, out_idx=None, out_score=None,
+def indexer_topk(batch: Batch, q_idx, w, k_cache, K: int, k_scale=None, q_scale=None, *, out_idx=None, out_score=None,
                  want_score: bool = True, workspace: Optional[Workspace] = None, stream=None):
     """Fused Lightning Indexer + Top-K.  Returns (idx [T,K] int32, score [T,K] fp32 or None)."""
     import torch
     lib = load_library()
-    ix, T = _indexer_struct(q_idx, w, k_cache, k_scale, K)
+    ix, T = _indexer_struct(q_idx, w, k_cache, k_scale, K, q_scale)
     cb = batch.c(T)
     if out_idx is None:
         out_idx = torch.empty((T, K), dtype=torch.int32, device=q_idx.device)
@@ -295,14 +317,14 @@ def sparse_mla_attn_static(batch: Batch, q, kv_cache, idx, sm_scale: float, *, o
     return out, lse
 
 
-def dsa_decode(batch: Batch, q_idx, w, k_cache, q, kv_cache, K: int, sm_scale: float, k_scale=None, *,
+def dsa_decode(batch: Batch, q_idx, w, k_cache, q, kv_cache, K: int, sm_scale: float, k_scale=None, q_scale=None, *,
                out_idx=None, out_score=None, out=None, lse=None, want_score=False, want_lse=False,
                workspace: Optional[Workspace] = None, stream=None):
     """Whole step (indexer + Top-K + sparse attention) on one stream.
     Returns (idx, score or None, out, lse or None)."""
     import torch
     lib = load_library()
-    ix, T = _indexer_struct(q_idx, w, k_cache, k_scale, K)
+    ix, T = _indexer_struct(q_idx, w, k_cache, k_scale, K, q_scale)
     at, T2 = _attn_struct(q, kv_cache, sm_scale)
     if T2 != T:
         raise ValueError("q_idx and q disagree on the number of tokens")
@@ -329,10 +351,10 @@ def dsa_decode(batch: Batch, q_idx, w, k_cache, q, kv_cache, K: int, sm_scale: f
 
 
 def decode_launch_count(batch: Batch, q_idx, w, k_cache, q, kv_cache, K: int, sm_scale: float,
-                        k_scale=None) -> int:
+                        k_scale=None, q_scale=None) -> int:
     """Kernel launches one dsa_decode call enqueues for these shapes."""
     lib = load_library()
-    ix, T = _indexer_struct(q_idx, w, k_cache, k_scale, K)
+    ix, T = _indexer_struct(q_idx, w, k_cache, k_scale, K, q_scale)
     at, _ = _attn_struct(q, kv_cache, sm_scale)
     cb = batch.c(T)
     n = lib.dsa_decode_launch_count(ctypes.byref(cb), ctypes.byref(ix), ctypes.byref(at))

@@ -43,13 +43,20 @@ dsa_status check_batch(const dsa_batch* bt) {
 
 dsa_status check_indexer(const dsa_indexer_inputs* ix) {
     if (!ix || !ix->q_idx || !ix->w || !ix->k_cache) return DSA_ERR_INVALID_ARG;
-    if (ix->key_dtype != DSA_KEY_BF16 && ix->key_dtype != DSA_KEY_FP8_E4M3) return DSA_ERR_INVALID_ARG;
-    if (ix->key_dtype == DSA_KEY_FP8_E4M3 && !ix->k_scale) return DSA_ERR_INVALID_ARG;
+    if (ix->key_dtype != DSA_KEY_BF16 && ix->key_dtype != DSA_KEY_FP8_E4M3 && ix->key_dtype != DSA_KEY_MXFP8)
+        return DSA_ERR_INVALID_ARG;
+    if (ix->key_dtype != DSA_KEY_BF16 && !ix->k_scale) return DSA_ERR_INVALID_ARG;
+    if (ix->q_dtype != DSA_Q_BF16 && ix->q_dtype != DSA_Q_MXFP8) return DSA_ERR_INVALID_ARG;
+    // MXFP8 queries and MXFP8 keys go together (the indexer's Q and K are both quantized)
+    if ((ix->q_dtype == DSA_Q_MXFP8) != (ix->key_dtype == DSA_KEY_MXFP8)) return DSA_ERR_INVALID_ARG;
+    if (ix->q_dtype == DSA_Q_MXFP8 && !ix->q_scale) return DSA_ERR_INVALID_ARG;
+    // MXFP8 key scales arrive by 16-byte aligned bulk copies, one per page
+    if (ix->key_dtype == DSA_KEY_MXFP8 && !aligned16(ix->k_scale)) return DSA_ERR_INVALID_ARG;
     if (ix->H_I != 8 && ix->H_I != 16 && ix->H_I != 32 && ix->H_I != 64) return DSA_ERR_UNSUPPORTED;
     if (ix->D_I != 64 && ix->D_I != 128) return DSA_ERR_UNSUPPORTED;
     if (ix->K < 1 || ix->K > kMaxTopK) return DSA_ERR_UNSUPPORTED;
     if (!aligned16(ix->q_idx) || !aligned16(ix->k_cache)) return DSA_ERR_INVALID_ARG;
-    if (ix->k_scale && (reinterpret_cast<uintptr_t>(ix->k_scale) & 3u)) return DSA_ERR_INVALID_ARG;
+    if (ix->key_dtype == DSA_KEY_FP8_E4M3 && (reinterpret_cast<uintptr_t>(ix->k_scale) & 3u)) return DSA_ERR_INVALID_ARG;
     return DSA_OK;
 }
 
@@ -64,9 +71,9 @@ dsa_status check_attn(const dsa_attn_inputs* at) {
 
 // ------------------------------------------------------------------ indexer planning
 // Fill the fields that depend on the kernel instantiation.
-template <bool FP8, int HI, int DI, int NQ>
+template <bool FP8, int HI, int DI, int NQ, bool MX>
 bool plan_for(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl) {
-    using Cfg = IdxCfg<FP8, HI, DI, NQ>;
+    using Cfg = IdxCfg<FP8, HI, DI, NQ, MX>;
     const int cap = (di.max_smem - Cfg::FIXED_SMEM) / 4;
     if (cap < kTileKeys * NQ) return false;
     pl.score_cap = (cap / (kTileKeys * NQ)) * (kTileKeys * NQ);
@@ -99,32 +106,32 @@ bool plan_for(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl) {
     return true;
 }
 
-template <bool FP8, int HI, int DI, int NQ>
+template <bool FP8, int HI, int DI, int NQ, bool MX>
 bool select_impl(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl, LaunchFn& fn) {
-    if (!plan_for<FP8, HI, DI, NQ>(bt, di, pl)) return false;
-    fn = &launch_indexer<FP8, HI, DI, NQ>;
+    if (!plan_for<FP8, HI, DI, NQ, MX>(bt, di, pl)) return false;
+    fn = &launch_indexer<FP8, HI, DI, NQ, MX>;
     return true;
 }
 
-template <bool FP8, int HI, int DI>
+template <bool FP8, int HI, int DI, bool MX>
 bool select_nq(const dsa_batch* bt, const DevInfo& di, IdxPlan& pl, LaunchFn& fn) {
-    if (pl.nq == 1) return select_impl<FP8, HI, DI, 1>(bt, di, pl, fn);
-    return select_impl<FP8, HI, DI, 2>(bt, di, pl, fn);
+    if (pl.nq == 1) return select_impl<FP8, HI, DI, 1, MX>(bt, di, pl, fn);
+    return select_impl<FP8, HI, DI, 2, MX>(bt, di, pl, fn);
 }
 
-template <bool FP8, int HI>
+template <bool FP8, int HI, bool MX>
 bool select_di(int D_I, const dsa_batch* bt, const DevInfo& di, IdxPlan& pl, LaunchFn& fn) {
-    if (D_I == 64) return select_nq<FP8, HI, 64>(bt, di, pl, fn);
-    return select_nq<FP8, HI, 128>(bt, di, pl, fn);
+    if (D_I == 64) return select_nq<FP8, HI, 64, MX>(bt, di, pl, fn);
+    return select_nq<FP8, HI, 128, MX>(bt, di, pl, fn);
 }
 
-template <bool FP8>
+template <bool FP8, bool MX>
 bool select_hi(int H_I, int D_I, const dsa_batch* bt, const DevInfo& di, IdxPlan& pl, LaunchFn& fn) {
     switch (H_I) {
-        case 8: return select_di<FP8, 8>(D_I, bt, di, pl, fn);
-        case 16: return select_di<FP8, 16>(D_I, bt, di, pl, fn);
-        case 32: return select_di<FP8, 32>(D_I, bt, di, pl, fn);
-        default: return select_di<FP8, 64>(D_I, bt, di, pl, fn);
+        case 8: return select_di<FP8, 8, MX>(D_I, bt, di, pl, fn);
+        case 16: return select_di<FP8, 16, MX>(D_I, bt, di, pl, fn);
+        case 32: return select_di<FP8, 32, MX>(D_I, bt, di, pl, fn);
+        default: return select_di<FP8, 64, MX>(D_I, bt, di, pl, fn);
     }
 }
 
@@ -135,9 +142,12 @@ bool select_hi(int H_I, int D_I, const dsa_batch* bt, const DevInfo& di, IdxPlan
 dsa_status plan_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, const DevInfo& di, IdxPlan& pl,
                         LaunchFn& fn) {
     const int nq = bt->max_q_per_seq < bt->num_tokens ? bt->max_q_per_seq : bt->num_tokens;
-    const bool fp8 = ix->key_dtype == DSA_KEY_FP8_E4M3;
     auto select = [&]() {
-        return fp8 ? select_hi<true>(ix->H_I, ix->D_I, bt, di, pl, fn) : select_hi<false>(ix->H_I, ix->D_I, bt, di, pl, fn);
+        switch (ix->key_dtype) {
+            case DSA_KEY_FP8_E4M3: return select_hi<true, false>(ix->H_I, ix->D_I, bt, di, pl, fn);
+            case DSA_KEY_MXFP8: return select_hi<true, true>(ix->H_I, ix->D_I, bt, di, pl, fn);
+            default: return select_hi<false, false>(ix->H_I, ix->D_I, bt, di, pl, fn);
+        }
     };
     if (nq <= 2) {
         pl.mode = 0;

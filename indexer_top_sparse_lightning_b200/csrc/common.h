@@ -42,7 +42,10 @@ struct IndexerParams {
     const int32_t* cu_q;
     const int32_t* block_table;
     const float* w;
-    const float* k_scale;
+    const float* k_scale;     // fp8 keys: [nblk, 64, D_I/64] fp32
+    const uint8_t* k_scale_e8;  // MXFP8 keys: [nblk, 64, D_I/32] shared exponents (2^(e-127))
+    const uint8_t* q_codes;   // MXFP8 queries: [T, H_I, D_I] e4m3 codes
+    const uint8_t* q_scale;   // MXFP8 queries: [T, H_I, D_I/32] shared exponents
     int32_t* out_idx;
     float* out_score;
     uint32_t* status;

@@ -62,7 +62,7 @@ using LaunchFn = dsa_status (*)(const dsa_batch*, const dsa_indexer_inputs*, int
 
 // Launches of one indexer kernel variant (defined in idx_launch.cuh,
 // instantiated in the idx_*.cu units).
-template <bool FP8, int HI, int DI, int NQ>
+template <bool FP8, int HI, int DI, int NQ, bool MX = false>
 dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int32_t* out_idx, float* out_score,
                           uint32_t* status, uint8_t* group_ws, const IdxPlan& pl, cudaStream_t stream);
 

@@ -12,12 +12,20 @@
 namespace dsa {
 namespace host {
 
-template <bool FP8, int HI, int DI, int NQ>
+template <bool FP8, int HI, int DI, int NQ, bool MX>
 dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int32_t* out_idx, float* out_score,
                           uint32_t* status, uint8_t* group_ws, const IdxPlan& pl, cudaStream_t stream) {
-    using Cfg = IdxCfg<FP8, HI, DI, NQ>;
+    using Cfg = IdxCfg<FP8, HI, DI, NQ, MX>;
     CUtensorMap tm_q, tm_k;
-    {
+    if (MX) {
+        // MXFP8 queries are read by the epilogue threads; the map (over the codes) is
+        // passed but never used by a copy
+        const uint64_t dims[3] = {(uint64_t)DI, (uint64_t)HI, (uint64_t)bt->num_tokens};
+        const uint64_t strides[2] = {(uint64_t)DI, (uint64_t)HI * DI};
+        const uint32_t box[3] = {(uint32_t)DI, (uint32_t)HI, 1};
+        if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, ix->q_idx, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return fail(DSA_ERR_CUDA, "indexer query tensor map encoding failed");
+    } else {
         const uint64_t dims[3] = {(uint64_t)DI, (uint64_t)HI, (uint64_t)bt->num_tokens};
         const uint64_t strides[2] = {(uint64_t)DI * 2, (uint64_t)HI * DI * 2};
         const uint32_t box[3] = {64, (uint32_t)HI, (uint32_t)NQ};
@@ -41,7 +49,7 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
                 return fail(DSA_ERR_CUDA, "indexer key tensor map encoding failed");
         }
     }
-    auto kern = &indexer_topk_kernel<FP8, HI, DI, NQ>;
+    auto kern = &indexer_topk_kernel<FP8, HI, DI, NQ, MX>;
     if (cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(kern), pl.smem))
         return fail(DSA_ERR_CUDA, "indexer shared memory attribute", e);
 
@@ -51,7 +59,10 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_inputs* ix, int
     p.cu_q = bt->cu_q;
     p.block_table = bt->block_table;
     p.w = ix->w;
-    p.k_scale = ix->k_scale;
+    p.k_scale = MX ? nullptr : ix->k_scale;
+    p.k_scale_e8 = MX ? reinterpret_cast<const uint8_t*>(ix->k_scale) : nullptr;
+    p.q_codes = MX ? reinterpret_cast<const uint8_t*>(ix->q_idx) : nullptr;
+    p.q_scale = MX ? ix->q_scale : nullptr;
     p.out_idx = out_idx;
     p.out_score = out_score;
     p.status = status;

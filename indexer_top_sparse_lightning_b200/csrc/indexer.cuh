@@ -43,18 +43,26 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
     return p;
 }
 
-template <bool FP8, int HI, int DI, int NQ>
+// FP8: e4m3 key codes, widened to bf16 in shared memory.  MX (with FP8): MXFP8
+// queries and keys -- each code times the power-of-two scale of its 32-element
+// group, applied exactly while widening (queries: while building the Q tile), so
+// the contraction and one accumulator are those of bf16 keys.
+template <bool FP8, int HI, int DI, int NQ, bool MX = false>
 struct IdxCfg {
+    static_assert(!MX || FP8, "MXFP8 keys are e4m3 codes");
     static constexpr int KB = DI / 64;                        // 64-wide K blocks
     static constexpr int N = (NQ * HI < 16) ? 16 : NQ * HI;   // MMA N (token-major heads)
-    static constexpr int ACC = FP8 ? KB : 1;                  // fp8: one accumulator per scale group
+    static constexpr int ACC = (FP8 && !MX) ? KB : 1;         // fp8 with fp32 scales: one accumulator per scale group
     static constexpr int COLS_BUF = N * ACC;
     static constexpr int TMEM_COLS = pow2_at_least(2 * COLS_BUF);
     // key stages in flight: fp8 keys keep three (their widened copies take two more
     // buffers), so that a CTA holds 16 K scores and a 128 K-context batch of eight
     // plans into one grouped launch
     static constexpr int NSTAGE = FP8 ? 3 : (NQ == 1 ? 4 : 3);
-    static constexpr int STAGE_BYTES = kTileKeys * DI * (FP8 ? 1 : 2);
+    static constexpr int CODE_BYTES = kTileKeys * DI * (FP8 ? 1 : 2);   // one tile of keys
+    // MXFP8: the tile's scale bytes follow its codes in the stage ([128 keys][D_I/32])
+    static constexpr int KSC_BYTES = MX ? kTileKeys * (DI / 32) : 0;
+    static constexpr int STAGE_BYTES = ((CODE_BYTES + KSC_BYTES + 1023) / 1024) * 1024;
     static constexpr int NCONV = FP8 ? 2 : 0;                 // widened-operand buffers
     static constexpr int NCV = FP8 ? 2 : 1;                   // (modulus for the ring index)
     static constexpr int CONV_BYTES = kTileKeys * DI * 2;
@@ -250,11 +258,11 @@ static __device__ void assign_groups(const IndexerParams& p, IdxMisc* m, int nq_
     });
 }
 
-template <bool FP8, int HI, int DI, int NQ>
-__global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
+template <bool FP8, int HI, int DI, int NQ, bool MX = false>
+__global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ, MX>::THREADS, 1)
     indexer_topk_kernel(const __grid_constant__ IndexerParams p, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k) {
-    using Cfg = IdxCfg<FP8, HI, DI, NQ>;
+    using Cfg = IdxCfg<FP8, HI, DI, NQ, MX>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_shared(smem_raw, 1024);
     uint8_t* s_stage = smem + Cfg::OFF_STAGE;
@@ -281,7 +289,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             mbar_init(&m->tfull[i], 1);
             mbar_init(&m->tempty[i], kEpiThreads);
         }
-        mbar_init(&m->q_full, 1);
+        mbar_init(&m->q_full, MX ? kEpiThreads : 1);   // MXFP8: the epilogue threads build Q
         mbar_init(&m->q_empty, 1);
         mbar_init(&m->drain, 1);
         mbar_init(&m->gbar, 1);
@@ -300,7 +308,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
         tmem_relinquish();
     }
     if (warp == Cfg::PRODUCER_WARP && lane == 0) {
-        prefetch_tmap(&tm_q);
+        if (!MX) prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
     }
     if (Cfg::Q_PAD) {
@@ -346,11 +354,13 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
             __syncwarp();
             int ok = 1;
             if (lane == 0) {
-                if (!mbar_wait(&m->q_empty, (k & 1) ^ 1, abort, wlim)) ok = 0;
-                if (ok) {
-                    mbar_arrive_expect_tx(&m->q_full, Cfg::Q_TX);
-                    for (int kb = 0; kb < Cfg::KB; ++kb)
-                        tma_load_3d(s_q + kb * Cfg::N * 128, &tm_q, &m->q_full, kb * 64, 0, item.t0);
+                if (!MX) {
+                    if (!mbar_wait(&m->q_empty, (k & 1) ^ 1, abort, wlim)) ok = 0;
+                    if (ok) {
+                        mbar_arrive_expect_tx(&m->q_full, Cfg::Q_TX);
+                        for (int kb = 0; kb < Cfg::KB; ++kb)
+                            tma_load_3d(s_q + kb * Cfg::N * 128, &tm_q, &m->q_full, kb * 64, 0, item.t0);
+                    }
                 }
                 for (int li = 0; ok && li < item.tile_count; ++li, ++it) {
                     const int s = it % Cfg::NSTAGE;
@@ -363,11 +373,20 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         nvalid += i < npg;
                     }
                     uint8_t* st = s_stage + s * Cfg::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&m->full[s], nvalid * kPage * DI * (FP8 ? 1 : 2));
+                    // MXFP8: a page's 64 scale words come along by one bulk copy (none for an
+                    // out-of-range page, whose codes read as zeros)
+                    constexpr uint32_t PSC = kPage * (DI / 32);
+                    uint32_t sc_bytes = 0;
+                    if (MX)
+                        for (int pp = 0; pp < 2; ++pp) sc_bytes += blk[pp] >= 0 ? PSC : 0u;
+                    mbar_arrive_expect_tx(&m->full[s], nvalid * kPage * DI * (FP8 ? 1 : 2) + sc_bytes);
                     for (int pp = 0; pp < 2; ++pp) {
                         if (blk[pp] == -2) continue;
                         if (FP8) {
                             tma_load_2d_hint(st + pp * kPage * DI, &tm_k, &m->full[s], 0, blk[pp] * kPage, pol);
+                            if (MX && blk[pp] >= 0)
+                                bulk_load(st + Cfg::CODE_BYTES + pp * PSC, p.k_scale_e8 + (int64_t)blk[pp] * PSC, PSC,
+                                          &m->full[s]);
                         } else {
                             for (int kb = 0; kb < Cfg::KB; ++kb)
                                 tma_load_2d_hint(st + kb * (kTileKeys * 128) + pp * (kPage * 128), &tm_k,
@@ -417,8 +436,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         for (int k16 = 0; k16 < 4; ++k16) {
                             const uint64_t ad = sdesc_sw128(a_addr + kb * (kTileKeys * 128) + k16 * 32, 16, 1024);
                             const uint64_t bd = sdesc_sw128(b_addr + kb * (Cfg::N * 128) + k16 * 32, 16, 1024);
-                            const uint32_t d = tmem_base + buf * Cfg::COLS_BUF + (FP8 ? kb * Cfg::N : 0);
-                            const uint32_t acc = FP8 ? (k16 > 0) : (kb > 0 || k16 > 0);
+                            const uint32_t d = tmem_base + buf * Cfg::COLS_BUF + (Cfg::ACC > 1 ? kb * Cfg::N : 0);
+                            const uint32_t acc = Cfg::ACC > 1 ? (k16 > 0) : (kb > 0 || k16 > 0);
                             umma_bf16(d, ad, bd, Cfg::IDESC, acc);
                         }
                     }
@@ -435,6 +454,8 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
         }
     } else if (FP8 && warp >= Cfg::CONV_WARP0) {
         // ---------------------------------------------------------------- fp8 -> bf16 widening
+        // MXFP8 keys: each 16-code chunk lies in one 32-element group, whose power-of-two
+        // scale multiplies the codes exactly before the (exact) conversion to bf16.
         const int ct = threadIdx.x - Cfg::CONV_WARP0 * 32;
         uint32_t it = 0;
         IdxItem item;
@@ -452,6 +473,13 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 for (int u = ct; u < kTileKeys * CH; u += kConvThreads) {
                     const int r = u / CH, c = u % CH;
                     const uint4 v = *reinterpret_cast<const uint4*>(raw + r * DI + c * 16);
+                    float sc = 1.0f;
+                    if (MX) {
+                        // scale byte of group c/2 of key r (rows of a page past the sequence
+                        // hold whatever the stage held; their keys are never selected)
+                        const uint32_t e = raw[Cfg::CODE_BYTES + r * (DI / 32) + (c >> 1)];
+                        sc = e ? __uint_as_float(e << 23) : __uint_as_float(0x00400000u);   // 2^(e - 127)
+                    }
                     uint32_t outw[8];
                     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -459,8 +487,14 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                         uint32_t h01, h23;
                         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"((uint16_t)(in[e] & 0xFFFFu)));
                         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"((uint16_t)(in[e] >> 16)));
-                        const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-                        const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+                        float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+                        float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+                        if (MX) {
+                            f01.x *= sc;
+                            f01.y *= sc;
+                            f23.x *= sc;
+                            f23.y *= sc;
+                        }
                         const __nv_bfloat162 b01 = __float22bfloat162_rn(f01);
                         const __nv_bfloat162 b23 = __float22bfloat162_rn(f23);
                         outw[2 * e] = *reinterpret_cast<const uint32_t*>(&b01);
@@ -500,6 +534,47 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 m->sel.kmin[threadIdx.x] = 0xFFFFFFFFu;
                 m->sel.kmax[threadIdx.x] = 0u;
             }
+            if (MX) {
+                // MXFP8 queries: once the previous item's MMAs are done with Q, build the
+                // bf16 Q tile (128-byte swizzled, token-major heads) from the codes, each
+                // times the power-of-two scale of its 32-element group (exact)
+                if (mbar_wait(&m->q_empty, (k & 1) ^ 1, abort, wlim)) {
+                    constexpr int CPR = DI / 8;   // 16-byte bf16 units per head row
+                    for (int u = threadIdx.x; u < NQ * HI * CPR; u += kEpiThreads) {
+                        const int r = u / CPR, c = u % CPR;
+                        const int j = r / HI, h = r % HI;
+                        uint32_t outw[4] = {0u, 0u, 0u, 0u};
+                        if (j < item.nq) {
+                            const int64_t qi = (int64_t)(item.t0 + j) * HI + h;
+                            const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.q_codes + qi * DI + c * 8));
+                            const uint32_t e = __ldg(p.q_scale + qi * (DI / 32) + (c * 8) / 32);
+                            const float sc = e ? __uint_as_float(e << 23) : __uint_as_float(0x00400000u);
+                            const uint32_t in[2] = {v.x, v.y};
+#pragma unroll
+                            for (int e2 = 0; e2 < 2; ++e2) {
+                                uint32_t h01, h23;
+                                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"((uint16_t)(in[e2] & 0xFFFFu)));
+                                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"((uint16_t)(in[e2] >> 16)));
+                                float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+                                float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+                                f01.x *= sc;
+                                f01.y *= sc;
+                                f23.x *= sc;
+                                f23.y *= sc;
+                                const __nv_bfloat162 b01 = __float22bfloat162_rn(f01);
+                                const __nv_bfloat162 b23 = __float22bfloat162_rn(f23);
+                                outw[2 * e2] = *reinterpret_cast<const uint32_t*>(&b01);
+                                outw[2 * e2 + 1] = *reinterpret_cast<const uint32_t*>(&b23);
+                            }
+                        }
+                        // 64-element K block c/8, 16-byte unit c%8 of the row, swizzled by row
+                        *reinterpret_cast<uint4*>(s_q + (c >> 3) * (Cfg::N * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4)) =
+                            make_uint4(outw[0], outw[1], outw[2], outw[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&m->q_full);
+            }
             GroupView gv{nullptr, nullptr, nullptr, item.G, item.rank};
             uint32_t gen = 0;
             if (item.G > 1) {
@@ -525,7 +600,7 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                 const int buf = it & 1;
                 const int64_t pos = chunk0 + (int64_t)li * kTileKeys + row;
                 float sc[2] = {1.0f, 1.0f};
-                if (FP8 && scorer) {
+                if (FP8 && !MX && scorer) {     // fp32 group scales, applied to the accumulators
                     const int64_t pg = pos / kPage;
                     if (pg < npages) {
                         const int bid = __ldg(p.block_table + (int64_t)item.b * p.max_blocks + pg);
@@ -557,13 +632,13 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
                             const uint32_t col = j * HI + h0;
                             if constexpr (CW == 32) {
                                 tmem_ld32(tb + col, a0);
-                                if (FP8 && Cfg::KB > 1) tmem_ld32(tb + Cfg::N + col, a1);
+                                if (Cfg::ACC > 1) tmem_ld32(tb + Cfg::N + col, a1);
                             } else if constexpr (CW == 16) {
                                 tmem_ld16(tb + col, *reinterpret_cast<uint32_t(*)[16]>(a0));
-                                if (FP8 && Cfg::KB > 1) tmem_ld16(tb + Cfg::N + col, *reinterpret_cast<uint32_t(*)[16]>(a1));
+                                if (Cfg::ACC > 1) tmem_ld16(tb + Cfg::N + col, *reinterpret_cast<uint32_t(*)[16]>(a1));
                             } else {
                                 tmem_ld8(tb + col, *reinterpret_cast<uint32_t(*)[8]>(a0));
-                                if (FP8 && Cfg::KB > 1) tmem_ld8(tb + Cfg::N + col, *reinterpret_cast<uint32_t(*)[8]>(a1));
+                                if (Cfg::ACC > 1) tmem_ld8(tb + Cfg::N + col, *reinterpret_cast<uint32_t(*)[8]>(a1));
                             }
                             tmem_wait_ld();
                             const float4* w4 = reinterpret_cast<const float4*>(s_w + j * HI + h0);
@@ -574,9 +649,11 @@ __global__ void __launch_bounds__(IdxCfg<FP8, HI, DI, NQ>::THREADS, 1)
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
                                     float x = __uint_as_float(a0[h + e]);
-                                    if (FP8) {
+                                    if (Cfg::ACC > 1) {
                                         x = x * sc[0];
-                                        if (Cfg::KB > 1) x = fmaf(__uint_as_float(a1[h + e]), sc[1], x);
+                                        x = fmaf(__uint_as_float(a1[h + e]), sc[1], x);
+                                    } else if (FP8 && !MX) {
+                                        x = x * sc[0];
                                     }
                                     part[e] = fmaf(wq[e], fmaxf(x, 0.0f), part[e]);
                                 }

@@ -34,11 +34,11 @@ def main(argv=None) -> int:
     ev[0].record()
     for i in range(a.steps):
         if a.indexer_only:
-            dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], wl.K, k_scale=d["k_scale"], workspace=ws,
+            dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], wl.K, k_scale=d["k_scale"], q_scale=d["q_scale"], workspace=ws,
                              want_score=False)
         else:
             dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], wl.K, wl.sm_scale,
-                           k_scale=d["k_scale"], workspace=ws)
+                           k_scale=d["k_scale"], q_scale=d["q_scale"], workspace=ws)
         ev[i + 1].record()
     torch.cuda.synchronize()
     st = dsa.get_status(ws)

@@ -36,7 +36,7 @@ def device_batch(wl, d):
 def run_indexer(wl, d=None, want_score=True):
     d = d if d is not None else W.to_device(wl, with_kv=False)
     idx, score = dsa.indexer_topk(device_batch(wl, d), d["q_idx"], d["w"], d["k_cache"], wl.K,
-                                  k_scale=d["k_scale"], want_score=want_score)
+                                  k_scale=d["k_scale"], q_scale=d["q_scale"], want_score=want_score)
     torch.cuda.synchronize()
     st = dsa.get_status()
     assert st == 0, f"device status {st}: {dsa.status_str(st)}"

@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 def run_decode(wl, d=None):
     d = d if d is not None else W.to_device(wl)
     idx, score, out, lse = dsa.dsa_decode(device_batch(wl, d), d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"],
-                                          wl.K, wl.sm_scale, k_scale=d["k_scale"], want_score=True,
+                                          wl.K, wl.sm_scale, k_scale=d["k_scale"], q_scale=d["q_scale"], want_score=True,
                                           want_lse=True)
     torch.cuda.synchronize()
     assert dsa.get_status() == 0
@@ -31,6 +31,12 @@ def check(wl, tokens, exact):
 
 def test_tiny_decode():
     check(W.preset("tiny"), [0], exact=True)
+
+
+def test_mxfp8_decode():
+    wl = W.make_workload("mxdec", seq_lens=[3000, 9000], nq=[2, 1], H_I=64, D_I=128, H=128, K=1024,
+                         key_dtype="mxfp8", seed=44)
+    check(wl, np.arange(wl.T), exact=False)
 
 
 def test_small_mixed_decode():

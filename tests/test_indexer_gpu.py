@@ -187,6 +187,32 @@ def test_uneven_windows_integer_inputs_bit_exact():
     assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
 
 
+@pytest.mark.parametrize("seq_lens,nq", [([3000], 1), ([900, 5000, 64], [1, 2, 1]), ([40000, 7000], 1)])
+def test_mxfp8_integer_inputs_bit_exact(seq_lens, nq):
+    # MXFP8 queries and keys holding integers in [-4, 4] (encoded exactly): every score
+    # is exact, so the Top-K must equal the oracle's bit for bit, single CTA and grouped
+    wl = W.make_workload("mxint", seq_lens=seq_lens, nq=nq, H_I=8, D_I=64, H=1, K=256, key_dtype="mxfp8",
+                         int_inputs=True, w_dist="u256", seed=41, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=True)
+
+
+@pytest.mark.parametrize("H_I,D_I,nq", [(64, 128, 1), (64, 128, 2), (32, 64, 1), (16, 128, 2)])
+def test_mxfp8_queries_and_keys(H_I, D_I, nq):
+    wl = W.make_workload("mx", seq_lens=[12000, 700, 5000], nq=nq, H_I=H_I, D_I=D_I, H=1, K=1024,
+                         key_dtype="mxfp8", seed=42, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
+def test_mxfp8_long_chunk_windows():
+    # MXFP8 through the grouped query windows (three tokens per sequence, long context)
+    wl = W.make_workload("mxwin", seq_lens=[70000], nq=3, H_I=64, D_I=128, H=1, K=2048, key_dtype="mxfp8",
+                         seed=43, with_kv=False)
+    idx, score = run_indexer(wl)
+    assert_topk(wl, np.arange(wl.T), idx, score, exact=False)
+
+
 def test_score_output_is_optional():
     wl = W.preset("tiny", with_kv=False)
     idx, score = run_indexer(wl, want_score=False)
@@ -238,6 +264,14 @@ def test_ragged_fp8_full_size_sampled():
     wl = W.preset("ragged", with_kv=False)
     idx, score = run_indexer(wl)
     tok = np.arange(wl.T)
+    assert_topk(wl, tok, idx[tok], score[tok], exact=False)
+
+
+@pytest.mark.slow
+def test_batch32_mxfp8_full_size_sampled():
+    wl = W.preset("batch32_mxfp8", with_kv=False)
+    idx, score = run_indexer(wl)
+    tok = np.arange(0, wl.T, 3)
     assert_topk(wl, tok, idx[tok], score[tok], exact=False)
 
 
