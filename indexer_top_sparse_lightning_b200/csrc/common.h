@@ -13,7 +13,7 @@ constexpr int kDqk = 576;             // latent 512 + RoPE 64
 constexpr int kDv = 512;
 constexpr int kEpiWarps = 8;          // indexer epilogue / Top-K warps (two per TMEM lane quarter)
 constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kConvThreads = 128;     // fp8 key widening threads (four warps)
+constexpr int kConvThreads = 192;     // fp8 key widening threads (six warps)
 
 // Device status word values (mirrors dsa_status).
 enum : uint32_t {

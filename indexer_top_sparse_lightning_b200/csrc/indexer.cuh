@@ -71,7 +71,7 @@ struct IdxCfg {
     static constexpr bool Q_PAD = NQ * HI < N;                // rows [NQ*HI, N) stay zero
     static constexpr int HIST_WORDS = kBins;                  // select histograms
     static constexpr int W_FLOATS = NQ * HI;
-    // warps 0-7 epilogue and Top-K, 8 TMA producer, 9 MMA issuer, 10-13 fp8 widening
+    // warps 0-7 epilogue and Top-K, 8 TMA producer, 9 MMA issuer, 10-15 fp8 widening
     static constexpr int THREADS = kEpiThreads + 64 + (FP8 ? kConvThreads : 0);
     static constexpr int PRODUCER_WARP = kEpiWarps;
     static constexpr int MMA_WARP = kEpiWarps + 1;
