@@ -47,7 +47,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="batch32", choices=["batch32", "tiny", "prefill16k", "ragged", "1m"])
+    ap.add_argument("--workload", default="batch32", choices=["batch32", "tiny", "prefill16k", "ragged", "1m",
+                                                              "batch32_mxfp8"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-extra-workloads", action="store_true",
