@@ -337,6 +337,39 @@ def preset(name: str, with_kv: bool = True) -> Workload:
     return make_workload(name, with_kv=with_kv, **kw)
 
 
+@dataclasses.dataclass
+class ProlWork:
+    """Inputs of the indexer prolog for the query tokens of a Workload: hidden
+    states x [T, d] and the stacked projection rows wt = [W_q; W_k; W_w]
+    [H_I*D_I + D_I + H_I, d] (bf16 bits), the key normalization weight gamma
+    [D_I] and eps.  Weights are N(0, 1/d) so that the projections are O(1)."""
+    T: int
+    d: int
+    H_I: int
+    D_I: int
+    x: np.ndarray
+    wt: np.ndarray
+    gamma: np.ndarray
+    eps: float
+
+
+def make_prolog(wl: Workload, d: int = 2048, seed: int = 0, int_inputs: bool = False) -> ProlWork:
+    """Synthetic prolog inputs sized for `wl` (its tokens, index heads and dim).  With
+    int_inputs, x and the weights are small integers (x in [-2, 2], weights in {-1, 0, 1})
+    so that every projection is an exact integer."""
+    n_out = wl.H_I * wl.D_I + wl.D_I + wl.H_I
+    r = _rng(seed, 11)
+    if int_inputs:
+        x = to_bf16_bits(r.integers(-2, 3, size=(wl.T, d)).astype(np.float32))
+        wt = to_bf16_bits(r.integers(-1, 2, size=(n_out, d)).astype(np.float32))
+        gamma = np.ones(wl.D_I, dtype=np.float32)
+    else:
+        x = _normal_bf16(seed, 12, (wl.T, d))
+        wt = to_bf16_bits((r.standard_normal((n_out, d), dtype=np.float32) / np.float32(math.sqrt(d))))
+        gamma = (0.5 + r.random(wl.D_I)).astype(np.float32)
+    return ProlWork(T=wl.T, d=d, H_I=wl.H_I, D_I=wl.D_I, x=x, wt=wt, gamma=gamma, eps=1e-6)
+
+
 def to_device(wl: Workload, device="cuda", with_kv: bool = True) -> dict:
     """Copy a workload's arrays to torch tensors on `device` (bf16 bits are
     reinterpreted as torch.bfloat16, e4m3 codes stay uint8)."""

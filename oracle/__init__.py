@@ -51,6 +51,11 @@ class _AttnArgs(ctypes.Structure):
                 ("q", ctypes.c_void_p), ("kv", ctypes.c_void_p), ("idx", ctypes.c_void_p)]
 
 
+class _PrologArgs(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("H_I", ctypes.c_int32), ("D_I", ctypes.c_int32),
+                ("x", ctypes.c_void_p), ("wt", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("eps", ctypes.c_double)]
+
+
 def _bind(path):
     lib = ctypes.CDLL(path)
     lib.oracle_indexer_topk.argtypes = [ctypes.POINTER(_IndexerArgs), ctypes.c_void_p,
@@ -65,6 +70,15 @@ def _bind(path):
     lib.oracle_e8m0_to_f64.argtypes = [ctypes.c_uint8]
     lib.oracle_e8m0_to_f64.restype = ctypes.c_double
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_indexer_prolog.argtypes = [ctypes.POINTER(_PrologArgs), ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p]
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_mx_encode.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+    lib.oracle_mx_encode.restype = None
+    lib.oracle_fp8_group_encode.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                            ctypes.c_void_p]
+    lib.oracle_fp8_group_encode.restype = None
     return lib
 
 
@@ -187,6 +201,46 @@ def sparse_attn(wl, idx, tokens=None, sm_scale=None):
     lse = np.empty((n, wl.H), dtype=np.float64)
     lib.oracle_sparse_attn(ctypes.byref(args), _ptr(tokens), n, _ptr(o), _ptr(lse))
     return o, lse
+
+
+def indexer_prolog(pw):
+    """Indexer prolog of a ProlWork (workloads.make_prolog): float64 q [T, H_I, D_I],
+    normalized keys k [T, D_I] and head weights w [T, H_I], before any rounding."""
+    lib = _load()
+    x = _c(pw.x, np.uint16)
+    wt = _c(pw.wt, np.uint16)
+    g = _c(pw.gamma, np.float32)
+    args = _PrologArgs(pw.T, pw.d, pw.H_I, pw.D_I, _ptr(x), _ptr(wt), _ptr(g), float(pw.eps))
+    q = np.empty((pw.T, pw.H_I * pw.D_I), dtype=np.float64)
+    k = np.empty((pw.T, pw.D_I), dtype=np.float64)
+    w = np.empty((pw.T, pw.H_I), dtype=np.float64)
+    lib.oracle_indexer_prolog(ctypes.byref(args), _ptr(q), _ptr(k), _ptr(w))
+    return q.reshape(pw.T, pw.H_I, pw.D_I), k, w
+
+
+def e4m3_encode(v: float) -> int:
+    """Nearest e4m3fn code of v (ties to even mantissa, saturated at +-448)."""
+    return int(_load().oracle_e4m3_encode(float(v)))
+
+
+def mx_encode(v):
+    """MXFP8 encoding along the last axis (a multiple of 32): (codes uint8, same
+    shape; shared exponents uint8, last axis / 32)."""
+    a = _c(v, np.float64)
+    codes = np.empty(a.shape, dtype=np.uint8)
+    sc = np.empty(a.shape[:-1] + (a.shape[-1] // 32,), dtype=np.uint8)
+    _load().oracle_mx_encode(_ptr(a), a.size, _ptr(codes), _ptr(sc))
+    return codes, sc
+
+
+def fp8_group_encode(v, group: int = 64):
+    """e4m3fn codes with one fp32 scale (amax / 448) per `group` values along the
+    last axis: (codes uint8, same shape; scales float32, last axis / group)."""
+    a = _c(v, np.float64)
+    codes = np.empty(a.shape, dtype=np.uint8)
+    sc = np.empty(a.shape[:-1] + (a.shape[-1] // group,), dtype=np.float32)
+    _load().oracle_fp8_group_encode(_ptr(a), a.size, int(group), _ptr(codes), _ptr(sc))
+    return codes, sc
 
 
 def e4m3_to_f64(code: int) -> float:

@@ -45,6 +45,15 @@
  *         o    = sum_j p_j * kv[s_j, 0:512],   lse = max l + ln sum_i exp(l_i - max l)
  *     Rows with index -1 are skipped.
  *
+ *  4. Indexer prolog (input preparation of the index stage).  "Day0
+ *     Adaptation and Performance Optimization ...", section 3 (query
+ *     projection, key RMS normalization, query quantization, head-weight
+ *     projection) and section 4 (projections kept in bf16, index Q/K in
+ *     MXFP8); "Large Model Inference Acceleration ...", section 1.2.  The
+ *     projections and the normalized key are returned in float64; the
+ *     encoders (e4m3fn, MXFP8 groups of 32, e4m3fn with one fp32 scale per
+ *     64) turn them into the stored formats.
+ *
  * All arithmetic is IEEE float64, no fused multiply-add contraction
  * (built with -ffp-contract=off), summation in index order.
  */
@@ -310,6 +319,108 @@ int oracle_sparse_attn(const oracle_attn_args* a, const int32_t* tokens, int n_t
         free(rows);
     }
     return 0;
+}
+
+/*
+ * Indexer prolog: the input preparation of the index stage ("Day0 Adaptation
+ * and Performance Optimization for Novel Long-Sequence Reasoning Models",
+ * section 3: query projection, key normalization, query quantization and
+ * head-weight projection; "Large Model Inference Acceleration ...", section
+ * 1.2).  For each new token t with hidden state x[t, 0:d] and the weight rows
+ * wt = [W_q (H_I*D_I rows) ; W_k (D_I rows) ; W_w (H_I rows)], each [d]:
+ *     p[n]      = sum_c x[t,c] * wt[n,c]
+ *     q[t,h,i]  = p[h*D_I + i]
+ *     k[t,i]    = p[HD + i] / sqrt(mean_j p[HD + j]^2 + eps) * gamma[i]   (RMS normalization)
+ *     w[t,h]    = p[HD + D_I + h]
+ * with HD = H_I*D_I.  Returned in float64, before any rounding or encoding.
+ */
+typedef struct {
+    int32_t T, d, H_I, D_I;
+    const uint16_t* x;               /* [T, d] bf16 bits */
+    const uint16_t* wt;              /* [H_I*D_I + D_I + H_I, d] bf16 bits */
+    const float* gamma;              /* [D_I] */
+    double eps;
+} oracle_prolog_args;
+
+int oracle_indexer_prolog(const oracle_prolog_args* a, double* q_out, double* k_out, double* w_out) {
+    const int HD = a->H_I * a->D_I, n_out = HD + a->D_I + a->H_I;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < a->T; t++) {
+        double* p = (double*)malloc(sizeof(double) * (size_t)n_out);
+        for (int n = 0; n < n_out; n++) {
+            double acc = 0.0;
+            for (int c = 0; c < a->d; c++)
+                acc += bf16_to_f64(a->x[(int64_t)t * a->d + c]) * bf16_to_f64(a->wt[(int64_t)n * a->d + c]);
+            p[n] = acc;
+        }
+        for (int i = 0; i < HD; i++) q_out[(int64_t)t * HD + i] = p[i];
+        double ms = 0.0;
+        for (int i = 0; i < a->D_I; i++) ms += p[HD + i] * p[HD + i];
+        ms /= (double)a->D_I;
+        double r = 1.0 / sqrt(ms + a->eps);
+        for (int i = 0; i < a->D_I; i++) k_out[(int64_t)t * a->D_I + i] = p[HD + i] * r * (double)a->gamma[i];
+        for (int h = 0; h < a->H_I; h++) w_out[(int64_t)t * a->H_I + h] = p[HD + a->D_I + h];
+        free(p);
+    }
+    return 0;
+}
+
+/*
+ * e4m3fn encoding of a real value: the nearest finite e4m3fn value, an exact tie
+ * going to the code with an even mantissa, magnitudes beyond the largest finite
+ * value (448) saturated to +-448.  Written as a search over the 127 non-negative
+ * finite codes, each decoded by oracle_e4m3_to_f64.
+ */
+uint8_t oracle_e4m3_encode(double v) {
+    double a = fabs(v);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c <= 126; c++) {
+        double d = fabs(oracle_e4m3_to_f64((uint8_t)c) - a);
+        if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) == 1)) { bd = d; best = c; }
+    }
+    if (best == 0) return 0;                          /* +0 for both signs of a zero result */
+    return (uint8_t)(best | (v < 0.0 ? 0x80 : 0));
+}
+
+/*
+ * MXFP8 encoding of n values (n a multiple of 32), 32 consecutive values per
+ * group ("Day0 Adaptation ...", section 4: every 32 elements share one scale;
+ * the OCP MX rule for the shared scale): X = 2^(floor(log2 amax) - 8), 8 being
+ * the exponent of the largest e4m3fn power of two, clamped to 2^-127..2^127;
+ * stored as the byte log2(X) + 127.  An all-zero group takes X = 1.  Each value
+ * is stored as oracle_e4m3_encode(v / X).
+ */
+void oracle_mx_encode(const double* v, int64_t n, uint8_t* codes, uint8_t* scales) {
+    for (int64_t g = 0; g < n / 32; g++) {
+        double amax = 0.0;
+        for (int i = 0; i < 32; i++) amax = fmax(amax, fabs(v[g * 32 + i]));
+        int e = 0;
+        if (amax > 0.0) {
+            int ex;
+            frexp(amax, &ex);                         /* amax = m * 2^ex, m in [0.5, 1) */
+            e = ex - 1 - 8;
+            if (e < -127) e = -127;
+            if (e > 127) e = 127;
+        }
+        scales[g] = (uint8_t)(e + 127);
+        for (int i = 0; i < 32; i++) codes[g * 32 + i] = oracle_e4m3_encode(ldexp(v[g * 32 + i], -e));
+    }
+}
+
+/*
+ * e4m3fn encoding with one fp32 scale per `group` consecutive values: s is
+ * amax / 448 rounded to fp32 (1 for an all-zero group) and each value is stored
+ * as oracle_e4m3_encode(v / s).
+ */
+void oracle_fp8_group_encode(const double* v, int64_t n, int group, uint8_t* codes, float* scales) {
+    for (int64_t g = 0; g < n / group; g++) {
+        double amax = 0.0;
+        for (int i = 0; i < group; i++) amax = fmax(amax, fabs(v[g * group + i]));
+        float sc = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+        scales[g] = sc;
+        for (int i = 0; i < group; i++) codes[g * group + i] = oracle_e4m3_encode(v[g * group + i] / (double)sc);
+    }
 }
 
 int oracle_num_threads(void) {

@@ -10,7 +10,11 @@
   a dominant logit;
 * the planted million-token workload: its Top-K must be the planted set;
 * exactness: integer-valued indexer inputs give scores equal to an
-  integer-arithmetic evaluation.
+  integer-arithmetic evaluation;
+* the indexer prolog: a hand case, the projections against a numpy float64
+  matmul, the key normalization against torch's rms_norm, scale invariance;
+  the e4m3 encoder against torch's float8_e4m3fn cast (ties and saturation
+  included), MX and per-64 encodings against their scale rules and error bounds.
 """
 import json
 import math
@@ -407,3 +411,126 @@ def test_million_token_planted_set_is_the_topk():
     wl = W.preset("1m", with_kv=False)
     r = oracle.indexer_topk(wl)
     np.testing.assert_array_equal(r["idx"][0], wl.planted.astype(np.int32))
+
+
+# ---------------------------------------------------------------- indexer prolog
+
+def _prolog_from_lists(x, wt, gamma, eps, H_I, D_I):
+    x = np.asarray(x, np.float32)[None, :] if np.ndim(x) == 1 else np.asarray(x, np.float32)
+    wt = np.asarray(wt, np.float32)
+    return W.ProlWork(T=x.shape[0], d=x.shape[1], H_I=H_I, D_I=D_I, x=W.to_bf16_bits(x),
+                      wt=W.to_bf16_bits(wt), gamma=np.asarray(gamma, np.float32), eps=float(eps))
+
+
+def test_hand_indexer_prolog():
+    g = GOLD["indexer_prolog"]
+    pw = _prolog_from_lists(g["x"], g["wt"], g["gamma"], g["eps"], H_I=1, D_I=2)
+    q, k, w = oracle.indexer_prolog(pw)
+    np.testing.assert_array_equal(q.reshape(-1), g["q"])
+    np.testing.assert_allclose(k.reshape(-1), g["k"], rtol=1e-15)
+    np.testing.assert_array_equal(w.reshape(-1), g["w"])
+
+
+def _small_prolog(seed=3, T=5, d=96, H_I=4, D_I=64):
+    wl = W.make_workload("p", seq_lens=[T + 7], nq=T, H_I=H_I, D_I=D_I, H=1, K=8, with_kv=False, seed=seed)
+    return W.make_prolog(wl, d=d, seed=seed)
+
+
+def test_prolog_projection_matches_numpy_matmul():
+    pw = _small_prolog()
+    q, k, w = oracle.indexer_prolog(pw)
+    x = W.bf16_bits_to_f32(pw.x).astype(np.float64)
+    wt = W.bf16_bits_to_f32(pw.wt).astype(np.float64)
+    p = x @ wt.T
+    HD = pw.H_I * pw.D_I
+    np.testing.assert_allclose(q.reshape(pw.T, HD), p[:, :HD], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(w, p[:, HD + pw.D_I:], rtol=1e-12, atol=1e-12)
+
+
+def test_prolog_key_matches_torch_rms_norm():
+    pw = _small_prolog(seed=4)
+    _, k, _ = oracle.indexer_prolog(pw)
+    x = torch.from_numpy(W.bf16_bits_to_f32(pw.x).astype(np.float64))
+    wt = torch.from_numpy(W.bf16_bits_to_f32(pw.wt).astype(np.float64))
+    HD = pw.H_I * pw.D_I
+    pk = x @ wt[HD:HD + pw.D_I].T
+    ref = torch.nn.functional.rms_norm(pk, (pw.D_I,), weight=torch.from_numpy(pw.gamma.astype(np.float64)),
+                                       eps=pw.eps)
+    np.testing.assert_allclose(k, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_prolog_key_is_invariant_to_key_row_scaling():
+    # with eps = 0, RMS normalization removes any positive factor on W_k
+    pw = _small_prolog(seed=5)
+    pw.eps = 0.0
+    _, k1, _ = oracle.indexer_prolog(pw)
+    HD = pw.H_I * pw.D_I
+    wt = pw.wt.copy()
+    wt[HD:HD + pw.D_I] = W.to_bf16_bits(W.bf16_bits_to_f32(wt[HD:HD + pw.D_I]) * np.float32(4.0))
+    pw2 = W.ProlWork(**{**pw.__dict__, "wt": wt})
+    _, k2, _ = oracle.indexer_prolog(pw2)
+    np.testing.assert_allclose(k2, k1, rtol=1e-13, atol=1e-13)
+    # and with gamma = 1 every key has unit mean square
+    pw3 = W.ProlWork(**{**pw.__dict__, "gamma": np.ones(pw.D_I, np.float32)})
+    _, k3, _ = oracle.indexer_prolog(pw3)
+    np.testing.assert_allclose((k3 ** 2).mean(axis=1), 1.0, rtol=1e-12)
+
+
+def test_hand_mx_encode_group():
+    g = GOLD["mx_encode_group"]
+    v = np.zeros(32)
+    v[:len(g["values"])] = g["values"]
+    codes, sc = oracle.mx_encode(v)
+    assert int(sc[0]) == g["scale"]
+    assert [int(c) for c in codes[:len(g["codes"])]] == g["codes"]
+    assert not codes[len(g["codes"]):].any()
+
+
+def test_e4m3_encode_matches_torch_cast_including_ties_and_saturation():
+    grid = np.array([0.0, -0.0, 2.0 ** -10, -(2.0 ** -10)])
+    decoded = np.array([oracle.e4m3_to_f64(c) for c in range(127)])
+    mids = (decoded[:-1] + decoded[1:]) / 2                      # every tie between neighbours
+    r = np.random.default_rng(0)
+    vals = np.concatenate([grid, decoded, mids, r.uniform(-500, 500, 2000), r.standard_normal(2000) * 1e-2,
+                           -decoded, -mids, [448.0, 449.0, 464.0, 465.0, 1e6, -1e6]])
+    vals = vals.astype(np.float32).astype(np.float64)            # torch casts from float32
+    got = np.array([oracle.e4m3_encode(v) for v in vals], np.uint8)
+    ref = W.encode_e4m3(vals.astype(np.float32))
+    # a negative value that rounds to zero is -0 in torch (code 0x80); the oracle stores +0
+    ref = np.where(ref == 0x80, 0, ref)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_mx_encode_scale_rule_and_error_bound():
+    r = np.random.default_rng(1)
+    v = r.standard_normal((64, 32)) * np.exp2(r.integers(-20, 20, size=(64, 1)))
+    v[3] = 0.0
+    codes, sc = oracle.mx_encode(v)
+    X = np.exp2(sc.astype(np.float64) - 127)[:, 0]
+    amax = np.abs(v).max(axis=1)
+    nz = amax > 0
+    ratio = amax[nz] / X[nz]
+    assert (ratio >= 256).all() and (ratio < 512).all()
+    assert sc[3, 0] == 127 and not codes[3].any()
+    dec = np.array([[oracle.e4m3_to_f64(c) for c in row] for row in codes]) * X[:, None]
+    # nearest e4m3 below 448: error at most half a step (1/16 of the binade), at 448 saturation
+    y = np.abs(v) / X[:, None]
+    step = np.exp2(np.floor(np.log2(np.maximum(y, 2.0 ** -6))) - 3)
+    err = np.abs(dec - v) / X[:, None]
+    ok = np.where(y <= 448, err <= step / 2 + 1e-12, np.abs(dec) / X[:, None] == 448)
+    assert ok.all()
+
+
+def test_fp8_group_encode_scale_is_amax_over_448():
+    r = np.random.default_rng(2)
+    v = r.standard_normal((16, 128)) * 3
+    v[5, :64] = 0.0
+    codes, sc = oracle.fp8_group_encode(v, 64)
+    amax = np.abs(v.reshape(16, 2, 64)).max(axis=2)
+    np.testing.assert_array_equal(sc, np.where(amax > 0, (amax / 448.0).astype(np.float32), 1.0))
+    dec = np.array([[oracle.e4m3_to_f64(c) for c in row] for row in codes]).reshape(16, 2, 64)
+    dec *= sc[..., None]
+    np.testing.assert_allclose(dec, v.reshape(16, 2, 64), rtol=2 ** -4, atol=np.abs(v).max() * 2.0 ** -9)
+    # the group maximum maps onto 448 (up to the fp32 rounding of the scale)
+    big = (codes.reshape(16, 2, 64) & 0x7F).max(axis=2)
+    assert (big[amax > 0] >= 0x7D).all()

@@ -43,6 +43,19 @@ MUTANTS = [
     ("mx_query_group_of_64", "oracle_e8m0_to_f64(a->q_scale[((int64_t)t * a->H_I + h) * (a->D_I / 32) + d / 32]);",
      "oracle_e8m0_to_f64(a->q_scale[((int64_t)t * a->H_I + h) * (a->D_I / 32) + d / 64]);"),
     ("e8m0_bias_126", "return ldexp(1.0, (int)e - 127);", "return ldexp(1.0, (int)e - 126);"),
+    ("prolog_rms_sum_not_mean", "ms /= (double)a->D_I;", "ms /= 1.0;"),
+    ("prolog_eps_outside_sqrt", "double r = 1.0 / sqrt(ms + a->eps);", "double r = 1.0 / (sqrt(ms) + a->eps);"),
+    ("prolog_gamma_reversed", "k_out[(int64_t)t * a->D_I + i] = p[HD + i] * r * (double)a->gamma[i];",
+     "k_out[(int64_t)t * a->D_I + i] = p[HD + i] * r * (double)a->gamma[a->D_I - 1 - i];"),
+    ("prolog_weight_rows_shifted", "w_out[(int64_t)t * a->H_I + h] = p[HD + a->D_I + h];",
+     "w_out[(int64_t)t * a->H_I + h] = p[HD + h];"),
+    ("prolog_x_transposed", "acc += bf16_to_f64(a->x[(int64_t)t * a->d + c])",
+     "acc += bf16_to_f64(a->x[(int64_t)(a->T - 1 - t) * a->d + c])"),
+    ("e4m3_ties_away", "if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) == 1))", "if (d <= bd)"),
+    ("mx_scale_minus_7", "e = ex - 1 - 8;", "e = ex - 1 - 7;"),
+    ("mx_zero_group_scale", "int e = 0;\n        if (amax > 0.0) {", "int e = -127;\n        if (amax > 0.0) {"),
+    ("fp8_group_scale_over_240", "float sc = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;",
+     "float sc = amax > 0.0 ? (float)(amax / 240.0) : 1.0f;"),
 ]
 
 PINS = [pins.test_hand_indexer_relu_gate_weights_and_tie, pins.test_hand_fp8_scale_groups,
@@ -50,7 +63,10 @@ PINS = [pins.test_hand_indexer_relu_gate_weights_and_tie, pins.test_hand_fp8_sca
         pins.test_hand_softmax_two_rows, pins.test_e4m3_decode_all_codes_vs_torch,
         pins.test_single_head_unit_weight_is_relu_dot_lexsort,
         pins.test_k_at_least_context_equals_dense_causal_attention, pins.test_hand_mxfp8_groups,
-        pins.test_e8m0_decode_all_exponents_vs_torch]
+        pins.test_e8m0_decode_all_exponents_vs_torch, pins.test_hand_indexer_prolog,
+        pins.test_prolog_projection_matches_numpy_matmul, pins.test_prolog_key_matches_torch_rms_norm,
+        pins.test_hand_mx_encode_group, pins.test_e4m3_encode_matches_torch_cast_including_ties_and_saturation,
+        pins.test_mx_encode_scale_rule_and_error_bound, pins.test_fp8_group_encode_scale_is_amax_over_448]
 
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
