@@ -14,7 +14,9 @@ indexer); per-kernel times come from separate launches with events between
 them.  On one GPU the line also carries the other four workloads (tiny
 decode, ragged verify with fp8 keys, million-token decode, 16K causal
 prefill) under "workloads", each with its step time, per-kernel times and
-roofline fractions.  Under torchrun each rank runs its own replica of the
+roofline fractions, and the indexer prolog (projections, key normalization,
+query and key encoding) at a decode and a prefill shape under "indexer_prolog".
+Under torchrun each rank runs its own replica of the
 batch (weak scaling, no data-path collective); the step time is the maximum
 over ranks.  Prints one JSON line on rank 0.
 """
@@ -288,6 +290,72 @@ def measure(dsa, W, wl, dev, steps, warmup, graph=True):
                 pct={"p10": q[0], "p50": statistics.median(per_step), "p90": q[-1]}, t_start=t_start, t_end=t_end)
 
 
+PROLOG_D_MODEL = 7168
+
+
+def measure_prolog(dsa, dev, name, B, ctx, nq, steps, peak, tf_peak):
+    """Time indexer_prolog (64 x 128 index heads, bf16 keys, d_model 7168) for B sequences of
+    `ctx` cached positions with `nq` new tokens each; synthetic device inputs (weights
+    N(0, 1/d)).  Decode shapes are weight-streaming (HBM roofline: weights + hidden states +
+    outputs); prefill shapes are a dense contraction (tensor roofline: 2 T n_out d)."""
+    import torch
+    H_I, D_I, d = 64, 128, PROLOG_D_MODEL
+    n_out = H_I * D_I + D_I + H_I
+    T = B * nq
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    x = torch.randn((T, d), generator=g, device=dev).to(torch.bfloat16)
+    wp = (torch.randn((n_out, d), generator=g, device=dev) / math.sqrt(d)).to(torch.bfloat16)
+    gamma = torch.rand((D_I,), generator=g, device=dev) + 0.5
+    pages = (ctx + 63) // 64
+    seq_lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    cu_q = torch.arange(0, T + 1, nq, dtype=torch.int32, device=dev)
+    table = torch.randperm(B * pages, generator=g, device=dev).to(torch.int32).view(B, pages)
+    k_cache = torch.zeros((B * pages, 64, D_I), dtype=torch.bfloat16, device=dev)
+    batch = dsa.Batch(seq_lens, cu_q, table, B * pages, ctx, nq)
+    q = torch.empty((T, H_I, D_I), dtype=torch.bfloat16, device=dev)
+    w = torch.empty((T, H_I), dtype=torch.float32, device=dev)
+    ws = dsa.Workspace(dev)
+    stream = torch.cuda.current_stream()
+    scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def call():
+        dsa.indexer_prolog(batch, x, wp, gamma, 1e-6, k_cache, None, q_out=q, w_out=w, workspace=ws)
+
+    for _ in range(3):
+        scrub.zero_()
+        call()
+    torch.cuda.synchronize()
+    if dsa.get_status(ws) != 0:
+        raise RuntimeError(f"prolog {name}: device reported an error")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        scrub.zero_()
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    if dsa.get_status(ws) != 0:
+        raise RuntimeError(f"prolog {name}: device reported an error")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    byts = n_out * d * 2 + T * d * 2 + T * (H_I * D_I * 2 + H_I * 4 + D_I * 2)
+    flops = 2.0 * T * n_out * d
+    gbs = byts / (ms * 1e-3) / 1e9
+    tfs = flops / (ms * 1e-3) / 1e12
+    e = {"shape": f"{B} sequences x {nq} new tokens (T={T}), ctx {ctx}, d_model {d}, index heads {H_I}x{D_I}, "
+                  f"bf16 queries and keys, {n_out} projection rows",
+         "steps": steps, "ms_per_launch": ms, "tokens_per_s": T / (ms * 1e-3),
+         "algorithmic_bytes": byts, "algorithmic_flops": flops, "gbs": gbs, "tflops": tfs,
+         "l2": "flushed between launches"}
+    if T <= 256:
+        e["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak}
+    else:
+        e["roofline"] = {"bound": "tensor", "achieved": tfs, "peak": tf_peak, "unit": "TFLOP/s", "frac": tfs / tf_peak}
+    del x, wp, k_cache, scrub, ws
+    torch.cuda.empty_cache()
+    return e
+
+
 def kernel_entry(wl, r, peak):
     """Per-kernel times and roofline fractions of one measured workload."""
     key_bytes, kv_bytes = wl.key_bytes(), wl.kv_bytes()
@@ -410,6 +478,13 @@ def run_ours(args, rank, world, local_rank):
             extra[name] = entry
             del xr, xw
             torch.cuda.empty_cache()
+    prolog = {}
+    if world == 1 and not args.no_extra_workloads:
+        tf_peak, _ = peaks_tensor()
+        prolog["decode32"] = measure_prolog(dsa, dev, "decode32", 32, 32768, 1, max(3, min(args.steps, 50)), peak,
+                                            tf_peak)
+        prolog["prefill16k"] = measure_prolog(dsa, dev, "prefill16k", 1, 16384, 16384, max(3, min(args.steps, 10)),
+                                              peak, tf_peak)
     if rank != 0:
         return
     idx_gbs = key_bytes / (idx_ms * 1e-3) / 1e9
@@ -458,6 +533,8 @@ def run_ours(args, rank, world, local_rank):
     line["kernels"]["sfa_decode_kernel"]["traffic"] = ncu_traffic("sfa_decode_kernel") if args.workload == "batch32" else None
     if extra:
         line["workloads"] = extra
+    if prolog:
+        line["indexer_prolog"] = prolog
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         value, dt = cpu_baseline(wl, np.arange(wl.T) if wl.T <= 64 else np.linspace(0, wl.T - 1, 32).astype(np.int64))

@@ -238,6 +238,67 @@ DSA_API dsa_status dsa_get_status(void* workspace, void* stream, int32_t* device
 DSA_API int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexer_inputs* ix,
                                         const dsa_attn_inputs* at);
 
+/*
+ * Indexer prolog: the input preparation of the index stage ("Day0 Adaptation
+ * and Performance Optimization for Novel Long-Sequence Reasoning Models",
+ * section 3: query projection, key RMS normalization, query quantization and
+ * head-weight projection, projections kept in bf16 (section 4); "Large Model
+ * Inference Acceleration ...", section 1.2).  For each query token t with
+ * hidden state x[t, :] and p = W . x[t, :] (fp32 accumulation of bf16 inputs):
+ *     q[t, h, i] = p[h*D_I + i]
+ *     k[t, i]    = p[HD + i] / sqrt(mean_j p[HD + j]^2 + eps) * k_gamma[i]
+ *     w[t, h]    = p[HD + D_I + h]                         (HD = H_I * D_I)
+ * q is written to q_out in q_dtype (bf16, round to nearest even; or MXFP8:
+ * e4m3fn codes [T, H_I, D_I] plus one shared exponent per 32 elements in
+ * q_scale_out [T, H_I, D_I/32], scale 2^(floor(log2 amax) - 8)); w to w_out
+ * [T, H_I] fp32; k into the token's row of the paged indexer-key cache
+ * (position seq_lens[b] - nq_b + j for token j of sequence b, page from the
+ * block table) in key_dtype: bf16; e4m3fn codes with one fp32 scale
+ * amax/448 per 64 elements in k_scale [num_blocks, 64, D_I/64]; or MXFP8
+ * codes with k_scale [num_blocks, 64, D_I/32] exponents.  e4m3fn codes are
+ * rounded to nearest even and saturated at +-448; a zero is stored as +0.
+ * All four come out of one kernel (a tensor-core GEMM over the stacked weight
+ * rows with the normalization and encoding applied to its accumulators).
+ */
+typedef struct {
+    const void* x;              /* device [T, d_model] bf16 hidden states of the step's tokens, 16-byte aligned */
+    const void* w_proj;         /* device [H_I*D_I + D_I + H_I, d_model] bf16, 16-byte aligned: the query    */
+                                /* rows (head h, element i at row h*D_I + i), then the D_I key rows, then   */
+                                /* the H_I head-weight rows                                                 */
+    const float* k_gamma;       /* device [D_I] key RMS-normalization weight                                */
+    float eps;                  /* RMS-normalization epsilon, >= 0                                           */
+    int32_t d_model;            /* hidden size: a multiple of 8                                              */
+    int32_t H_I;                /* 8, 16, 32 or 64                                                           */
+    int32_t D_I;                /* 64 or 128                                                                 */
+    int32_t key_dtype;          /* dsa_key_dtype of the key cache written                                    */
+    int32_t q_dtype;            /* dsa_query_dtype of q_out (MXFP8 exactly when key_dtype is MXFP8)          */
+} dsa_prolog_inputs;
+
+/*
+ * Bytes of workspace indexer_prolog needs for this shape (0 if the arguments
+ * are invalid).  Layout: [256-byte status area][split counters][fp32 partial
+ * tiles when the contraction is split along d_model].  The status area and
+ * the counters must be zero-filled before the first call and stay so after
+ * every successful call; the partial tiles are scratch, so a workspace that
+ * indexer_prolog has used must be zero-filled again before indexer_topk,
+ * sparse_mla_attn or dsa_decode use it.
+ */
+DSA_API size_t dsa_prolog_workspace_size(const dsa_batch* batch, const dsa_prolog_inputs* pr);
+
+/*
+ * Runs the prolog for the batch's T tokens (batch->max_seq_len and
+ * max_q_per_seq are not used).  Outputs: q_out (bf16 [T, H_I, D_I], or e4m3
+ * codes with q_scale_out for MXFP8), w_out [T, H_I] fp32, and the tokens'
+ * rows of k_cache / k_scale (layouts of dsa_indexer_inputs); no other cache
+ * row is touched.  A token whose page id is out of range is skipped and
+ * recorded as DSA_ERR_DEVICE_BOUNDS in the status word.  Returns
+ * DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED / DSA_ERR_WORKSPACE before
+ * launching anything, DSA_ERR_CUDA if the launch fails.
+ */
+DSA_API dsa_status indexer_prolog(const dsa_batch* batch, const dsa_prolog_inputs* pr, void* q_out,
+                                  uint8_t* q_scale_out, float* w_out, void* k_cache, void* k_scale,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static description of a status code. */
 DSA_API const char* dsa_status_str(int32_t status);
 

@@ -13,6 +13,9 @@ Entry points (same names as the C ABI):
     dsa_decode(batch, q_idx, w, k_cache, q, kv_cache, K, sm_scale, k_scale=None, q_scale=None)
         -> (idx, score, out, lse)
 
+    indexer_prolog(batch, x, w_proj, k_gamma, eps, k_cache, k_scale=None, mx=False)
+        -> (q_idx, q_scale or None, w)   (also writes the tokens' keys into k_cache / k_scale)
+
 Key formats: bf16 keys (k_scale None); e4m3 keys (uint8) with fp32 k_scale
 [nblk, 64, D_I/64]; MXFP8 queries and keys when q_scale is given: q_idx and
 k_cache hold e4m3 codes (uint8), q_scale [T, H_I, D_I/32] and k_scale
@@ -25,7 +28,8 @@ import os
 from dataclasses import dataclass
 from typing import Optional
 
-__all__ = ["Batch", "Workspace", "indexer_topk", "sparse_mla_attn", "dsa_decode", "get_status",
+__all__ = ["Batch", "Workspace", "indexer_topk", "sparse_mla_attn", "dsa_decode", "indexer_prolog",
+           "get_status",
            "DsaError", "library_path", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +74,12 @@ class _Attn(ctypes.Structure):
                 ("sm_scale", ctypes.c_float)]
 
 
+class _Prolog(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("w_proj", ctypes.c_void_p), ("k_gamma", ctypes.c_void_p),
+                ("eps", ctypes.c_float), ("d_model", ctypes.c_int32), ("H_I", ctypes.c_int32),
+                ("D_I", ctypes.c_int32), ("key_dtype", ctypes.c_int32), ("q_dtype", ctypes.c_int32)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -103,6 +113,12 @@ def load_library():
     lib.dsa_get_status.restype = ctypes.c_int
     lib.dsa_decode_launch_count.argtypes = [P(_Batch), P(_Indexer), P(_Attn)]
     lib.dsa_decode_launch_count.restype = ctypes.c_int32
+    lib.dsa_prolog_workspace_size.argtypes = [P(_Batch), P(_Prolog)]
+    lib.dsa_prolog_workspace_size.restype = ctypes.c_size_t
+    lib.indexer_prolog.argtypes = [P(_Batch), P(_Prolog), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                   ctypes.c_void_p]
+    lib.indexer_prolog.restype = ctypes.c_int
     lib.dsa_status_str.argtypes = [ctypes.c_int32]
     lib.dsa_status_str.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
@@ -348,6 +364,73 @@ def dsa_decode(batch: Batch, q_idx, w, k_cache, q, kv_cache, K: int, sm_scale: f
     if rc != 0:
         raise DsaError(rc, "dsa_decode")
     return out_idx, out_score, out, lse
+
+
+_prolog_ws = {}
+
+
+def prolog_workspace(device=None) -> Workspace:
+    """The default workspace of indexer_prolog on a device (kept apart from the
+    other entry points' workspace: its partial-tile region is scratch)."""
+    import torch
+    device = torch.device("cuda") if device is None else torch.device(device)
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    if key not in _prolog_ws:
+        _prolog_ws[key] = Workspace(torch.device("cuda", key))
+    return _prolog_ws[key]
+
+
+def indexer_prolog(batch: Batch, x, w_proj, k_gamma, eps: float, k_cache, k_scale=None, mx: bool = False, *,
+                   H_I: Optional[int] = None, q_out=None, q_scale_out=None, w_out=None,
+                   workspace: Optional[Workspace] = None, stream=None):
+    """Indexer prolog: projects the step's hidden states x [T, d] with the stacked rows
+    w_proj [H_I*D_I + D_I + H_I, d] (bf16), RMS-normalizes the keys (k_gamma [D_I] fp32,
+    eps) and writes them into the tokens' rows of the paged key cache (format given by
+    k_cache / k_scale as for indexer_topk; MXFP8 when mx).  Returns (q_idx [T, H_I, D_I]
+    bf16 or e4m3 codes, q_scale [T, H_I, D_I/32] uint8 or None, w [T, H_I] fp32)."""
+    import torch
+    lib = load_library()
+    _check(x, "x", torch.bfloat16, 2)
+    _check(w_proj, "w_proj", torch.bfloat16, 2, (None, x.shape[1]))
+    _check(k_gamma, "k_gamma", torch.float32, 1)
+    T, d = x.shape
+    D_I = int(k_gamma.shape[0])
+    n_out = int(w_proj.shape[0])
+    H_I = (n_out - D_I) // (D_I + 1) if H_I is None else int(H_I)
+    if H_I * D_I + D_I + H_I != n_out:
+        raise ValueError(f"w_proj has {n_out} rows; H_I*D_I + D_I + H_I rows are needed")
+    if mx:
+        _check(k_cache, "k_cache", torch.uint8, 3, (None, 64, D_I))
+        if k_scale is None:
+            raise ValueError("MXFP8 keys need k_scale")
+        _check(k_scale, "k_scale", torch.uint8, 3, (k_cache.shape[0], 64, D_I // 32))
+        kt, qt = KEY_MXFP8, Q_MXFP8
+    elif k_scale is None:
+        _check(k_cache, "k_cache", torch.bfloat16, 3, (None, 64, D_I))
+        kt, qt = KEY_BF16, Q_BF16
+    else:
+        _check(k_cache, "k_cache", torch.uint8, 3, (None, 64, D_I))
+        _check(k_scale, "k_scale", torch.float32, 3, (k_cache.shape[0], 64, D_I // 64))
+        kt, qt = KEY_FP8_E4M3, Q_BF16
+    dev = x.device
+    if q_out is None:
+        q_out = torch.empty((T, H_I, D_I), dtype=torch.uint8 if mx else torch.bfloat16, device=dev)
+    if mx and q_scale_out is None:
+        q_scale_out = torch.empty((T, H_I, D_I // 32), dtype=torch.uint8, device=dev)
+    if w_out is None:
+        w_out = torch.empty((T, H_I), dtype=torch.float32, device=dev)
+    pr = _Prolog(_ptr(x), _ptr(w_proj), _ptr(k_gamma), float(eps), int(d), H_I, D_I, kt, qt)
+    cb = batch.c(T)
+    ws = workspace if workspace is not None else prolog_workspace(dev)
+    need = lib.dsa_prolog_workspace_size(ctypes.byref(cb), ctypes.byref(pr))
+    if need == 0:
+        raise DsaError(2, "dsa_prolog_workspace_size")
+    buf = ws.get(need)
+    rc = lib.indexer_prolog(ctypes.byref(cb), ctypes.byref(pr), _ptr(q_out), _ptr(q_scale_out), _ptr(w_out),
+                            _ptr(k_cache), _ptr(k_scale), _ptr(buf), buf.numel(), _stream(stream))
+    if rc != 0:
+        raise DsaError(rc, "indexer_prolog")
+    return q_out, q_scale_out, w_out
 
 
 def decode_launch_count(batch: Batch, q_idx, w, k_cache, q, kv_cache, K: int, sm_scale: float,
