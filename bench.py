@@ -193,10 +193,26 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+class L2Flush:
+    """Clears the L2 between timed steps, outside their events: writes a buffer of twice the
+    L2, then reads another one of the same size, so that the lines the write left dirty are
+    written back before the next step starts (the step then pays neither for reads that hit
+    the L2 nor for another buffer's write-backs)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.max()
+
+
 def measure(dsa, W, wl, dev, steps, warmup, graph=True):
     """Time one workload on `dev`: the fused step (dsa_decode, the attention launch overlapping the end of
     the indexer), each kernel alone (events between the two launches), and a CUDA-graph replay of the step.
-    Inputs smaller than twice the L2 are scrubbed from it between steps (outside the per-step events) and
+    Inputs smaller than twice the L2 are flushed from it between steps (L2Flush, outside the per-step events) and
     each step is timed on its own."""
     import torch
     d = W.to_device(wl, dev)
@@ -208,7 +224,7 @@ def measure(dsa, W, wl, dev, steps, warmup, graph=True):
     stream = torch.cuda.current_stream()
     step_bytes = wl.key_bytes() + wl.kv_bytes()
     flush = step_bytes < 2 * L2_BYTES
-    scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
+    scrub = L2Flush(dev) if flush else None
 
     def fused():
         dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], wl.K, wl.sm_scale,
@@ -223,7 +239,7 @@ def measure(dsa, W, wl, dev, steps, warmup, graph=True):
 
     for _ in range(max(3, warmup)):
         if flush:
-            scrub.zero_()
+            scrub()
         fused()
     torch.cuda.synchronize()
     if dsa.get_status(ws) != 0:
@@ -236,7 +252,7 @@ def measure(dsa, W, wl, dev, steps, warmup, graph=True):
     e0.record(stream)
     for a, b in ev:
         if flush:
-            scrub.zero_()
+            scrub()
         a.record(stream)
         fused()
         b.record(stream)
@@ -250,7 +266,7 @@ def measure(dsa, W, wl, dev, steps, warmup, graph=True):
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     for a, b, c in kev:
         if flush:
-            scrub.zero_()
+            scrub()
         a.record(stream)
         indexer()
         b.record(stream)
@@ -293,11 +309,12 @@ def measure(dsa, W, wl, dev, steps, warmup, graph=True):
 PROLOG_D_MODEL = 7168
 
 
-def measure_prolog(dsa, dev, name, B, ctx, nq, steps, peak, tf_peak):
+def measure_prolog(dsa, dev, name, B, ctx, nq, steps, peak, tf_peak, packed=True):
     """Time indexer_prolog (64 x 128 index heads, bf16 keys, d_model 7168) for B sequences of
     `ctx` cached positions with `nq` new tokens each; synthetic device inputs (weights
-    N(0, 1/d)).  Decode shapes are weight-streaming (HBM roofline: weights + hidden states +
-    outputs); prefill shapes are a dense contraction (tensor roofline: 2 T n_out d)."""
+    N(0, 1/d), tile-packed once before timing unless packed=False).  Decode shapes are
+    weight-streaming (HBM roofline: weights + hidden states + outputs); prefill shapes are a
+    dense contraction (tensor roofline: 2 T n_out d)."""
     import torch
     H_I, D_I, d = 64, 128, PROLOG_D_MODEL
     n_out = H_I * D_I + D_I + H_I
@@ -306,6 +323,8 @@ def measure_prolog(dsa, dev, name, B, ctx, nq, steps, peak, tf_peak):
     g.manual_seed(7)
     x = torch.randn((T, d), generator=g, device=dev).to(torch.bfloat16)
     wp = (torch.randn((n_out, d), generator=g, device=dev) / math.sqrt(d)).to(torch.bfloat16)
+    if packed:
+        wp = dsa.prolog_pack_weights(wp, H_I, D_I)
     gamma = torch.rand((D_I,), generator=g, device=dev) + 0.5
     pages = (ctx + 63) // 64
     seq_lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
@@ -317,20 +336,20 @@ def measure_prolog(dsa, dev, name, B, ctx, nq, steps, peak, tf_peak):
     w = torch.empty((T, H_I), dtype=torch.float32, device=dev)
     ws = dsa.Workspace(dev)
     stream = torch.cuda.current_stream()
-    scrub = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    scrub = L2Flush(dev)
 
     def call():
         dsa.indexer_prolog(batch, x, wp, gamma, 1e-6, k_cache, None, q_out=q, w_out=w, workspace=ws)
 
     for _ in range(3):
-        scrub.zero_()
+        scrub()
         call()
     torch.cuda.synchronize()
     if dsa.get_status(ws) != 0:
         raise RuntimeError(f"prolog {name}: device reported an error")
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in ev:
-        scrub.zero_()
+        scrub()
         a.record(stream)
         call()
         b.record(stream)
@@ -346,7 +365,7 @@ def measure_prolog(dsa, dev, name, B, ctx, nq, steps, peak, tf_peak):
                   f"bf16 queries and keys, {n_out} projection rows",
          "steps": steps, "ms_per_launch": ms, "tokens_per_s": T / (ms * 1e-3),
          "algorithmic_bytes": byts, "algorithmic_flops": flops, "gbs": gbs, "tflops": tfs,
-         "l2": "flushed between launches"}
+         "l2": "flushed between launches (write then read of 2x L2)", "weights": "tile-packed" if packed else "row-major"}
     if T <= 256:
         e["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak}
     else:
@@ -442,7 +461,7 @@ def run_ours(args, rank, world, local_rank):
     ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.e2e_steps)]
     for a, b in ee:
         if flush:
-            scrub.zero_()
+            scrub()
         a.record(stream)
         e2e_step()
         b.record(stream)
@@ -473,7 +492,7 @@ def run_ours(args, rank, world, local_rank):
                      "tokens_per_s": xw.T / (xr["ms_step"] * 1e-3), "step_ms_percentiles": xr["pct"],
                      "bytes_per_step": xw.key_bytes() + xw.kv_bytes(),
                      "step_gbs": (xw.key_bytes() + xw.kv_bytes()) / (xr["ms_step"] * 1e-3) / 1e9,
-                     "l2": "flushed between steps" if xr["flush"] else "inputs larger than L2",
+                     "l2": "flushed between steps (write then read of 2x L2)" if xr["flush"] else "inputs larger than L2",
                      "kernels": kernel_entry(xw, xr, peak)}
             extra[name] = entry
             del xr, xw
@@ -493,7 +512,8 @@ def run_ours(args, rank, world, local_rank):
     tokens_total = T * world
     clocks = sampler.summary(t_start, t_end) or sampler.summary(t_warm, soak_end)
     window = "timed region" if sampler.summary(t_start, t_end) else "warm-up + timed + soak of the same step"
-    l2 = (f"L2 flushed between steps ({2 * L2_BYTES / 1e6:.0f} MB written outside the per-step events): "
+    l2 = (f"L2 flushed between steps ({2 * L2_BYTES / 1e6:.0f} MB written, then {2 * L2_BYTES / 1e6:.0f} MB read, "
+          f"outside the per-step events): "
           f"{step_bytes / 1e6:.1f} MB read per step vs {L2_BYTES / 1e6:.0f} MB L2" if flush else
           f"inputs larger than L2: {step_bytes / 1e6:.1f} MB read per step vs {L2_BYTES / 1e6:.0f} MB L2, no flush")
     if wl.T > 64:

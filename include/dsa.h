@@ -260,6 +260,12 @@ DSA_API int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexe
  * All four come out of one kernel (a tensor-core GEMM over the stacked weight
  * rows with the normalization and encoding applied to its accumulators).
  */
+typedef enum {
+    DSA_W_ROW_MAJOR = 0,        /* w_proj row-major [H_I*D_I + D_I + H_I, d_model]                          */
+    DSA_W_TILE_PACKED = 1       /* w_proj as written by indexer_prolog_pack: each 128-row x 64-column block */
+                                /* contiguous, so that the weights stream from HBM in 16 KB pieces         */
+} dsa_weight_layout;
+
 typedef struct {
     const void* x;              /* device [T, d_model] bf16 hidden states of the step's tokens, 16-byte aligned */
     const void* w_proj;         /* device [H_I*D_I + D_I + H_I, d_model] bf16, 16-byte aligned: the query    */
@@ -272,7 +278,28 @@ typedef struct {
     int32_t D_I;                /* 64 or 128                                                                 */
     int32_t key_dtype;          /* dsa_key_dtype of the key cache written                                    */
     int32_t q_dtype;            /* dsa_query_dtype of q_out (MXFP8 exactly when key_dtype is MXFP8)          */
+    int32_t w_layout;           /* dsa_weight_layout of w_proj                                               */
 } dsa_prolog_inputs;
+
+/*
+ * Bytes of the tile-packed copy of the prolog weights (0 for invalid sizes):
+ * ceil(n_out/128) * ceil(d_model/64) blocks of 128 x 64 bf16, n_out =
+ * H_I*D_I + D_I + H_I.  Block (i, j) holds rows 128i.. and columns 64j.. of
+ * the row-major matrix (zeros past its edges), row-major, at element offset
+ * (i * ceil(d_model/64) + j) * 8192.
+ */
+DSA_API size_t dsa_prolog_packed_bytes(int32_t H_I, int32_t D_I, int32_t d_model);
+
+/*
+ * Writes the tile-packed copy of the row-major prolog weights w_proj into
+ * w_packed (dsa_prolog_packed_bytes bytes, 16-byte aligned; both device
+ * pointers), enqueued on `stream`.  Done once when the weights are loaded
+ * ("Day0 Adaptation and Performance Optimization ...", section 2: hardware-
+ * friendly weight layouts).  Returns DSA_ERR_INVALID_ARG for bad sizes or
+ * pointers, DSA_ERR_CUDA if the launch fails.
+ */
+DSA_API dsa_status indexer_prolog_pack(const void* w_proj, void* w_packed, int32_t H_I, int32_t D_I,
+                                       int32_t d_model, void* stream);
 
 /*
  * Bytes of workspace indexer_prolog needs for this shape (0 if the arguments

@@ -14,7 +14,8 @@ Entry points (same names as the C ABI):
         -> (idx, score, out, lse)
 
     indexer_prolog(batch, x, w_proj, k_gamma, eps, k_cache, k_scale=None, mx=False)
-        -> (q_idx, q_scale or None, w)   (also writes the tokens' keys into k_cache / k_scale)
+        -> (q_idx, q_scale or None, w)   (also writes the tokens' keys into k_cache / k_scale;
+        w_proj row-major, or prolog_pack_weights(w_proj, H_I, D_I) for weight streaming)
 
 Key formats: bf16 keys (k_scale None); e4m3 keys (uint8) with fp32 k_scale
 [nblk, 64, D_I/64]; MXFP8 queries and keys when q_scale is given: q_idx and
@@ -29,7 +30,7 @@ from dataclasses import dataclass
 from typing import Optional
 
 __all__ = ["Batch", "Workspace", "indexer_topk", "sparse_mla_attn", "dsa_decode", "indexer_prolog",
-           "get_status",
+           "prolog_pack_weights", "PackedWeights", "get_status",
            "DsaError", "library_path", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -77,7 +78,8 @@ class _Attn(ctypes.Structure):
 class _Prolog(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("w_proj", ctypes.c_void_p), ("k_gamma", ctypes.c_void_p),
                 ("eps", ctypes.c_float), ("d_model", ctypes.c_int32), ("H_I", ctypes.c_int32),
-                ("D_I", ctypes.c_int32), ("key_dtype", ctypes.c_int32), ("q_dtype", ctypes.c_int32)]
+                ("D_I", ctypes.c_int32), ("key_dtype", ctypes.c_int32), ("q_dtype", ctypes.c_int32),
+                ("w_layout", ctypes.c_int32)]
 
 
 def library_path() -> str:
@@ -119,6 +121,11 @@ def load_library():
                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                    ctypes.c_void_p]
     lib.indexer_prolog.restype = ctypes.c_int
+    lib.dsa_prolog_packed_bytes.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+    lib.dsa_prolog_packed_bytes.restype = ctypes.c_size_t
+    lib.indexer_prolog_pack.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int32, ctypes.c_void_p]
+    lib.indexer_prolog_pack.restype = ctypes.c_int
     lib.dsa_status_str.argtypes = [ctypes.c_int32]
     lib.dsa_status_str.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
@@ -380,6 +387,30 @@ def prolog_workspace(device=None) -> Workspace:
     return _prolog_ws[key]
 
 
+class PackedWeights:
+    """Prolog weights in the tile-packed layout (see prolog_pack_weights)."""
+
+    def __init__(self, data, H_I: int, D_I: int, d_model: int):
+        self.data, self.H_I, self.D_I, self.d_model = data, int(H_I), int(D_I), int(d_model)
+
+
+def prolog_pack_weights(w_proj, H_I: int, D_I: int, stream=None) -> PackedWeights:
+    """Tile-packed copy of the row-major prolog weights w_proj [H_I*D_I + D_I + H_I, d] (bf16):
+    each 128-row x 64-column block contiguous (done once, when the weights are loaded)."""
+    import torch
+    lib = load_library()
+    _check(w_proj, "w_proj", torch.bfloat16, 2, (H_I * D_I + D_I + H_I, None))
+    d = int(w_proj.shape[1])
+    n = lib.dsa_prolog_packed_bytes(int(H_I), int(D_I), d)
+    if n == 0:
+        raise DsaError(1, "dsa_prolog_packed_bytes")
+    out = torch.empty(n // 2, dtype=torch.bfloat16, device=w_proj.device)
+    rc = lib.indexer_prolog_pack(_ptr(w_proj), _ptr(out), int(H_I), int(D_I), d, _stream(stream))
+    if rc != 0:
+        raise DsaError(rc, "indexer_prolog_pack")
+    return PackedWeights(out, H_I, D_I, d)
+
+
 def indexer_prolog(batch: Batch, x, w_proj, k_gamma, eps: float, k_cache, k_scale=None, mx: bool = False, *,
                    H_I: Optional[int] = None, q_out=None, q_scale_out=None, w_out=None,
                    workspace: Optional[Workspace] = None, stream=None):
@@ -391,14 +422,20 @@ def indexer_prolog(batch: Batch, x, w_proj, k_gamma, eps: float, k_cache, k_scal
     import torch
     lib = load_library()
     _check(x, "x", torch.bfloat16, 2)
-    _check(w_proj, "w_proj", torch.bfloat16, 2, (None, x.shape[1]))
     _check(k_gamma, "k_gamma", torch.float32, 1)
     T, d = x.shape
     D_I = int(k_gamma.shape[0])
-    n_out = int(w_proj.shape[0])
-    H_I = (n_out - D_I) // (D_I + 1) if H_I is None else int(H_I)
-    if H_I * D_I + D_I + H_I != n_out:
-        raise ValueError(f"w_proj has {n_out} rows; H_I*D_I + D_I + H_I rows are needed")
+    if isinstance(w_proj, PackedWeights):
+        if w_proj.D_I != D_I or w_proj.d_model != d:
+            raise ValueError("packed weights were made for another D_I or d_model")
+        H_I, w_ptr, layout = w_proj.H_I, _ptr(w_proj.data), 1
+    else:
+        _check(w_proj, "w_proj", torch.bfloat16, 2, (None, x.shape[1]))
+        n_out = int(w_proj.shape[0])
+        H_I = (n_out - D_I) // (D_I + 1) if H_I is None else int(H_I)
+        if H_I * D_I + D_I + H_I != n_out:
+            raise ValueError(f"w_proj has {n_out} rows; H_I*D_I + D_I + H_I rows are needed")
+        w_ptr, layout = _ptr(w_proj), 0
     if mx:
         _check(k_cache, "k_cache", torch.uint8, 3, (None, 64, D_I))
         if k_scale is None:
@@ -419,7 +456,7 @@ def indexer_prolog(batch: Batch, x, w_proj, k_gamma, eps: float, k_cache, k_scal
         q_scale_out = torch.empty((T, H_I, D_I // 32), dtype=torch.uint8, device=dev)
     if w_out is None:
         w_out = torch.empty((T, H_I), dtype=torch.float32, device=dev)
-    pr = _Prolog(_ptr(x), _ptr(w_proj), _ptr(k_gamma), float(eps), int(d), H_I, D_I, kt, qt)
+    pr = _Prolog(_ptr(x), w_ptr, _ptr(k_gamma), float(eps), int(d), H_I, D_I, kt, qt, layout)
     cb = batch.c(T)
     ws = workspace if workspace is not None else prolog_workspace(dev)
     need = lib.dsa_prolog_workspace_size(ctypes.byref(cb), ctypes.byref(pr))

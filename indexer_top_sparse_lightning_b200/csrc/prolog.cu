@@ -19,7 +19,7 @@ constexpr size_t kProlStatusBytes = 256;
 constexpr int kGroupM = 16;
 
 struct ProlPlan {
-    int bn = 0, MT = 0, NT = 0, S = 1, KB = 0, units = 0, grid = 0, smem = 0;
+    int bn = 0, MT = 0, NT = 0, S = 1, Sk = 1, mk = 0, KB = 0, units = 0, grid = 0, smem = 0;
     size_t counters_off = 0, partials_off = 0, ws = 0;
 };
 
@@ -33,36 +33,34 @@ int prolog_smem(int bn) {
 }
 
 // Token tile: the smallest of 32/64/128/256 that covers T (256 beyond).
-// Splits: with fewer tiles than SMs, the K range is split S ways so that the
-// units fill whole waves of the SMs (each split keeps at least 4 k-blocks).
-ProlPlan plan_prolog(int T, int d, int n_out, int sms) {
+// Splits: with fewer tiles than SMs, the K range is split S ways, S the largest
+// count whose units still fit one wave of the SMs (one unit per CTA, so the
+// weights stream at full depth and each tile's partials are added once; each
+// split keeps at least 4 k-blocks, at most 16 splits).  In such a single-wave
+// plan the row tile holding the key rows takes twice as many splits when they
+// still fit: its epilogue is the longest, and shorter streaming hides it.
+ProlPlan plan_prolog(int T, int d, int n_out, int HD, int sms) {
     ProlPlan pl;
     pl.bn = T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256;
     pl.MT = (n_out + 127) / 128;
     pl.NT = (T + pl.bn - 1) / pl.bn;
     pl.KB = (d + 63) / 64;
+    pl.mk = HD / 128;
     const int64_t tiles = (int64_t)pl.MT * pl.NT;
-    auto eff = [&](int s) {
-        const int64_t u = tiles * s;
-        const int64_t waves = (u + sms - 1) / sms;
-        return (double)u / (double)(waves * sms);
-    };
-    int best = 1;
-    double best_eff = eff(1);
-    const int smax = pl.KB / 4 < 16 ? pl.KB / 4 : 16;
-    if (best_eff < 0.85)
-        for (int s = 2; s <= smax; ++s)
-            if (eff(s) > best_eff + 0.02) {
-                best = s;
-                best_eff = eff(s);
-            }
-    pl.S = best;
-    pl.units = (int)(tiles * pl.S);
+    const int smax = pl.KB / 4 < 16 ? (pl.KB / 4 < 1 ? 1 : pl.KB / 4) : 16;
+    int64_t s = tiles < sms ? sms / tiles : 1;
+    if (s > smax) s = smax;
+    if (s < 1) s = 1;
+    pl.S = (int)s;
+    pl.Sk = pl.S;
+    if (tiles < sms && 2 * pl.S <= smax && (tiles - pl.NT) * pl.S + (int64_t)pl.NT * 2 * pl.S <= sms) pl.Sk = 2 * pl.S;
+    pl.units = (int)((tiles - pl.NT) * pl.S + (int64_t)pl.NT * pl.Sk);
     pl.grid = pl.units < sms ? pl.units : sms;
     pl.smem = prolog_smem(pl.bn);
+    const int smx = pl.S > pl.Sk ? pl.S : pl.Sk;
     pl.counters_off = kProlStatusBytes;
     pl.partials_off = pl.counters_off + align256((size_t)tiles * 4);
-    pl.ws = pl.partials_off + (pl.S > 1 ? (size_t)pl.S * (size_t)tiles * (size_t)pl.bn * 128 * 4 : 0);
+    pl.ws = pl.partials_off + (smx > 1 ? (size_t)smx * (size_t)tiles * (size_t)pl.bn * 128 * 4 : 0);
     return pl;
 }
 
@@ -82,6 +80,7 @@ dsa_status check_prolog(const dsa_batch* bt, const dsa_prolog_inputs* pr) {
     if (pr->q_dtype != DSA_Q_BF16 && pr->q_dtype != DSA_Q_MXFP8) return DSA_ERR_INVALID_ARG;
     if ((pr->q_dtype == DSA_Q_MXFP8) != (pr->key_dtype == DSA_KEY_MXFP8)) return DSA_ERR_INVALID_ARG;
     if (!(pr->eps >= 0.0f)) return DSA_ERR_INVALID_ARG;
+    if (pr->w_layout != DSA_W_ROW_MAJOR && pr->w_layout != DSA_W_TILE_PACKED) return DSA_ERR_INVALID_ARG;
     if (!aligned(pr->x, 16) || !aligned(pr->w_proj, 16) || !aligned(pr->k_gamma, 4)) return DSA_ERR_INVALID_ARG;
     return DSA_OK;
 }
@@ -91,7 +90,15 @@ dsa_status launch_prolog(const dsa_batch* bt, const dsa_prolog_inputs* pr, const
                          cudaStream_t stream) {
     const int n_out = p.n_out;
     CUtensorMap tm_w, tm_x;
-    {
+    if (pr->w_layout == DSA_W_TILE_PACKED) {
+        // [MT*KB blocks][128 rows][64 columns]: one box is one 16 KB block
+        const uint64_t dims[3] = {64, 128, (uint64_t)pl.MT * pl.KB};
+        const uint64_t strides[2] = {64 * 2, 128 * 64 * 2};
+        const uint32_t box[3] = {64, 128, 1};
+        if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pr->w_proj, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return fail(DSA_ERR_CUDA, "prolog weight tensor map encoding failed");
+    } else {
         const uint64_t dims[2] = {(uint64_t)pr->d_model, (uint64_t)n_out};
         const uint64_t strides[1] = {(uint64_t)pr->d_model * 2};
         const uint32_t box[2] = {64, 128};
@@ -124,12 +131,36 @@ dsa_status launch_prolog(const dsa_batch* bt, const dsa_prolog_inputs* pr, const
 
 extern "C" {
 
+DSA_API size_t dsa_prolog_packed_bytes(int32_t H_I, int32_t D_I, int32_t d_model) {
+    if (H_I < 1 || D_I < 1 || d_model < 8 || d_model % 8 != 0) return 0;
+    const int64_t n_out = (int64_t)H_I * D_I + D_I + H_I;
+    return (size_t)((n_out + 127) / 128) * (size_t)((d_model + 63) / 64) * 128 * 64 * 2;
+}
+
+DSA_API dsa_status indexer_prolog_pack(const void* w_proj, void* w_packed, int32_t H_I, int32_t D_I, int32_t d_model,
+                                       void* stream) {
+    const size_t bytes = dsa_prolog_packed_bytes(H_I, D_I, d_model);
+    if (!bytes || !w_proj || !w_packed) return fail(DSA_ERR_INVALID_ARG, "indexer_prolog_pack: invalid arguments");
+    if (!aligned(w_proj, 16) || !aligned(w_packed, 16))
+        return fail(DSA_ERR_INVALID_ARG, "indexer_prolog_pack: pointers must be 16-byte aligned");
+    const DevInfo di = dev_info();
+    if (di.sms < 1) return fail(DSA_ERR_CUDA, "indexer_prolog_pack: no device");
+    const int n_out = H_I * D_I + D_I + H_I;
+    const int64_t chunks = (int64_t)(bytes / 16);
+    int64_t blocks = (chunks + 255) / 256;
+    if (blocks > (int64_t)di.sms * 16) blocks = (int64_t)di.sms * 16;
+    prolog_pack_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(w_proj), static_cast<uint4*>(w_packed), n_out, d_model, (d_model + 63) / 64, chunks);
+    if (cudaError_t e = cudaGetLastError()) return fail(DSA_ERR_CUDA, "indexer_prolog_pack launch", e);
+    return DSA_OK;
+}
+
 DSA_API size_t dsa_prolog_workspace_size(const dsa_batch* batch, const dsa_prolog_inputs* pr) {
     if (check_prolog(batch, pr) != DSA_OK) return 0;
     const DevInfo di = dev_info();
     if (di.sms < 1) return 0;
     const int n_out = pr->H_I * pr->D_I + pr->D_I + pr->H_I;
-    return plan_prolog(batch->num_tokens, pr->d_model, n_out, di.sms).ws;
+    return plan_prolog(batch->num_tokens, pr->d_model, n_out, pr->H_I * pr->D_I, di.sms).ws;
 }
 
 DSA_API dsa_status indexer_prolog(const dsa_batch* batch, const dsa_prolog_inputs* pr, void* q_out,
@@ -145,7 +176,7 @@ DSA_API dsa_status indexer_prolog(const dsa_batch* batch, const dsa_prolog_input
     const DevInfo di = dev_info();
     if (di.sms < 1) return fail(DSA_ERR_CUDA, "indexer_prolog: no device");
     const int n_out = pr->H_I * pr->D_I + pr->D_I + pr->H_I;
-    const ProlPlan pl = plan_prolog(batch->num_tokens, pr->d_model, n_out, di.sms);
+    const ProlPlan pl = plan_prolog(batch->num_tokens, pr->d_model, n_out, pr->H_I * pr->D_I, di.sms);
     if (!workspace || workspace_bytes < pl.ws || !aligned(workspace, 256))
         return fail(DSA_ERR_WORKSPACE, "indexer_prolog: workspace missing, too small or not 256-byte aligned");
     if (pl.smem > di.max_smem) return fail(DSA_ERR_UNSUPPORTED, "indexer_prolog: shared memory");
@@ -179,10 +210,13 @@ DSA_API dsa_status indexer_prolog(const dsa_batch* batch, const dsa_prolog_input
     p.MT = pl.MT;
     p.NT = pl.NT;
     p.S = pl.S;
+    p.Sk = pl.Sk;
+    p.mk = pl.mk;
     p.KB = pl.KB;
     p.units = pl.units;
     p.group_m = kGroupM;
     p.evict_w = pl.NT == 1;
+    p.w_packed = pr->w_layout == DSA_W_TILE_PACKED;
     p.eps = pr->eps;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     switch (pl.bn) {

@@ -49,23 +49,25 @@ struct PrologParams {
     uint8_t* k_scale_e8;         // [num_blocks*64, D_I/32] (MXFP8 keys), else null
     uint32_t* status;
     uint32_t* counters;          // [tiles] split arrivals (zero between launches)
-    float* partials;             // [S][tiles][BN][128] fp32 partial tiles (S > 1)
+    float* partials;             // [max(S, Sk)][tiles][BN][128] fp32 partial tiles (split tiles)
     int32_t T, H_I, D_I, HD, n_out;
     int32_t B, max_blocks, num_blocks;
     int32_t MT, NT, S, KB, units, group_m;
+    int32_t mk, Sk;              // the row tile holding the key rows, and its split count
     int32_t evict_w;             // weights are read once: stream them with an evict-first hint
+    int32_t w_packed;            // weights in the tile-packed layout (one 16 KB block per row tile and k-block)
     float eps;
 };
 
 struct PrologMisc {
-    uint64_t full[8], empty[8], tfull[2], tempty[2], drain;
+    uint64_t full[8], empty[8], tfull[2], tempty[2], drain, pbar;
     uint32_t tmem_base;
     int abort;
     int last;
     int pad_;
     uint64_t wait_ns;
-    float red_ss[2][4][32];      // key sum of squares per (warp, token column), double-buffered by chunk
-    float red_am[2][4][32];      // key amax per (warp, token column) for the per-64 fp8 scale
+    float red_ss[2][4][8];       // key sum of squares per (warp, token column), double-buffered by sub-chunk
+    float red_am[2][4][8];       // key amax per (warp, token column) for the per-64 fp8 scale
     int64_t row[256];            // key-cache row of each token column (-1: none)
 };
 
@@ -88,23 +90,40 @@ struct PrologCfg {
 
 __device__ __forceinline__ void prolog_status(uint32_t* status, uint32_t code) { atomicCAS(status, 0u, code); }
 
-// Unit u -> (row tile, token tile, split, k-block range).  Splits of one tile
-// are consecutive units; tiles go in groups of group_m row tiles, token tile
-// slowest inside a group, so that the CTAs running at one time share their
-// weight and token tiles in L2.
+// Unit u -> (row tile, token tile, split, splits of that tile, k-block range).
+// The row tile holding the key rows (mk) may be split more ways (Sk) than the
+// others (S): its epilogue (RMS norm, scattered cache-row stores) is the
+// longest, so in a single-wave plan its units stream fewer k-blocks and its
+// epilogue overlaps the other tiles' streaming.  Its units come first; the
+// others follow with their splits consecutive, in groups of group_m row tiles,
+// token tile slowest inside a group, so that the CTAs running at one time
+// share their weight and token tiles in L2.
 __device__ __forceinline__ void prolog_unit(const PrologParams& p, int u, int& tile, int& mt, int& nt, int& ks,
-                                            int& kb0, int& kb1) {
-    ks = u % p.S;
-    tile = u / p.S;
-    const int per_group = p.group_m * p.NT;
-    const int g = tile / per_group;
-    const int r = tile - g * per_group;
-    int gm = p.MT - g * p.group_m;
-    if (gm > p.group_m) gm = p.group_m;
-    mt = g * p.group_m + r % gm;
-    nt = r / gm;
-    kb0 = (int)((int64_t)ks * p.KB / p.S);
-    kb1 = (int)((int64_t)(ks + 1) * p.KB / p.S);
+                                            int& ns, int& kb0, int& kb1) {
+    const int nk = p.NT * p.Sk;
+    if (u < nk) {
+        ns = p.Sk;
+        ks = u % p.Sk;
+        nt = u / p.Sk;
+        mt = p.mk;
+    } else {
+        u -= nk;
+        ns = p.S;
+        ks = u % p.S;
+        const int t = u / p.S;                // among the row tiles other than mk
+        const int rows = p.MT - 1;
+        const int per_group = p.group_m * p.NT;
+        const int g = t / per_group;
+        const int r = t - g * per_group;
+        int gm = rows - g * p.group_m;
+        if (gm > p.group_m) gm = p.group_m;
+        mt = g * p.group_m + r % gm;
+        if (mt >= p.mk) ++mt;
+        nt = r / gm;
+    }
+    tile = mt * p.NT + nt;
+    kb0 = (int)((int64_t)ks * p.KB / ns);
+    kb1 = (int)((int64_t)(ks + 1) * p.KB / ns);
 }
 
 // Key-cache row of query token t: its position is seq_len - nq + (t - first
@@ -183,6 +202,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
             mbar_init(&m->tempty[i], Cfg::EPI_THREADS);
         }
         mbar_init(&m->drain, 1);
+        mbar_init(&m->pbar, 1);
         m->abort = 0;
         m->last = 0;
         // status area word 1: wait limit in microseconds (0: the default)
@@ -212,8 +232,8 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-                int tile, mt, nt, ks, kb0, kb1;
-                prolog_unit(p, u, tile, mt, nt, ks, kb0, kb1);
+                int tile, mt, nt, ks, ns, kb0, kb1;
+                prolog_unit(p, u, tile, mt, nt, ks, ns, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % Cfg::NS;
                     if (!mbar_wait(&m->empty[s], ((it / Cfg::NS) & 1) ^ 1, abort, wlim)) { ok = false; break; }
@@ -221,8 +241,15 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                     // rows or columns past the tensor's edge (last row tile, last token
                     // tile, a ragged last k-block) are filled with zeros by the copy
                     mbar_arrive_expect_tx(&m->full[s], Cfg::STAGE_BYTES);
-                    if (p.evict_w) tma_load_2d_hint(st, &tm_w, &m->full[s], kb * 64, mt * 128, pol);
-                    else tma_load_2d(st, &tm_w, &m->full[s], kb * 64, mt * 128);
+                    if (p.w_packed) {
+                        // block (mt, kb) of the packed weights: 16 KB contiguous
+                        if (p.evict_w) tma_load_3d_hint(st, &tm_w, &m->full[s], 0, 0, mt * p.KB + kb, pol);
+                        else tma_load_3d(st, &tm_w, &m->full[s], 0, 0, mt * p.KB + kb);
+                    } else if (p.evict_w) {
+                        tma_load_2d_hint(st, &tm_w, &m->full[s], kb * 64, mt * 128, pol);
+                    } else {
+                        tma_load_2d(st, &tm_w, &m->full[s], kb * 64, mt * 128);
+                    }
                     tma_load_2d(st + Cfg::A_BYTES, &tm_x, &m->full[s], kb * 64, nt * BN);
                 }
             }
@@ -240,8 +267,8 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
             int lu = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x, ++lu) {
-                int tile, mt, nt, ks, kb0, kb1;
-                prolog_unit(p, u, tile, mt, nt, ks, kb0, kb1);
+                int tile, mt, nt, ks, ns, kb0, kb1;
+                prolog_unit(p, u, tile, mt, nt, ks, ns, kb0, kb1);
                 const int buf = lu & 1;
                 if (!mbar_wait(&m->tempty[buf], ((lu >> 1) & 1) ^ 1, abort, wlim)) { ok = false; break; }
                 tc_fence_after();
@@ -275,8 +302,8 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
         const int key_fp8_groups = p.k_scale_f32 != nullptr;
         int lu = 0;
         for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++lu) {
-            int tile, mt, nt, ks, kb0, kb1;
-            prolog_unit(p, u, tile, mt, nt, ks, kb0, kb1);
+            int tile, mt, nt, ks, ns, kb0, kb1;
+            prolog_unit(p, u, tile, mt, nt, ks, ns, kb0, kb1);
             const int buf = lu & 1;
             const int row0 = mt * 128;
             const int base = row0 + warp * 32;          // first output row of this warp
@@ -304,21 +331,22 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
             const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * BN;
             const int r_in = warp * 32 + lane;
             bool fin = true;
-            if (p.S > 1) {
-                float* mine = p.partials + ((int64_t)ks * p.MT * p.NT + tile) * (BN * 128);
+            if (ns > 1) {
+                // this split's partial tile, [BN columns][128 rows] fp32
+                float* mine = p.partials + ((int64_t)ks * p.MT * p.NT + tile) * (BN * 128) + r_in;
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(tb + c0, r);
+                for (int c0 = 0; c0 < BN; c0 += 8) {
+                    uint32_t r[8];
+                    tmem_ld8(tb + c0, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) __stcg(mine + (c0 + j) * 128 + r_in, __uint_as_float(r[j]));
+                    for (int j = 0; j < 8; ++j) __stcg(mine + (c0 + j) * 128, __uint_as_float(r[j]));
                 }
                 __threadfence();
                 named_bar_sync(3, Cfg::EPI_THREADS);
                 if (et == 0) {
                     const uint32_t old = atomicAdd(p.counters + tile, 1u);
-                    const int last = old == (uint32_t)(p.S - 1);
+                    const int last = old == (uint32_t)(ns - 1);
                     if (last) p.counters[tile] = 0u;     // ready for the next launch
                     __threadfence();
                     m->last = last;
@@ -326,59 +354,131 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                 named_bar_sync(3, Cfg::EPI_THREADS);
                 fin = m->last != 0;
             }
-            if (fin) {
+            if (fin && ns > 1) {
+                // Add the S partials in split order into this CTA's accumulator (TMEM), then run
+                // the epilogue from TMEM as for one split.  When every CTA has one unit (the
+                // split plan makes it so) the stage ring is idle by now: the other splits'
+                // tiles come in by bulk copies and are added from shared memory.  Otherwise
+                // they are read from L2, four splits' loads in flight.
+                const int64_t tsz = (int64_t)BN * 128;    // floats per partial tile
+                const int64_t tiles = (int64_t)p.MT * p.NT;
+                const bool staged = (int)gridDim.x >= p.units &&
+                                    (ns - 1) * BN * 512 <= Cfg::NS * Cfg::STAGE_BYTES;
+                const float* stg = reinterpret_cast<const float*>(smem);
+                bool ok = true;
+                if (staged) {
+                    if (et == 0) {
+                        fence_proxy_async_global();
+                        mbar_arrive_expect_tx(&m->pbar, (uint32_t)((ns - 1) * BN * 512));
+                        for (int s = 0, k = 0; s < ns; ++s) {
+                            if (s == ks) continue;
+                            bulk_load(smem + (int64_t)k * BN * 512, p.partials + ((int64_t)s * tiles + tile) * tsz,
+                                      BN * 512, &m->pbar);
+                            ++k;
+                        }
+                    }
+                    ok = mbar_wait(&m->pbar, 0, abort, wlim);
+                }
+                if (!named_bar_and(2, Cfg::EPI_THREADS, ok)) {
+                    m->abort = 1;
+                    // no copy may still be writing shared memory when the CTA exits
+                    if (et == 0) {
+                        volatile int no_abort = 0;
+                        mbar_wait(&m->pbar, 0, &no_abort, wlim);
+                    }
+                    break;
+                }
 #pragma unroll 1
-                for (int c0 = 0, cc = 0; c0 < BN; c0 += 32, ++cc) {
-                    uint32_t r[32];
-                    tmem_ld32(tb + c0, r);
+                for (int c0 = 0; c0 < BN; c0 += 8) {
+                    uint32_t r[8];
+                    tmem_ld8(tb + c0, r);
                     tmem_wait_ld();
-                    float v[32];
-                    if (p.S > 1) {
+                    float v[8];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+                    for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+                    if (staged) {
 #pragma unroll 1
-                        for (int s = 0; s < p.S; ++s) {
+                        for (int s = 0; s < ns; ++s) {
                             if (s == ks) {
 #pragma unroll
-                                for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(r[j]);
+                                for (int j = 0; j < 8; ++j) v[j] += __uint_as_float(r[j]);
                             } else {
-                                const float* ps = p.partials + ((int64_t)s * p.MT * p.NT + tile) * (BN * 128);
+                                const float* ps = stg + (s - (s > ks ? 1 : 0)) * tsz + c0 * 128 + r_in;
 #pragma unroll
-                                for (int j = 0; j < 32; ++j) v[j] += __ldcg(ps + (c0 + j) * 128 + r_in);
+                                for (int j = 0; j < 8; ++j) v[j] += ps[j * 128];
                             }
                         }
                     } else {
+                        const float* part0 = p.partials + tile * tsz + c0 * 128 + r_in;
+#pragma unroll 1
+                        for (int s0 = 0; s0 < ns; s0 += 4) {
+                            float a[4][8];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+                            for (int q = 0; q < 4; ++q) {
+                                const int s = s0 + q;
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    a[q][j] = (s < ns && s != ks) ? __ldcg(part0 + s * tiles * tsz + j * 128)
+                                                                   : __uint_as_float(r[j]);
+                            }
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                if (s0 + q < ns)
+#pragma unroll
+                                    for (int j = 0; j < 8; ++j) v[j] += a[q][j];
+                        }
                     }
+                    uint32_t o[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) o[j] = __float_as_uint(v[j]);
+                    tmem_st8(tb + c0, o);
+                }
+                tmem_wait_st();
+            }
+            if (fin) {
+                // The epilogue walks the tile in sub-chunks of 8 token columns with rolled
+                // loops: its code runs once per tile (the key tile on one CTA only), so it is
+                // kept small enough to stay in the instruction cache.
+                const int kw0 = (p.HD - row0) / 32;      // first warp holding key rows (has_k)
+                const float g = kw ? __ldg(p.gamma + (base - p.HD) + lane) : 0.0f;
+#pragma unroll 1
+                for (int c0 = 0, cc = 0; c0 < BN; c0 += 8, ++cc) {
+                    uint32_t r[8];
+                    tmem_ld8(tb + c0, r);
+                    tmem_wait_ld();
+                    float v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[j]);
                     const int t0 = nt * BN + c0;
                     const int rb = cc & 1;
                     if (has_k) {
                         // key rows: RMS normalization over the D_I rows of each token column
-                        const int kw0 = (p.HD - row0) / 32;
                         if (kw) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
+                            for (int j = 0; j < 8; ++j) {
                                 const float s2 = warp_sum(v[j] * v[j]);
                                 if (lane == 0) m->red_ss[rb][warp][j] = s2;
                             }
                         }
                         named_bar_sync(4, Cfg::EPI_THREADS);
                         if (kw) {
-                            const float g = __ldg(p.gamma + (base - p.HD) + lane);
-                            const int nkw = p.D_I / 32;
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) {
+                            // lane j totals column j over the key warps (in warp order) and
+                            // forms its factor; the factors are then broadcast
+                            float fac = 0.0f;
+                            if (lane < 8) {
                                 float ss = 0.0f;
-                                for (int w = 0; w < nkw; ++w) ss += m->red_ss[rb][kw0 + w][j];
-                                const float rr = rsqrtf(ss / (float)p.D_I + p.eps);
-                                v[j] = v[j] * rr * g;
+#pragma unroll
+                                for (int w = 0; w < 4; ++w)
+                                    if (w < p.D_I / 32) ss += m->red_ss[rb][kw0 + w][lane];
+                                fac = rsqrtf(ss / (float)p.D_I + p.eps);
                             }
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) v[j] = v[j] * __shfl_sync(0xffffffffu, fac, j) * g;
                         }
                         if (key_fp8_groups) {
                             if (kw) {
 #pragma unroll
-                                for (int j = 0; j < 32; ++j) {
+                                for (int j = 0; j < 8; ++j) {
                                     const float a = warp_max(fabsf(v[j]));
                                     if (lane == 0) m->red_am[rb][warp][j] = a;
                                 }
@@ -390,7 +490,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                         // ------------------------------------------------ queries
                         if (p.q_codes) {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
+                            for (int j = 0; j < 8; ++j) {
                                 const int e = mx_exponent(warp_max(fabsf(v[j])));
                                 const uint8_t c = e4m3_code(v[j] * mx_inv_scale(e));
                                 const int t = t0 + j;
@@ -401,7 +501,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                             }
                         } else {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
+                            for (int j = 0; j < 8; ++j) {
                                 const int t = t0 + j;
                                 if (t < p.T) p.q_bf16[(int64_t)t * p.HD + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
                             }
@@ -409,23 +509,36 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                     } else if (kw) {
                         // ------------------------------------------------ keys into the paged cache
                         const int i = base - p.HD + lane;     // element of the key
+                        const long long rowl = lane < 8 ? (long long)m->row[c0 + lane] : -1ll;
+                        if (p.k_bf16) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int64_t row = m->row[c0 + j];
-                            if (p.k_bf16) {
+                            for (int j = 0; j < 8; ++j) {
+                                const int64_t row = __shfl_sync(0xffffffffu, rowl, j);
                                 if (row >= 0) p.k_bf16[row * p.D_I + i] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
-                            } else if (key_fp8_groups) {
-                                // the two warps of this 64-element scale group
-                                const int w0 = (p.HD - row0) / 32 + ((base - p.HD) / 64) * 2;
-                                const float a = fmaxf(m->red_am[rb][w0][j], m->red_am[rb][w0 + 1][j]);
-                                const float sc = a > 0.0f ? a / 448.0f : 1.0f;
+                            }
+                        } else if (key_fp8_groups) {
+                            // the two warps of this 64-element scale group
+                            const int w0 = kw0 + ((base - p.HD) / 64) * 2;
+                            const bool first = ((base - p.HD) & 63) == 0;
+                            float scl = 1.0f;
+                            if (lane < 8) {
+                                const float a = fmaxf(m->red_am[rb][w0][lane], m->red_am[rb][w0 + 1][lane]);
+                                scl = a > 0.0f ? a / 448.0f : 1.0f;
+                            }
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int64_t row = __shfl_sync(0xffffffffu, rowl, j);
+                                const float sc = __shfl_sync(0xffffffffu, scl, j);
                                 const uint8_t c = e4m3_code(v[j] / sc);
                                 if (row >= 0) {
                                     p.k_codes[row * p.D_I + i] = c;
-                                    if (lane == 0 && ((base - p.HD) & 63) == 0)
-                                        p.k_scale_f32[row * (p.D_I / 64) + (base - p.HD) / 64] = sc;
+                                    if (lane == 0 && first) p.k_scale_f32[row * (p.D_I / 64) + (base - p.HD) / 64] = sc;
                                 }
-                            } else {
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int64_t row = __shfl_sync(0xffffffffu, rowl, j);
                                 const int e = mx_exponent(warp_max(fabsf(v[j])));
                                 const uint8_t c = e4m3_code(v[j] * mx_inv_scale(e));
                                 if (row >= 0) {
@@ -438,7 +551,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                         // ------------------------------------------------ head weights
                         const int h = n - p.HD - p.D_I;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
+                        for (int j = 0; j < 8; ++j) {
                             const int t = t0 + j;
                             if (t < p.T) p.w_out[(int64_t)t * p.H_I + h] = v[j];
                         }
@@ -458,6 +571,26 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
     if (threadIdx.x == 0 && m->abort) prolog_status(p.status, kStTimeout);
+}
+
+// Tile-packed weight layout: block (mt, kb) -- rows 128*mt .. 128*mt+127 and
+// columns 64*kb .. 64*kb+63 of the row-major [n_out, d] matrix, zero past its
+// edges -- is stored row-major [128][64] at element offset (mt*KB + kb)*8192.
+// One thread per 16-byte chunk of the packed array.
+__global__ void __launch_bounds__(256) prolog_pack_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                          int n_out, int d, int KB, int64_t chunks) {
+    for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < chunks; c += (int64_t)gridDim.x * blockDim.x) {
+        const int c8 = (int)(c & 7);                  // 8 chunks of 8 elements per 64-column row
+        const int r = (int)((c >> 3) & 127);
+        const int64_t blk = c >> 10;
+        const int kb = (int)(blk % KB);
+        const int mt = (int)(blk / KB);
+        const int row = mt * 128 + r;
+        const int col = kb * 64 + c8 * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row < n_out && col < d) v = src[((int64_t)row * d + col) / 8];   // d is a multiple of 8
+        dst[c] = v;
+    }
 }
 
 }  // namespace dsa

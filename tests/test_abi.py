@@ -103,3 +103,43 @@ def test_attention_rejects_bad_inputs(lib):
 def test_get_status_rejects_null(lib):
     v = ctypes.c_int32(0)
     assert lib.dsa_get_status(None, None, ctypes.byref(v)) == 1
+
+
+def _pr(**kw):
+    d = dict(x=16, w_proj=16, k_gamma=16, eps=1e-6, d_model=7168, H_I=64, D_I=128, key_dtype=0, q_dtype=0,
+             w_layout=0)
+    d.update(kw)
+    return dsa._Prolog(**d)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(H_I=12), 2), (dict(D_I=96), 2), (dict(d_model=100), 2), (dict(d_model=0), 2), (dict(key_dtype=5), 1),
+    (dict(q_dtype=1), 1), (dict(key_dtype=2), 1), (dict(eps=-1.0), 1), (dict(w_layout=2), 1), (dict(x=8), 1),
+    (dict(w_proj=None), 1), (dict(k_gamma=None), 1),
+])
+def test_prolog_rejects_bad_inputs(lib, bad, code):
+    rc = lib.indexer_prolog(ctypes.byref(_batch()), ctypes.byref(_pr(**bad)), 16, None, 16, 16, None, 256, 1 << 20,
+                            None)
+    assert rc == code
+    assert lib.dsa_prolog_workspace_size(ctypes.byref(_batch()), ctypes.byref(_pr(**bad))) == 0
+
+
+def test_prolog_rejects_missing_outputs(lib):
+    b, pr = ctypes.byref(_batch()), ctypes.byref(_pr())
+    assert lib.indexer_prolog(b, pr, None, None, 16, 16, None, 256, 1 << 20, None) == 1       # q_out
+    assert lib.indexer_prolog(b, pr, 16, None, None, 16, None, 256, 1 << 20, None) == 1       # w_out
+    assert lib.indexer_prolog(b, pr, 16, None, 16, None, None, 256, 1 << 20, None) == 1       # k_cache
+    fp8 = ctypes.byref(_pr(key_dtype=1))
+    assert lib.indexer_prolog(b, fp8, 16, None, 16, 16, None, 256, 1 << 20, None) == 1       # k_scale
+    mx = ctypes.byref(_pr(key_dtype=2, q_dtype=1))
+    assert lib.indexer_prolog(b, mx, 16, None, 16, 16, 16, 256, 1 << 20, None) == 1          # q_scale_out
+
+
+def test_prolog_packed_bytes(lib):
+    # ceil(n_out / 128) * ceil(d / 64) blocks of 128 x 64 bf16
+    assert lib.dsa_prolog_packed_bytes(64, 128, 7168) == 66 * 112 * 16384
+    assert lib.dsa_prolog_packed_bytes(8, 64, 200) == 5 * 4 * 16384
+    assert lib.dsa_prolog_packed_bytes(8, 64, 100) == 0
+    assert lib.indexer_prolog_pack(16, 16, 8, 64, 100, None) == 1
+    assert lib.indexer_prolog_pack(None, 16, 8, 64, 128, None) == 1
+    assert lib.indexer_prolog_pack(16, 24, 8, 64, 128, None) == 1

@@ -37,11 +37,13 @@ def _setup(seq_lens, nq, H_I, D_I, key_dtype, d, seed, int_inputs=False):
     return wl, pw
 
 
-def _run(wl, pw, tokens=None):
+def _run(wl, pw, packed=False):
     """Runs the prolog on the device; returns host copies of (q, q_scale, w, k_cache, k_scale)."""
     dd = W.to_device(wl, with_kv=False)
     x = torch.from_numpy(pw.x).view(torch.bfloat16).cuda()
     wt = torch.from_numpy(pw.wt).view(torch.bfloat16).cuda()
+    if packed:
+        wt = dsa.prolog_pack_weights(wt, pw.H_I, pw.D_I)
     g = torch.from_numpy(pw.gamma).cuda()
     mx = wl.key_dtype == "mxfp8"
     ws = dsa.Workspace()
@@ -143,10 +145,10 @@ def _assert_prolog(wl, pw, out, exact=False):
 
 @pytest.mark.parametrize("key_dtype", ["bf16", "mxfp8"])
 @pytest.mark.parametrize("H_I,D_I", [(8, 64), (16, 128)])
-@pytest.mark.parametrize("d", [200, 1024])
+@pytest.mark.parametrize("d", [200, 1024, 4096])
 def test_integer_inputs_queries_and_weights_bit_exact(key_dtype, H_I, D_I, d):
     # ragged batch (1, 5 and 2 new tokens); d_model 200 = three 64-blocks and a ragged 8,
-    # d_model 1024 = the contraction split across CTAs (few row tiles)
+    # d_model 1024 and 4096 = the contraction split 4 and 16 ways across CTAs (few row tiles)
     wl, pw = _setup([70, 130, 300], [1, 5, 2], H_I, D_I, key_dtype, d=d, seed=41, int_inputs=True)
     _assert_prolog(wl, pw, _run(wl, pw), exact=True)
 
@@ -161,6 +163,38 @@ def test_random_inputs_against_oracle(key_dtype, T, d):
     lens = [2048 + 64 * i + n for i, n in enumerate(nq)]
     wl, pw = _setup(lens, nq, 64, 128, key_dtype, d=d, seed=43 + T)
     _assert_prolog(wl, pw, _run(wl, pw))
+
+
+def _pack_host(wt, d):
+    """The tile-packed layout written out with numpy: 128 x 64 blocks, zeros past the edges."""
+    n_out = wt.shape[0]
+    MT, KB = -(-n_out // 128), -(-d // 64)
+    full = np.zeros((MT * 128, KB * 64), np.uint16)
+    full[:n_out, :d] = wt
+    return full.reshape(MT, 128, KB, 64).transpose(0, 2, 1, 3).reshape(-1)
+
+
+@pytest.mark.parametrize("H_I,D_I,d", [(8, 64, 200), (64, 128, 1024)])
+def test_pack_layout(H_I, D_I, d):
+    wl, pw = _setup([100], [1], H_I, D_I, "bf16", d=d, seed=61)
+    wt = torch.from_numpy(pw.wt).view(torch.bfloat16).cuda()
+    pk = dsa.prolog_pack_weights(wt, H_I, D_I)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(pk.data.view(torch.uint16).cpu().numpy(), _pack_host(pw.wt, d))
+
+
+@pytest.mark.parametrize("key_dtype", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("T,d", [(3, 200), (32, 1024), (300, 384)])
+def test_packed_weights_give_identical_outputs(key_dtype, T, d):
+    nb = min(4, T)
+    nq = [T // nb + (1 if i < T % nb else 0) for i in range(nb)]
+    wl, pw = _setup([4096] * nb, nq, 64, 128, key_dtype, d=d, seed=67 + T)
+    a = _run(wl, pw)
+    b = _run(wl, pw, packed=True)
+    for u, v in zip(a, b):
+        if u is not None:
+            np.testing.assert_array_equal(u, v)
+    _assert_prolog(wl, pw, b)
 
 
 def test_split_contraction_is_deterministic():
