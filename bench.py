@@ -367,12 +367,57 @@ def measure_prolog(dsa, dev, name, B, ctx, nq, steps, peak, tf_peak, packed=True
          "algorithmic_bytes": byts, "algorithmic_flops": flops, "gbs": gbs, "tflops": tfs,
          "l2": "flushed between launches (write then read of 2x L2)", "weights": "tile-packed" if packed else "row-major"}
     if T <= 256:
-        e["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak}
+        e["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": ncu_traffic("indexer_prolog_kernel") if name == "decode32" and packed else None}
     else:
         e["roofline"] = {"bound": "tensor", "achieved": tfs, "peak": tf_peak, "unit": "TFLOP/s", "frac": tfs / tf_peak}
     del x, wp, k_cache, scrub, ws
     torch.cuda.empty_cache()
     return e
+
+
+def cp_emulation(dsa, wl, d, ws, idx_ms, worlds=(2, 4, 8), reps=3):
+    """Zigzag context parallelism of the prefill indexer, emulated on one GPU: each rank's share
+    of the chunk (two pieces for zigzag, one range for the contiguous split) runs alone, timed
+    with CUDA events; a CP step would take the slowest rank's time plus the two all-gathers
+    (new keys, index lists), which one GPU cannot time."""
+    import numpy as np
+    import torch
+    from indexer_top_sparse_lightning_b200 import cp
+    n, seq_len = wl.T, int(wl.seq_lens[0])
+    dev = d["q_idx"].device
+    stream = torch.cuda.current_stream()
+    out = {}
+    for world in worlds:
+        e = {"ideal_ms": idx_ms / world}
+        for name, fn in (("zigzag", cp.zigzag_pieces), ("contiguous", cp.contiguous_pieces)):
+            times = []
+            for r in range(world):
+                lens, cu, toks = cp.local_batch(seq_len, n, fn(n, world, r))
+                t = torch.as_tensor(toks, device=dev)
+                q, w = d["q_idx"].index_select(0, t).contiguous(), d["w"].index_select(0, t).contiguous()
+                batch = dsa.Batch(torch.as_tensor(lens, device=dev), torch.as_tensor(cu, device=dev),
+                                  d["block_table"][:1].repeat(len(lens), 1).contiguous(), wl.num_blocks,
+                                  int(lens.max()), int(np.diff(cu).max()))
+                out_idx = torch.empty((len(toks), wl.K), dtype=torch.int32, device=dev)
+
+                def run():
+                    dsa.indexer_topk(batch, q, w, d["k_cache"], wl.K, k_scale=d["k_scale"], q_scale=d["q_scale"],
+                                     out_idx=out_idx, want_score=False, workspace=ws)
+                run()
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+                for a, b in ev:
+                    a.record(stream)
+                    run()
+                    b.record(stream)
+                torch.cuda.synchronize()
+                times.append(statistics.mean(a.elapsed_time(b) for a, b in ev))
+            e[name + "_rank_ms"] = times
+            e[name + "_max_rank_ms"] = max(times)
+        out[str(world)] = e
+    if dsa.get_status(ws) != 0:
+        raise RuntimeError("cp emulation: device reported an error")
+    return out
 
 
 def kernel_entry(wl, r, peak):
@@ -494,6 +539,8 @@ def run_ours(args, rank, world, local_rank):
                      "step_gbs": (xw.key_bytes() + xw.kv_bytes()) / (xr["ms_step"] * 1e-3) / 1e9,
                      "l2": "flushed between steps (write then read of 2x L2)" if xr["flush"] else "inputs larger than L2",
                      "kernels": kernel_entry(xw, xr, peak)}
+            if name == "prefill16k":
+                entry["cp_emulated"] = cp_emulation(dsa, xw, xr["d"], xr["ws"], xr["idx_ms"])
             extra[name] = entry
             del xr, xw
             torch.cuda.empty_cache()
