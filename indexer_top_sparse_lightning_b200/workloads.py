@@ -86,6 +86,7 @@ class Workload:
     planted: Optional[np.ndarray] = None   # sorted positions of a planted Top-K set
     seed: int = 0
     q_scale: Optional[np.ndarray] = None   # [T, H_I, D_I//32] uint8 (mxfp8 queries)
+    kv_scale: Optional[np.ndarray] = None  # [nblk, 64, 5] float32 (fp8 latent cache; kv holds e4m3 codes)
 
     @property
     def max_blocks(self) -> int:
@@ -183,6 +184,22 @@ def _quantize_fp8_groups(x: np.ndarray, group: int = 64):
     return codes.reshape(x.shape), scale
 
 
+def _quantize_fp8_tiles(x: np.ndarray, tile: int = 128):
+    """Per-row tiles of `tile` elements along the last axis (the last tile may be shorter):
+    scale = amax/448 (1 for an all-zero tile), e4m3 codes of x / scale."""
+    n = x.shape[-1]
+    nt = -(-n // tile)
+    codes = np.empty(x.shape, np.uint8)
+    scales = np.empty(x.shape[:-1] + (nt,), np.float32)
+    for i in range(nt):
+        g = x[..., i * tile:(i + 1) * tile]
+        amax = np.abs(g).max(axis=-1)
+        sc = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32)
+        scales[..., i] = sc
+        codes[..., i * tile:(i + 1) * tile] = encode_e4m3((g / sc[..., None]).astype(np.float32))
+    return codes, scales
+
+
 def _quantize_mx(x: np.ndarray):
     """MXFP8 encoding along the last axis, 32 contiguous elements per group: the
     shared scale is X = 2^(floor(log2 amax) - 8) (8 = the largest e4m3 exponent),
@@ -200,7 +217,7 @@ def _quantize_mx(x: np.ndarray):
 def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=128, K=2048,
                   key_dtype="bf16", int_inputs=False, w_dist="u8", shuffle=True,
                   planted_k: int = 0, planted_tail: bool = False, seed: int = 0,
-                  with_kv: bool = True) -> Workload:
+                  with_kv: bool = True, kv_dtype: str = "bf16") -> Workload:
     """Draw one synthetic step.
 
     seq_lens: per-sequence cached lengths (including the step's own tokens).
@@ -294,9 +311,13 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
         k_idx = codes.reshape(num_blocks, BLOCK, D_I)
         k_scale = scale.reshape(num_blocks, BLOCK, D_I // 64)
 
+    kv_scale = None
     if with_kv:
         q = _normal_bf16(seed, 6, (T, H, D_QK))
         kv = _normal_bf16(seed, 7, (num_blocks, BLOCK, D_QK))
+        if kv_dtype == "fp8":
+            # the same N(0,1) rows, stored as e4m3 codes with one fp32 scale per 128-element tile
+            kv, kv_scale = _quantize_fp8_tiles(bf16_bits_to_f32(kv), 128)
     else:
         q = np.zeros((T, H, D_QK), dtype=np.uint16)
         kv = np.zeros((0, BLOCK, D_QK), dtype=np.uint16)
@@ -304,7 +325,8 @@ def make_workload(name: str = "custom", *, seq_lens, nq=1, H_I=64, D_I=128, H=12
     return Workload(name=name, B=B, T=T, H_I=H_I, D_I=D_I, H=H, K=K, key_dtype=key_dtype,
                     seq_lens=seq_lens, cu_q=cu_q, block_table=table, num_blocks=num_blocks,
                     q_idx=q_idx, w=w, k_idx=k_idx, k_scale=k_scale, q=q, kv=kv,
-                    sm_scale=1.0 / math.sqrt(D_QK), planted=planted, seed=seed, q_scale=q_scale)
+                    sm_scale=1.0 / math.sqrt(D_QK), planted=planted, seed=seed, q_scale=q_scale,
+                    kv_scale=kv_scale)
 
 
 # The five workloads.  Seeds are 1000 + index.
@@ -393,5 +415,10 @@ def to_device(wl: Workload, device="cuda", with_kv: bool = True) -> dict:
         d["k_scale"] = t(wl.k_scale)
     if with_kv:
         d["q"] = t(wl.q, torch.bfloat16)
-        d["kv"] = t(wl.kv, torch.bfloat16)
+        if wl.kv_scale is not None:
+            d["kv"] = t(wl.kv)
+            d["kv_scale"] = t(wl.kv_scale)
+        else:
+            d["kv"] = t(wl.kv, torch.bfloat16)
+            d["kv_scale"] = None
     return d

@@ -48,7 +48,8 @@ class _AttnArgs(ctypes.Structure):
                 ("K", ctypes.c_int32), ("sm_scale", ctypes.c_double),
                 ("seq_lens", ctypes.c_void_p), ("cu_q", ctypes.c_void_p),
                 ("block_table", ctypes.c_void_p), ("max_blocks", ctypes.c_int32),
-                ("q", ctypes.c_void_p), ("kv", ctypes.c_void_p), ("idx", ctypes.c_void_p)]
+                ("q", ctypes.c_void_p), ("kv", ctypes.c_void_p), ("idx", ctypes.c_void_p),
+                ("kv_fp8", ctypes.c_int32), ("kv_scale", ctypes.c_void_p)]
 
 
 class _PrologArgs(ctypes.Structure):
@@ -191,12 +192,15 @@ def sparse_attn(wl, idx, tokens=None, sm_scale=None):
     n = int(tokens.shape[0])
     idx = _c(idx, np.int32)
     assert idx.shape == (wl.T, wl.K)
+    fp8 = getattr(wl, "kv_scale", None) is not None
     arrs = dict(seq_lens=_c(wl.seq_lens, np.int32), cu_q=_c(wl.cu_q, np.int32),
                 block_table=_c(wl.block_table, np.int32), q=_c(wl.q, np.uint16),
-                kv=_c(wl.kv, np.uint16))
+                kv=_c(wl.kv, np.uint8 if fp8 else np.uint16),
+                kv_scale=_c(wl.kv_scale, np.float32) if fp8 else None)
     args = _AttnArgs(wl.B, wl.T, wl.H, wl.K, float(wl.sm_scale if sm_scale is None else sm_scale),
                      _ptr(arrs["seq_lens"]), _ptr(arrs["cu_q"]), _ptr(arrs["block_table"]),
-                     wl.block_table.shape[1], _ptr(arrs["q"]), _ptr(arrs["kv"]), _ptr(idx))
+                     wl.block_table.shape[1], _ptr(arrs["q"]), _ptr(arrs["kv"]), _ptr(idx),
+                     1 if fp8 else 0, _ptr(arrs["kv_scale"]))
     o = np.empty((n, wl.H, 512), dtype=np.float64)
     lse = np.empty((n, wl.H), dtype=np.float64)
     lib.oracle_sparse_attn(ctypes.byref(args), _ptr(tokens), n, _ptr(o), _ptr(lse))

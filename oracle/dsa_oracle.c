@@ -268,9 +268,24 @@ typedef struct {
     const int32_t* block_table;
     int32_t max_blocks;
     const uint16_t* q;               /* [T, H, 576] bf16 bits */
-    const uint16_t* kv;              /* [nblk, 64, 576] bf16 bits */
+    const void* kv;                  /* [nblk, 64, 576] bf16 bits, or e4m3 codes (kv_fp8) */
     const int32_t* idx;              /* [T, K] logical positions, -1 = skip */
+    int32_t kv_fp8;                  /* 1: kv holds e4m3 codes with per-row tile scales */
+    const float* kv_scale;           /* [nblk, 64, 5] fp32: one scale per 128 elements of a row */
 } oracle_attn_args;
+
+/*
+ * Element d of latent cache row `row`.  FP8 latent cache ("Day0 Adaptation and
+ * Performance Optimization ...", section 4: FP8 KV cache quantized per token and
+ * per head in tiles of 128 elements; "Large Model Inference Acceleration ...",
+ * section 2.2): the 576-element row is cut into tiles of 128 (the last one, the
+ * RoPE part, has 64) and each tile has its own fp32 scale:
+ *     kv[row, d] = e4m3(code[row, d]) * scale[row, d / 128].
+ */
+static double kv_elem(const oracle_attn_args* a, int64_t row, int d) {
+    if (!a->kv_fp8) return bf16_to_f64(((const uint16_t*)a->kv)[row * ORACLE_DQK + d]);
+    return oracle_e4m3_to_f64(((const uint8_t*)a->kv)[row * ORACLE_DQK + d]) * (double)a->kv_scale[row * 5 + d / 128];
+}
 
 /*
  * Step 3 for the tokens listed: out_o [n_tokens, H, 512] double,
@@ -300,9 +315,8 @@ int oracle_sparse_attn(const oracle_attn_args* a, const int32_t* tokens, int n_t
             if (n == 0) { out_lse[(int64_t)i * a->H + g] = -INFINITY; continue; }
             double m = -INFINITY;
             for (int j = 0; j < n; j++) {
-                const uint16_t* kr = a->kv + rows[j] * ORACLE_DQK;
                 double dot = 0.0;
-                for (int d = 0; d < ORACLE_DQK; d++) dot += bf16_to_f64(qg[d]) * bf16_to_f64(kr[d]);
+                for (int d = 0; d < ORACLE_DQK; d++) dot += bf16_to_f64(qg[d]) * kv_elem(a, rows[j], d);
                 logit[j] = a->sm_scale * dot;
                 if (logit[j] > m) m = logit[j];
             }
@@ -310,8 +324,7 @@ int oracle_sparse_attn(const oracle_attn_args* a, const int32_t* tokens, int n_t
             for (int j = 0; j < n; j++) den += exp(logit[j] - m);
             for (int j = 0; j < n; j++) {
                 double p = exp(logit[j] - m) / den;
-                const uint16_t* kr = a->kv + rows[j] * ORACLE_DQK;
-                for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d]);
+                for (int d = 0; d < ORACLE_DV; d++) o[d] += p * kv_elem(a, rows[j], d);
             }
             out_lse[(int64_t)i * a->H + g] = m + log(den);
         }

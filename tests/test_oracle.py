@@ -16,6 +16,7 @@
   the e4m3 encoder against torch's float8_e4m3fn cast (ties and saturation
   included), MX and per-64 encodings against their scale rules and error bounds.
 """
+import dataclasses
 import json
 import math
 import os
@@ -190,6 +191,44 @@ def test_hand_softmax_two_rows():
     assert abs(o[0, 0, 1] - g["o1"]) < 1e-15
     assert np.all(o[0, 0, 2:] == 0.0)
     assert abs(lse[0, 0] - g["lse"]) < 1e-14
+
+
+def test_hand_fp8_latent_rows():
+    g = GOLD["fp8_latent_rows"]
+    q = np.zeros((1, 1, W.D_QK), np.float32)
+    q[0, 0, g["q_ones"]] = 1.0
+    codes = np.zeros((1, W.BLOCK, W.D_QK), np.uint8)
+    scales = np.ones((1, W.BLOCK, 5), np.float32)
+    for r, (cd, sc) in enumerate([(g["row0_codes"], g["row0_scales"]), (g["row1_codes"], g["row1_scales"])]):
+        for k, v in cd.items():
+            codes[0, r, int(k)] = v
+        scales[0, r] = sc
+    wl = manual_workload(np.zeros((1, 64)), [0.0], np.zeros((2, 64)), K=2, H=1, q_mla=W.to_bf16_bits(q), kv=codes)
+    wl.kv_scale = scales
+    o, lse = oracle.sparse_attn(wl, np.array([[0, 1]], np.int32))
+    assert abs(o[0, 0, 0] - g["o0"]) < 1e-14
+    assert abs(o[0, 0, 128] - g["o128"]) < 1e-14
+    others = np.delete(o[0, 0], [0, 128])
+    assert np.all(others == 0.0)
+    assert abs(lse[0, 0] - g["lse"]) < 1e-13
+
+
+def test_fp8_latent_rows_equal_the_bf16_rows_they_encode():
+    # power-of-two tile scales and e4m3 codes give values that bf16 holds exactly, so the fp8
+    # path must equal the (pinned) bf16 path on the decoded rows, bit for bit
+    wl = W.make_workload("f", seq_lens=[300, 150], nq=[2, 1], H_I=8, D_I=64, H=4, K=64, with_kv=True,
+                         kv_dtype="fp8", seed=9)
+    r = np.random.default_rng(3)
+    wl.kv_scale = np.exp2(r.integers(-4, 5, size=wl.kv_scale.shape)).astype(np.float32)
+    dec = np.array([oracle.e4m3_to_f64(c) for c in range(256)])[wl.kv]
+    dec *= np.repeat(wl.kv_scale.astype(np.float64), 128, axis=-1)[..., :W.D_QK]
+    ref = dataclasses.replace(wl, kv=W.to_bf16_bits(dec.astype(np.float32)), kv_scale=None)
+    assert np.array_equal(W.bf16_bits_to_f32(ref.kv).astype(np.float64), dec)
+    idx = oracle.indexer_topk(wl)["idx"]
+    o1, l1 = oracle.sparse_attn(wl, idx)
+    o2, l2 = oracle.sparse_attn(ref, idx)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
 
 
 def test_hand_score_pairs():

@@ -54,6 +54,9 @@ MUTANTS = [
     ("e4m3_ties_away", "if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) == 1))", "if (d <= bd)"),
     ("mx_scale_minus_7", "e = ex - 1 - 8;", "e = ex - 1 - 7;"),
     ("mx_zero_group_scale", "int e = 0;\n        if (amax > 0.0) {", "int e = -127;\n        if (amax > 0.0) {"),
+    ("kv_fp8_tile_shifted", "* (double)a->kv_scale[row * 5 + d / 128];",
+     "* (double)a->kv_scale[row * 5 + (d / 128 + 1) % 5];"),
+    ("kv_fp8_scale_row_stride", "* (double)a->kv_scale[row * 5 + d / 128];", "* (double)a->kv_scale[row * 4 + d / 128];"),
     ("fp8_group_scale_over_240", "float sc = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;",
      "float sc = amax > 0.0 ? (float)(amax / 240.0) : 1.0f;"),
 ]
@@ -66,7 +69,8 @@ PINS = [pins.test_hand_indexer_relu_gate_weights_and_tie, pins.test_hand_fp8_sca
         pins.test_e8m0_decode_all_exponents_vs_torch, pins.test_hand_indexer_prolog,
         pins.test_prolog_projection_matches_numpy_matmul, pins.test_prolog_key_matches_torch_rms_norm,
         pins.test_hand_mx_encode_group, pins.test_e4m3_encode_matches_torch_cast_including_ties_and_saturation,
-        pins.test_mx_encode_scale_rule_and_error_bound, pins.test_fp8_group_encode_scale_is_amax_over_448]
+        pins.test_mx_encode_scale_rule_and_error_bound, pins.test_fp8_group_encode_scale_is_amax_over_448,
+        pins.test_hand_fp8_latent_rows, pins.test_fp8_latent_rows_equal_the_bf16_rows_they_encode]
 
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
