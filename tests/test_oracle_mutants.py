@@ -36,8 +36,8 @@ MUTANTS = [
      "acc += (double)a->w[(int64_t)t * a->H_I + (a->H_I - 1 - h)] * (dot > 0.0 ? dot : 0.0);"),
     ("pair_score_causal_edge", "if (s < 0 || s > pos) { out[i] = NAN; continue; }",
      "if (s < 0 || s >= pos) { out[i] = NAN; continue; }"),
-    ("softmax_value_from_rope", "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d]);",
-     "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * bf16_to_f64(kr[d + 64]);"),
+    ("softmax_value_from_rope", "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * kv_elem(a, rows[j], d);",
+     "for (int d = 0; d < ORACLE_DV; d++) o[d] += p * kv_elem(a, rows[j], d + 64);"),
     ("mx_key_group_of_64", "oracle_e8m0_to_f64(e[row * (a->D_I / 32) + d / 32]);",
      "oracle_e8m0_to_f64(e[row * (a->D_I / 32) + d / 64]);"),
     ("mx_query_group_of_64", "oracle_e8m0_to_f64(a->q_scale[((int64_t)t * a->H_I + h) * (a->D_I / 32) + d / 32]);",
