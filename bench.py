@@ -50,7 +50,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="batch32", choices=["batch32", "tiny", "prefill16k", "ragged", "1m",
-                                                              "batch32_mxfp8"])
+                                                              "batch32_mxfp8", "batch32_fp8kv"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-extra-workloads", action="store_true",
@@ -100,8 +100,9 @@ def ncu_traffic(kernel: str):
 
 
 def describe(wl):
+    kv = "fp8 (e4m3 + fp32 scale per 128-element tile)" if wl.kv_scale is not None else "bf16"
     return (f"{wl.name}: B={wl.B}, tokens={wl.T}, ctx max {int(wl.seq_lens.max())}, indexer {wl.H_I}x{wl.D_I} "
-            f"{wl.key_dtype} keys, K={wl.K}, MLA {wl.H} heads x (512+64) bf16, page 64, "
+            f"{wl.key_dtype} keys, K={wl.K}, MLA {wl.H} heads x (512+64) {kv}, page 64, "
             f"{'permuted' if wl.name != 'prefill16k' else 'contiguous'} block tables")
 
 
@@ -228,14 +229,15 @@ def measure(dsa, W, wl, dev, steps, warmup, graph=True):
 
     def fused():
         dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], wl.K, wl.sm_scale,
-                       k_scale=d["k_scale"], q_scale=d["q_scale"], out_idx=out_idx, out=out, workspace=ws)
+                       k_scale=d["k_scale"], q_scale=d["q_scale"], kv_scale=d["kv_scale"], out_idx=out_idx, out=out, workspace=ws)
 
     def indexer():
         dsa.indexer_topk(batch, d["q_idx"], d["w"], d["k_cache"], wl.K, k_scale=d["k_scale"], q_scale=d["q_scale"], out_idx=out_idx,
                          want_score=False, workspace=ws)
 
     def attention():
-        dsa.sparse_mla_attn(batch, d["q"], d["kv"], out_idx, wl.sm_scale, out=out, want_lse=False, workspace=ws)
+        dsa.sparse_mla_attn(batch, d["q"], d["kv"], out_idx, wl.sm_scale, kv_scale=d["kv_scale"], out=out,
+                            want_lse=False, workspace=ws)
 
     for _ in range(max(3, warmup)):
         if flush:
@@ -494,7 +496,7 @@ def run_ours(args, rank, world, local_rank):
         for k, v in host_in.items():
             d[k].copy_(v, non_blocking=True)
         dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], K, wl.sm_scale,
-                       k_scale=d["k_scale"], q_scale=d["q_scale"], out_idx=out_idx, out=out, workspace=ws)
+                       k_scale=d["k_scale"], q_scale=d["q_scale"], kv_scale=d["kv_scale"], out_idx=out_idx, out=out, workspace=ws)
         host_out.copy_(out, non_blocking=True)
         host_idx.copy_(out_idx, non_blocking=True)
 
@@ -519,7 +521,7 @@ def run_ours(args, rank, world, local_rank):
     sampler.stop()
 
     launches = dsa.decode_launch_count(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], K, wl.sm_scale,
-                                       k_scale=d["k_scale"], q_scale=d["q_scale"])
+                                       k_scale=d["k_scale"], q_scale=d["q_scale"], kv_scale=d["kv_scale"])
     peak, peak_kind = peaks()
     # ------------------------------------------------------------ the other workloads (one GPU): fused step,
     # each kernel, roofline fractions; fewer steps (each input set is generated on the host first)
@@ -527,7 +529,7 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_extra_workloads:
         del r, d, out, out_idx
         torch.cuda.empty_cache()
-        for name in ("tiny", "ragged", "1m", "prefill16k", "batch32_mxfp8"):
+        for name in ("tiny", "ragged", "1m", "prefill16k", "batch32_mxfp8", "batch32_fp8kv"):
             if name == args.workload:
                 continue
             xw = W.preset(name)

@@ -115,12 +115,24 @@ typedef struct {
     const uint8_t* q_scale;     /* device [T, H_I, D_I/32] exponents of MXFP8 queries, or NULL */
 } dsa_indexer_inputs;
 
+typedef enum {
+    DSA_KV_BF16 = 0,            /* latent cache rows in bf16 [num_blocks, 64, 576]                              */
+    DSA_KV_FP8 = 1              /* FP8 latent cache: e4m3fn codes [num_blocks, 64, 576] (uint8, 16-byte aligned)  */
+                                /* plus fp32 scales [num_blocks, 64, 5]: one per 128-element tile of a row, the  */
+                                /* fifth covering the 64 RoPE elements ("Day0 Adaptation and Performance         */
+                                /* Optimization ...", section 4: FP8 KV cache per token and head, tiles of 128). */
+                                /* The selected rows are dequantized to bf16 (code x scale, rounded once) into   */
+                                /* the workspace, 64 tokens at a time, before the attention                      */
+} dsa_kv_dtype;
+
 /* Sparse MLA attention inputs. */
 typedef struct {
     const void* q;              /* device [T, H, 576] bf16 (512 latent + 64 RoPE)   */
-    const void* kv_cache;       /* device [num_blocks, 64, 576] bf16                */
+    const void* kv_cache;       /* device latent cache, layout per kv_dtype         */
     int32_t H;                  /* query heads, 1..128                              */
     float sm_scale;             /* softmax scale applied to q . row[0:576]          */
+    int32_t kv_dtype;           /* dsa_kv_dtype                                     */
+    const float* kv_scale;      /* device [num_blocks, 64, 5] fp32 (FP8), else NULL */
 } dsa_attn_inputs;
 
 /*

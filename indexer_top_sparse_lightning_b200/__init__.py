@@ -9,7 +9,7 @@ fallback: if the library is missing, importing the entry points raises.
 
 Entry points (same names as the C ABI):
     indexer_topk(batch, q_idx, w, k_cache, K, k_scale=None, q_scale=None) -> (idx, score)
-    sparse_mla_attn(batch, q, kv_cache, idx, sm_scale) -> (out, lse)
+    sparse_mla_attn(batch, q, kv_cache, idx, sm_scale, kv_scale=None) -> (out, lse)
     dsa_decode(batch, q_idx, w, k_cache, q, kv_cache, K, sm_scale, k_scale=None, q_scale=None)
         -> (idx, score, out, lse)
 
@@ -42,6 +42,8 @@ KEY_FP8_E4M3 = 1
 KEY_MXFP8 = 2
 Q_BF16 = 0
 Q_MXFP8 = 1
+KV_BF16 = 0
+KV_FP8 = 1
 
 
 DSA_ERR_CUDA = 4   # dsa_status code of a failed CUDA runtime / driver call
@@ -72,7 +74,7 @@ class _Indexer(ctypes.Structure):
 
 class _Attn(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("kv_cache", ctypes.c_void_p), ("H", ctypes.c_int32),
-                ("sm_scale", ctypes.c_float)]
+                ("sm_scale", ctypes.c_float), ("kv_dtype", ctypes.c_int32), ("kv_scale", ctypes.c_void_p)]
 
 
 class _Prolog(ctypes.Structure):
@@ -230,11 +232,18 @@ def _indexer_struct(q_idx, w, k_cache, k_scale, K, q_scale=None):
                     _ptr(q_scale)), T
 
 
-def _attn_struct(q, kv_cache, sm_scale):
+def _attn_struct(q, kv_cache, sm_scale, kv_scale=None):
     import torch
     _check(q, "q", torch.bfloat16, 3, (None, None, 576))
-    _check(kv_cache, "kv_cache", torch.bfloat16, 3, (None, 64, 576))
-    return _Attn(_ptr(q), _ptr(kv_cache), int(q.shape[1]), float(sm_scale)), int(q.shape[0])
+    if kv_scale is None:
+        _check(kv_cache, "kv_cache", torch.bfloat16, 3, (None, 64, 576))
+        kt = KV_BF16
+    else:
+        # FP8 latent cache: e4m3 codes and one fp32 scale per 128-element tile of a row
+        _check(kv_cache, "kv_cache", torch.uint8, 3, (None, 64, 576))
+        _check(kv_scale, "kv_scale", torch.float32, 3, (kv_cache.shape[0], 64, 5))
+        kt = KV_FP8
+    return _Attn(_ptr(q), _ptr(kv_cache), int(q.shape[1]), float(sm_scale), kt, _ptr(kv_scale)), int(q.shape[0])
 
 
 class Workspace:
@@ -294,12 +303,13 @@ def indexer_topk(batch: Batch, q_idx, w, k_cache, K: int, k_scale=None, q_scale=
     return out_idx, out_score
 
 
-def sparse_mla_attn(batch: Batch, q, kv_cache, idx, sm_scale: float, *, out=None, lse=None,
+def sparse_mla_attn(batch: Batch, q, kv_cache, idx, sm_scale: float, *, kv_scale=None, out=None, lse=None,
                     want_lse: bool = True, workspace: Optional[Workspace] = None, stream=None):
-    """Sparse Flash Attention over the selected latent rows.  Returns (out [T,H,512] bf16, lse [T,H] fp32)."""
+    """Sparse Flash Attention over the selected latent rows (bf16 cache, or an FP8 cache of e4m3
+    codes with kv_scale).  Returns (out [T,H,512] bf16, lse [T,H] fp32)."""
     import torch
     lib = load_library()
-    at, T = _attn_struct(q, kv_cache, sm_scale)
+    at, T = _attn_struct(q, kv_cache, sm_scale, kv_scale)
     _check(idx, "idx", torch.int32, 2, (T, None))
     K = int(idx.shape[1])
     cb = batch.c(T)
@@ -341,14 +351,14 @@ def sparse_mla_attn_static(batch: Batch, q, kv_cache, idx, sm_scale: float, *, o
 
 
 def dsa_decode(batch: Batch, q_idx, w, k_cache, q, kv_cache, K: int, sm_scale: float, k_scale=None, q_scale=None, *,
-               out_idx=None, out_score=None, out=None, lse=None, want_score=False, want_lse=False,
+               kv_scale=None, out_idx=None, out_score=None, out=None, lse=None, want_score=False, want_lse=False,
                workspace: Optional[Workspace] = None, stream=None):
     """Whole step (indexer + Top-K + sparse attention) on one stream.
     Returns (idx, score or None, out, lse or None)."""
     import torch
     lib = load_library()
     ix, T = _indexer_struct(q_idx, w, k_cache, k_scale, K, q_scale)
-    at, T2 = _attn_struct(q, kv_cache, sm_scale)
+    at, T2 = _attn_struct(q, kv_cache, sm_scale, kv_scale)
     if T2 != T:
         raise ValueError("q_idx and q disagree on the number of tokens")
     cb = batch.c(T)
@@ -471,11 +481,11 @@ def indexer_prolog(batch: Batch, x, w_proj, k_gamma, eps: float, k_cache, k_scal
 
 
 def decode_launch_count(batch: Batch, q_idx, w, k_cache, q, kv_cache, K: int, sm_scale: float,
-                        k_scale=None, q_scale=None) -> int:
+                        k_scale=None, q_scale=None, kv_scale=None) -> int:
     """Kernel launches one dsa_decode call enqueues for these shapes."""
     lib = load_library()
     ix, T = _indexer_struct(q_idx, w, k_cache, k_scale, K, q_scale)
-    at, _ = _attn_struct(q, kv_cache, sm_scale)
+    at, _ = _attn_struct(q, kv_cache, sm_scale, kv_scale)
     cb = batch.c(T)
     n = lib.dsa_decode_launch_count(ctypes.byref(cb), ctypes.byref(ix), ctypes.byref(at))
     if n < 0:

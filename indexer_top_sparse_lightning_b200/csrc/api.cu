@@ -13,6 +13,7 @@
 #include "common.h"
 #include "host.h"
 #include "indexer.cuh"
+#include "kvfp8.cuh"
 #include "sfa.cuh"
 
 using namespace dsa;
@@ -64,6 +65,9 @@ dsa_status check_attn(const dsa_attn_inputs* at) {
     if (!at || !at->q || !at->kv_cache) return DSA_ERR_INVALID_ARG;
     if (at->H < 1 || at->H > 128) return DSA_ERR_UNSUPPORTED;
     if (!aligned16(at->q) || !aligned16(at->kv_cache)) return DSA_ERR_INVALID_ARG;
+    if (at->kv_dtype != DSA_KV_BF16 && at->kv_dtype != DSA_KV_FP8) return DSA_ERR_INVALID_ARG;
+    if (at->kv_dtype == DSA_KV_FP8 && (!at->kv_scale || (reinterpret_cast<uintptr_t>(at->kv_scale) & 3u)))
+        return DSA_ERR_INVALID_ARG;
     if (!(at->sm_scale > 0.0f) || at->sm_scale != at->sm_scale) return DSA_ERR_INVALID_ARG;
     return DSA_OK;
 }
@@ -294,6 +298,103 @@ dsa_status launch_attn(const dsa_batch* bt, const dsa_attn_inputs* at, const int
     return DSA_OK;
 }
 
+// ------------------------------------------------------------------ FP8 latent cache
+// The selected rows of up to kFp8ChunkTokens tokens at a time are dequantized
+// into a bf16 staging area of the workspace, then the attention runs over them
+// through a staging batch (one sequence per token; see kvfp8.cuh).
+constexpr int kFp8ChunkTokens = 64;
+
+struct Fp8Stage {
+    int tc = 0, KP = 0;
+    size_t stage_bytes = 0, lens_off = 0, cu_off = 0, table_off = 0, idx_off = 0, total = 0;
+};
+
+Fp8Stage fp8_stage_layout(int64_t T, int K) {
+    Fp8Stage f;
+    f.tc = (int)(T < kFp8ChunkTokens ? T : kFp8ChunkTokens);
+    f.KP = (K + kPage - 1) / kPage * kPage;
+    f.stage_bytes = align256((size_t)f.tc * f.KP * kDqk * 2);
+    f.lens_off = f.stage_bytes;
+    f.cu_off = f.lens_off + align256((size_t)f.tc * 4);
+    f.table_off = f.cu_off + align256((size_t)(f.tc + 1) * 4);
+    f.idx_off = f.table_off + align256((size_t)f.tc * (f.KP / kPage) * 4);
+    f.total = f.idx_off + align256((size_t)f.tc * K * 4);
+    return f;
+}
+
+// Attention over an FP8 latent cache, chunk by chunk.  The first staging launch is
+// a plain stream-ordered launch (after the indexer, in dsa_decode); each attention
+// launch is a programmatic dependent of its staging launch.
+dsa_status launch_attn_fp8(const dsa_batch* bt, const dsa_attn_inputs* at, const int32_t* idx, int K, void* out,
+                           float* lse, uint32_t* status, uint8_t* attn_ws, uint8_t* stage_ws, const DevInfo& di,
+                           cudaStream_t stream) {
+    const int64_t T = bt->num_tokens;
+    const Fp8Stage f = fp8_stage_layout(T, K);
+    for (int64_t t0 = 0; t0 < T; t0 += f.tc) {
+        const int tc = (int)(T - t0 < f.tc ? T - t0 : f.tc);
+        KvStageParams kp;
+        memset(&kp, 0, sizeof kp);
+        kp.seq_lens = bt->seq_lens;
+        kp.cu_q = bt->cu_q;
+        kp.block_table = bt->block_table;
+        kp.kv_codes = static_cast<const uint8_t*>(at->kv_cache);
+        kp.kv_scale = at->kv_scale;
+        kp.idx = idx;
+        kp.stage = reinterpret_cast<uint16_t*>(stage_ws);
+        kp.s_seq_lens = reinterpret_cast<int32_t*>(stage_ws + f.lens_off);
+        kp.s_cu_q = reinterpret_cast<int32_t*>(stage_ws + f.cu_off);
+        kp.s_table = reinterpret_cast<int32_t*>(stage_ws + f.table_off);
+        kp.s_idx = reinterpret_cast<int32_t*>(stage_ws + f.idx_off);
+        kp.status = status;
+        kp.B = bt->batch;
+        kp.max_blocks = bt->max_blocks_per_seq;
+        kp.num_blocks = bt->num_blocks;
+        kp.K = K;
+        kp.KP = f.KP;
+        kp.t0 = (int32_t)t0;
+        kp.tc = tc;
+        const dim3 grid((unsigned)((K + kKvStageWarps - 1) / kKvStageWarps), (unsigned)tc, 1);
+        kv_fp8_stage_kernel<<<grid, 32 * kKvStageWarps, 0, stream>>>(kp);
+        if (cudaError_t e = cudaGetLastError()) return fail(DSA_ERR_CUDA, "latent staging launch", e);
+        // the chunk's tokens as sequences of their own staged rows
+        dsa_batch sb;
+        memset(&sb, 0, sizeof sb);
+        sb.batch = tc;
+        sb.num_tokens = tc;
+        sb.seq_lens = kp.s_seq_lens;
+        sb.cu_q = kp.s_cu_q;
+        sb.block_table = kp.s_table;
+        sb.max_blocks_per_seq = f.KP / kPage;
+        sb.num_blocks = tc * (f.KP / kPage);
+        sb.max_seq_len = f.KP;
+        sb.max_q_per_seq = 1;
+        dsa_attn_inputs sa = *at;
+        sa.q = static_cast<const uint8_t*>(at->q) + t0 * at->H * kDqk * 2;
+        sa.kv_cache = stage_ws;
+        sa.kv_dtype = DSA_KV_BF16;
+        sa.kv_scale = nullptr;
+        const AttnPlan ap = plan_attn(&sb, K, di);
+        void* o = static_cast<uint8_t*>(out) + t0 * at->H * kDv * 2;
+        float* l = lse ? lse + t0 * at->H : nullptr;
+        if (dsa_status st = launch_attn(&sb, &sa, kp.s_idx, K, o, l, status, attn_ws, ap, stream, true, true))
+            return st;
+    }
+    return DSA_OK;
+}
+
+int64_t fp8_launches(const dsa_batch* bt, int K, const DevInfo& di) {
+    const Fp8Stage f = fp8_stage_layout(bt->num_tokens, K);
+    int64_t n = 0;
+    for (int64_t t0 = 0; t0 < bt->num_tokens; t0 += f.tc) {
+        const int tc = (int)(bt->num_tokens - t0 < f.tc ? bt->num_tokens - t0 : f.tc);
+        dsa_batch sb = *bt;
+        sb.batch = tc;
+        sb.num_tokens = tc;
+        n += 2 + (plan_attn(&sb, K, di).combine ? 1 : 0);
+    }
+    return n;
+}
+
 // ------------------------------------------------------------------ allocation-free attention
 // Scratch of sparse_mla_attn_static, in module memory: the status area and the
 // partial slots of tokens shared by several CTA pairs.  20 MiB holds the
@@ -376,6 +477,7 @@ size_t dsa_workspace_size(const dsa_batch* batch, const dsa_indexer_inputs* ix, 
         if (check_attn(at) != DSA_OK) return 0;
         // sized for the largest Top-K, so one workspace serves any K
         need += attn_region_bytes(plan_attn(batch, kMaxTopK, di));
+        if (at->kv_dtype == DSA_KV_FP8) need += fp8_stage_layout(batch->num_tokens, ix ? ix->K : kMaxTopK).total;
     }
     return need;
 }
@@ -412,8 +514,14 @@ dsa_status sparse_mla_attn(const dsa_batch* batch, const dsa_attn_inputs* at, co
     if (di.max_smem < SfaCfg::SMEM) return fail(DSA_ERR_UNSUPPORTED, "device shared memory per block too small");
     const AttnPlan ap = plan_attn(batch, K, di);
     const size_t off = kHeaderBytes + idx_region_bytes(di);
-    if (workspace_bytes < off + attn_region_bytes(ap)) return DSA_ERR_WORKSPACE;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    if (at->kv_dtype == DSA_KV_FP8) {
+        const size_t aoff = off + attn_region_bytes(plan_attn(batch, kMaxTopK, di));
+        if (workspace_bytes < aoff + fp8_stage_layout(batch->num_tokens, K).total) return DSA_ERR_WORKSPACE;
+        return launch_attn_fp8(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + off, ws + aoff, di,
+                               reinterpret_cast<cudaStream_t>(stream));
+    }
+    if (workspace_bytes < off + attn_region_bytes(ap)) return DSA_ERR_WORKSPACE;
     return launch_attn(batch, at, idx, K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + off, ap,
                        reinterpret_cast<cudaStream_t>(stream), true, false);
 }
@@ -425,6 +533,8 @@ dsa_status sparse_mla_attn_static(const dsa_batch* batch, const dsa_attn_inputs*
     if ((st = check_attn(at)) != DSA_OK) return st;
     if (!idx || !out || K < 1 || K > kMaxTopK) return DSA_ERR_INVALID_ARG;
     if (!aligned16(out)) return DSA_ERR_INVALID_ARG;
+    if (at->kv_dtype != DSA_KV_BF16)
+        return fail(DSA_ERR_UNSUPPORTED, "sparse_mla_attn_static: the FP8 latent cache needs a caller workspace");
     const DevInfo di = dev_info();
     if (di.sms <= 0) return fail(DSA_ERR_CUDA, "device query failed");
     if (di.max_smem < SfaCfg::SMEM) return fail(DSA_ERR_UNSUPPORTED, "device shared memory per block too small");
@@ -469,11 +579,17 @@ dsa_status dsa_decode(const dsa_batch* batch, const dsa_indexer_inputs* ix, cons
     if (pl.group_ws > group_region_bytes(di.sms)) return DSA_ERR_UNSUPPORTED;
     const AttnPlan ap = plan_attn(batch, ix->K, di);
     const size_t off = kHeaderBytes + idx_region_bytes(di);
+    const size_t aoff = off + attn_region_bytes(plan_attn(batch, kMaxTopK, di));
     if (workspace_bytes < off + attn_region_bytes(ap)) return DSA_ERR_WORKSPACE;
+    if (at->kv_dtype == DSA_KV_FP8 && workspace_bytes < aoff + fp8_stage_layout(batch->num_tokens, ix->K).total)
+        return DSA_ERR_WORKSPACE;
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     st = fn(batch, ix, out_idx, out_score, reinterpret_cast<uint32_t*>(ws), ws + kHeaderBytes, pl, s);
     if (st != DSA_OK) return st;
+    if (at->kv_dtype == DSA_KV_FP8)
+        return launch_attn_fp8(batch, at, out_idx, ix->K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + off, ws + aoff,
+                               di, s);
     // the attention launch depends programmatically on the indexer launch just made
     return launch_attn(batch, at, out_idx, ix->K, out, lse, reinterpret_cast<uint32_t*>(ws), ws + off, ap, s, true,
                        true);
@@ -502,6 +618,7 @@ int32_t dsa_decode_launch_count(const dsa_batch* batch, const dsa_indexer_inputs
     LaunchFn fn = nullptr;
     if (plan_indexer(batch, ix, di, pl, fn) != DSA_OK) return -1;
     const int64_t n_idx = pl.mode == 1 ? 1 : idx_launches(pl.windows, pl.windows_per_launch);
+    if (at->kv_dtype == DSA_KV_FP8) return (int32_t)(n_idx + fp8_launches(batch, ix->K, di));   // staging + attention per chunk
     return (int32_t)n_idx + 1 + (plan_attn(batch, ix->K, di).combine ? 1 : 0);   // attention (+ merge)
 }
 

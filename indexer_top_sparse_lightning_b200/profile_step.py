@@ -80,7 +80,7 @@ def main(argv=None) -> int:
                              want_score=False)
         else:
             dsa.dsa_decode(batch, d["q_idx"], d["w"], d["k_cache"], d["q"], d["kv"], wl.K, wl.sm_scale,
-                           k_scale=d["k_scale"], q_scale=d["q_scale"], workspace=ws)
+                           k_scale=d["k_scale"], q_scale=d["q_scale"], kv_scale=d["kv_scale"], workspace=ws)
         ev[i + 1].record()
     torch.cuda.synchronize()
     st = dsa.get_status(ws)

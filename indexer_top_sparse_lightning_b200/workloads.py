@@ -124,9 +124,11 @@ class Workload:
         return int(np.sum(vis)) * 2 * self.H_I * self.D_I
 
     def kv_bytes(self) -> int:
-        """Latent-cache bytes gathered by sparse attention: min(K, visible) rows per token."""
+        """Latent-cache bytes gathered by sparse attention: min(K, visible) rows per token
+        (576 bf16, or 576 e4m3 codes plus five fp32 tile scales)."""
         vis = self.token_pos() + 1
-        return int(np.sum(np.minimum(vis, self.K))) * D_QK * 2
+        per = D_QK + 5 * 4 if self.kv_scale is not None else D_QK * 2
+        return int(np.sum(np.minimum(vis, self.K))) * per
 
 
 def _rng(seed: int, stream: int) -> np.random.Generator:
@@ -349,6 +351,9 @@ PRESETS = {
     # batch32 with MXFP8 index queries and keys (e4m3, one power-of-two scale per 32 elements)
     "batch32_mxfp8": dict(seq_lens=[32768] * 32, nq=1, H_I=64, D_I=128, H=128, K=2048, key_dtype="mxfp8",
                           w_dist="u8", seed=1005),
+    # batch32 with the FP8 latent cache (e4m3, one fp32 scale per 128-element tile of a row)
+    "batch32_fp8kv": dict(seq_lens=[32768] * 32, nq=1, H_I=64, D_I=128, H=128, K=2048, kv_dtype="fp8",
+                          w_dist="u8", seed=1006),
 }
 
 

@@ -143,3 +143,15 @@ def test_prolog_packed_bytes(lib):
     assert lib.indexer_prolog_pack(16, 16, 8, 64, 100, None) == 1
     assert lib.indexer_prolog_pack(None, 16, 8, 64, 128, None) == 1
     assert lib.indexer_prolog_pack(16, 24, 8, 64, 128, None) == 1
+
+
+def test_attention_rejects_bad_latent_format(lib):
+    b = ctypes.byref(_batch())
+    bad = dsa._Attn(16, 16, 128, 0.04, 7, None)
+    assert lib.sparse_mla_attn(b, ctypes.byref(bad), 16, 64, 16, None, 256, 1 << 20, None) == 1
+    no_scale = dsa._Attn(16, 16, 128, 0.04, 1, None)
+    assert lib.sparse_mla_attn(b, ctypes.byref(no_scale), 16, 64, 16, None, 256, 1 << 20, None) == 1
+    odd_scale = dsa._Attn(16, 16, 128, 0.04, 1, 18)
+    assert lib.sparse_mla_attn(b, ctypes.byref(odd_scale), 16, 64, 16, None, 256, 1 << 20, None) == 1
+    fp8 = dsa._Attn(16, 16, 128, 0.04, 1, 16)
+    assert lib.sparse_mla_attn_static(b, ctypes.byref(fp8), 16, 64, 16, None, None) == 2
