@@ -45,7 +45,27 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
     return __half22float2(*reinterpret_cast<__half2*>(&h2));
 }
 
-// grid (ceil(KP / 8), tc), 256 threads: one warp per selected row of one token.
+// Dequantizes one 16-code chunk (tile scale s) into 16 bf16 values at dst.
+__device__ __forceinline__ void stage_chunk(uint4 raw, float s, uint4* dst) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 lo = e4m3x2_to_float2((uint16_t)(w[k] & 0xFFFFu));
+        const float2 hi = e4m3x2_to_float2((uint16_t)(w[k] >> 16));
+        const __nv_bfloat162 a = __floats2bfloat162_rn(lo.x * s, lo.y * s);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(hi.x * s, hi.y * s);
+        o[2 * k] = *reinterpret_cast<const uint32_t*>(&a);
+        o[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// grid (ceil(K / 256), tc), 256 threads.  Each warp takes 32 consecutive selected
+// rows of one token: lane l resolves row j0 + l (index, page, cache row), then the
+// warp copies the 32 rows four at a time, every load of the four issued before
+// any conversion, so that each lane keeps about ten loads in flight.
 __global__ void __launch_bounds__(32 * kKvStageWarps) kv_fp8_stage_kernel(const KvStageParams p) {
     // the attention launch that follows may be scheduled now (it waits for this grid
     // before reading anything written here)
@@ -53,7 +73,6 @@ __global__ void __launch_bounds__(32 * kKvStageWarps) kv_fp8_stage_kernel(const 
     const int i = blockIdx.y;                   // token of the chunk
     const int t = p.t0 + i;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int j = blockIdx.x * kKvStageWarps + warp;
     const int pages = p.KP / kPage;
     __shared__ int s_b;
     if (threadIdx.x == 0) {
@@ -74,41 +93,55 @@ __global__ void __launch_bounds__(32 * kKvStageWarps) kv_fp8_stage_kernel(const 
         }
     }
     __syncthreads();
-    if (j >= p.K) return;
-    const int pos = __ldg(p.idx + (int64_t)t * p.K + j);
-    if (lane == 0) p.s_idx[(int64_t)i * p.K + j] = pos >= 0 ? j : -1;
-    if (pos < 0) return;                        // never read by the attention
-    const int b = s_b;
-    int64_t row = -1;
-    if (pos < __ldg(p.seq_lens + b) && pos / kPage < p.max_blocks) {
-        const int blk = __ldg(p.block_table + (int64_t)b * p.max_blocks + pos / kPage);
-        if (blk >= 0 && blk < p.num_blocks) row = (int64_t)blk * kPage + pos % kPage;
-    }
-    uint16_t* dst = p.stage + ((int64_t)i * p.KP + j) * kDqk;
-    if (row < 0) {
-        if (lane == 0) atomicCAS(p.status, 0u, (uint32_t)kStBounds);
-        for (int c = lane; c < kDqk / 8; c += 32) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0u, 0u, 0u, 0u);
-        return;
-    }
-    const uint8_t* src = p.kv_codes + row * kDqk;
-    const float* sc = p.kv_scale + row * kKvTiles;
-    // 36 chunks of 16 codes; chunk c lies in tile c / 8
-    for (int c = lane; c < kDqk / 16; c += 32) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src) + c);
-        const float s = __ldg(sc + c / 8);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        uint32_t o[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 lo = e4m3x2_to_float2((uint16_t)(w[k] & 0xFFFFu));
-            const float2 hi = e4m3x2_to_float2((uint16_t)(w[k] >> 16));
-            const __nv_bfloat162 a = __floats2bfloat162_rn(lo.x * s, lo.y * s);
-            const __nv_bfloat162 bb = __floats2bfloat162_rn(hi.x * s, hi.y * s);
-            o[2 * k] = *reinterpret_cast<const uint32_t*>(&a);
-            o[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&bb);
+    const int j0 = (blockIdx.x * kKvStageWarps + warp) * 32;
+    if (j0 >= p.K) return;
+    const int j = j0 + lane;
+    const int pos = j < p.K ? __ldg(p.idx + (int64_t)t * p.K + j) : -1;
+    if (j < p.K) p.s_idx[(int64_t)i * p.K + j] = pos >= 0 ? j : -1;
+    long long row = -1;                          // cache row; -2: selected but out of range
+    if (pos >= 0) {
+        const int b = s_b;
+        row = -2;
+        if (pos < __ldg(p.seq_lens + b) && pos / kPage < p.max_blocks) {
+            const int blk = __ldg(p.block_table + (int64_t)b * p.max_blocks + pos / kPage);
+            if (blk >= 0 && blk < p.num_blocks) row = (long long)blk * kPage + pos % kPage;
         }
-        reinterpret_cast<uint4*>(dst)[2 * c] = make_uint4(o[0], o[1], o[2], o[3]);
-        reinterpret_cast<uint4*>(dst)[2 * c + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    if (__any_sync(0xffffffffu, row == -2) && lane == 0) atomicCAS(p.status, 0u, (uint32_t)kStBounds);
+    uint4* dst0 = reinterpret_cast<uint4*>(p.stage + ((int64_t)i * p.KP + j0) * kDqk);
+    // 36 chunks of 16 codes per row: lane l takes chunk l and, for l < 4, chunk 32 + l;
+    // chunk c lies in tile c / 8
+    const int c1 = 32 + (lane & 3);
+#pragma unroll 1
+    for (int r0 = 0; r0 < 32; r0 += 4) {
+        long long rr[4];
+        uint4 a[4], b[4];
+        float sa[4], sb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            rr[u] = __shfl_sync(0xffffffffu, row, r0 + u);
+            if (rr[u] >= 0) {
+                const uint4* src = reinterpret_cast<const uint4*>(p.kv_codes + rr[u] * kDqk);
+                const float* sc = p.kv_scale + rr[u] * kKvTiles;
+                a[u] = __ldg(src + lane);
+                sa[u] = __ldg(sc + lane / 8);
+                if (lane < 4) {
+                    b[u] = __ldg(src + c1);
+                    sb[u] = __ldg(sc + c1 / 8);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            uint4* dst = dst0 + (int64_t)(r0 + u) * (kDqk / 8);
+            if (rr[u] >= 0) {
+                stage_chunk(a[u], sa[u], dst + 2 * lane);
+                if (lane < 4) stage_chunk(b[u], sb[u], dst + 2 * c1);
+            } else if (rr[u] == -2) {
+                // a selected position past the cache: zeros (reported above)
+                for (int c = lane; c < kDqk / 8; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
     }
 }
 
