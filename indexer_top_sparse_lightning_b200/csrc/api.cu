@@ -353,7 +353,8 @@ dsa_status launch_attn_fp8(const dsa_batch* bt, const dsa_attn_inputs* at, const
         kp.KP = f.KP;
         kp.t0 = (int32_t)t0;
         kp.tc = tc;
-        const dim3 grid((unsigned)((K + 32 * kKvStageWarps - 1) / (32 * kKvStageWarps)), (unsigned)tc, 1);
+        const int rows_per_block = kKvRowsPerWarp * kKvStageWarps;
+        const dim3 grid((unsigned)((K + rows_per_block - 1) / rows_per_block), (unsigned)tc, 1);
         kv_fp8_stage_kernel<<<grid, 32 * kKvStageWarps, 0, stream>>>(kp);
         if (cudaError_t e = cudaGetLastError()) return fail(DSA_ERR_CUDA, "latent staging launch", e);
         // the chunk's tokens as sequences of their own staged rows

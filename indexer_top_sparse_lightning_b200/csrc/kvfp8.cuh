@@ -37,6 +37,7 @@ struct KvStageParams {
 
 constexpr int kKvTiles = 5;                 // 4 latent tiles of 128 + the 64-element RoPE tile
 constexpr int kKvStageWarps = 8;
+constexpr int kKvRowsPerWarp = 8;
 
 // Two e4m3 codes (low byte first) -> two floats, exactly.
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
@@ -62,10 +63,10 @@ __device__ __forceinline__ void stage_chunk(uint4 raw, float s, uint4* dst) {
     dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// grid (ceil(K / 256), tc), 256 threads.  Each warp takes 32 consecutive selected
-// rows of one token: lane l resolves row j0 + l (index, page, cache row), then the
-// warp copies the 32 rows four at a time, every load of the four issued before
-// any conversion, so that each lane keeps about ten loads in flight.
+// grid (ceil(K / 64), tc), 256 threads.  Each warp takes 8 consecutive selected
+// rows of one token: lane l < 8 resolves row j0 + l (index, page, cache row), then
+// every load of the 8 rows is issued before any conversion, so that a warp waits
+// for one round of memory latency per row group.
 __global__ void __launch_bounds__(32 * kKvStageWarps) kv_fp8_stage_kernel(const KvStageParams p) {
     // the attention launch that follows may be scheduled now (it waits for this grid
     // before reading anything written here)
@@ -93,11 +94,12 @@ __global__ void __launch_bounds__(32 * kKvStageWarps) kv_fp8_stage_kernel(const 
         }
     }
     __syncthreads();
-    const int j0 = (blockIdx.x * kKvStageWarps + warp) * 32;
+    const int j0 = (blockIdx.x * kKvStageWarps + warp) * kKvRowsPerWarp;
     if (j0 >= p.K) return;
     const int j = j0 + lane;
-    const int pos = j < p.K ? __ldg(p.idx + (int64_t)t * p.K + j) : -1;
-    if (j < p.K) p.s_idx[(int64_t)i * p.K + j] = pos >= 0 ? j : -1;
+    const bool mine = lane < kKvRowsPerWarp && j < p.K;
+    const int pos = mine ? __ldg(p.idx + (int64_t)t * p.K + j) : -1;
+    if (mine) p.s_idx[(int64_t)i * p.K + j] = pos >= 0 ? j : -1;
     long long row = -1;                          // cache row; -2: selected but out of range
     if (pos >= 0) {
         const int b = s_b;
@@ -112,35 +114,33 @@ __global__ void __launch_bounds__(32 * kKvStageWarps) kv_fp8_stage_kernel(const 
     // 36 chunks of 16 codes per row: lane l takes chunk l and, for l < 4, chunk 32 + l;
     // chunk c lies in tile c / 8
     const int c1 = 32 + (lane & 3);
-#pragma unroll 1
-    for (int r0 = 0; r0 < 32; r0 += 4) {
-        long long rr[4];
-        uint4 a[4], b[4];
-        float sa[4], sb[4];
+    constexpr int R = kKvRowsPerWarp;
+    long long rr[R];
+    uint4 a[R], b[R];
+    float sa[R], sb[R];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            rr[u] = __shfl_sync(0xffffffffu, row, r0 + u);
-            if (rr[u] >= 0) {
-                const uint4* src = reinterpret_cast<const uint4*>(p.kv_codes + rr[u] * kDqk);
-                const float* sc = p.kv_scale + rr[u] * kKvTiles;
-                a[u] = __ldg(src + lane);
-                sa[u] = __ldg(sc + lane / 8);
-                if (lane < 4) {
-                    b[u] = __ldg(src + c1);
-                    sb[u] = __ldg(sc + c1 / 8);
-                }
+    for (int u = 0; u < R; ++u) {
+        rr[u] = __shfl_sync(0xffffffffu, row, u);
+        if (rr[u] >= 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.kv_codes + rr[u] * kDqk);
+            const float* sc = p.kv_scale + rr[u] * kKvTiles;
+            a[u] = __ldg(src + lane);
+            sa[u] = __ldg(sc + lane / 8);
+            if (lane < 4) {
+                b[u] = __ldg(src + c1);
+                sb[u] = __ldg(sc + c1 / 8);
             }
         }
+    }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            uint4* dst = dst0 + (int64_t)(r0 + u) * (kDqk / 8);
-            if (rr[u] >= 0) {
-                stage_chunk(a[u], sa[u], dst + 2 * lane);
-                if (lane < 4) stage_chunk(b[u], sb[u], dst + 2 * c1);
-            } else if (rr[u] == -2) {
-                // a selected position past the cache: zeros (reported above)
-                for (int c = lane; c < kDqk / 8; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-            }
+    for (int u = 0; u < R; ++u) {
+        uint4* dst = dst0 + (int64_t)u * (kDqk / 8);
+        if (rr[u] >= 0) {
+            stage_chunk(a[u], sa[u], dst + 2 * lane);
+            if (lane < 4) stage_chunk(b[u], sb[u], dst + 2 * c1);
+        } else if (rr[u] == -2) {
+            // a selected position past the cache: zeros (reported above)
+            for (int c = lane; c < kDqk / 8; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
 }
