@@ -59,22 +59,35 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, result_dir):
+def _chunk_workload(key_dtype):
+    return W.make_workload("cp", seq_lens=[3000], nq=1000, H_I=8, D_I=64, H=1, K=96, int_inputs=True,
+                           w_dist="u256", key_dtype=key_dtype, with_kv=False, seed=71)
+
+
+def _rank_main(rank, world, port, result_dir, key_dtype):
     import oracle
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        wl = W.make_workload("cp", seq_lens=[3000], nq=1000, H_I=8, D_I=64, H=1, K=96, int_inputs=True,
-                             w_dist="u256", with_kv=False, seed=71)
+        wl = _chunk_workload(key_dtype)
         n, seq_len = wl.T, int(wl.seq_lens[0])
         rows_all = cp.cache_rows(wl.block_table[0], seq_len, n, range(n))
         # this rank's cache: the prefix and its own new rows; the other ranks' new rows are zero
-        k = torch.from_numpy(wl.k_idx.copy()).view(torch.int16)   # bf16 bits
+        if key_dtype == "bf16":
+            k = torch.from_numpy(wl.k_idx.copy()).view(torch.int16)   # bf16 bits
+            ks = None
+        else:
+            k = torch.from_numpy(wl.k_idx.copy())                      # e4m3 codes
+            ks = torch.from_numpy(wl.k_scale.copy())                   # fp32 per-64 scales
         own = cp.local_batch(seq_len, n, cp.zigzag_pieces(n, world, rank))[2]
-        others = np.setdiff1d(np.arange(n), own)
-        k.view(-1, wl.D_I)[torch.as_tensor(rows_all[others])] = 0
-        cp.share_new_keys(k, None, wl.block_table[0], seq_len, n, world, rank)
-        np.testing.assert_array_equal(k.numpy().view(np.uint16), wl.k_idx)
+        others = torch.as_tensor(rows_all[np.setdiff1d(np.arange(n), own)])
+        k.view(-1, wl.D_I)[others] = 0
+        if ks is not None:
+            ks.view(k.shape[0] * k.shape[1], -1)[others] = 0
+        cp.share_new_keys(k, ks, wl.block_table[0], seq_len, n, world, rank)
+        np.testing.assert_array_equal(k.numpy().view(wl.k_idx.dtype), wl.k_idx)
+        if ks is not None:
+            np.testing.assert_array_equal(ks.numpy(), wl.k_scale)
         # select the local tokens, then restore the chunk order on every rank
         lwl, toks = _local_workload(wl, world, rank)
         idx = torch.from_numpy(oracle.indexer_topk(lwl)["idx"])
@@ -84,19 +97,17 @@ def _rank_main(rank, world, port, result_dir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 4])
-def test_cp_gloo_gathers_keys_and_restores_order(tmp_path, world):
+@pytest.mark.parametrize("world,key_dtype", [(2, "bf16"), (4, "bf16"), (2, "fp8")])
+def test_cp_gloo_gathers_keys_and_restores_order(tmp_path, world, key_dtype):
     import oracle
     ctx = mp.get_context("spawn")
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, str(tmp_path))) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, str(tmp_path), key_dtype)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(240)
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
-    wl = W.make_workload("cp", seq_lens=[3000], nq=1000, H_I=8, D_I=64, H=1, K=96, int_inputs=True,
-                         w_dist="u256", with_kv=False, seed=71)
-    ref = oracle.indexer_topk(wl)["idx"]
+    ref = oracle.indexer_topk(_chunk_workload(key_dtype))["idx"]
     for r in range(world):
         np.testing.assert_array_equal(np.load(tmp_path / f"idx{r}.npy"), ref)
