@@ -197,6 +197,18 @@ def test_packed_weights_give_identical_outputs(key_dtype, T, d):
     _assert_prolog(wl, pw, b)
 
 
+@pytest.mark.parametrize("key_dtype,H_I,D_I,T,d", [("fp8", 32, 64, 40, 768), ("fp8", 8, 128, 5, 2048),
+                                                   ("mxfp8", 8, 64, 70, 512), ("bf16", 16, 64, 129, 320)])
+def test_other_head_shapes_against_oracle(key_dtype, H_I, D_I, T, d):
+    # the key tile holding a 64-element key next to head-weight rows (D_I = 64), few row tiles
+    # (splits of 16), and token tiles of 64 / 256 with ragged ends
+    nb = min(3, T)
+    nq = [T // nb + (1 if i < T % nb else 0) for i in range(nb)]
+    wl, pw = _setup([900 + 100 * i + n for i, n in enumerate(nq)], nq, H_I, D_I, key_dtype, d=d, seed=89 + T)
+    _assert_prolog(wl, pw, _run(wl, pw))
+    _assert_prolog(wl, pw, _run(wl, pw, packed=True))
+
+
 def test_split_contraction_is_deterministic():
     wl, pw = _setup([4096] * 32, 1, 64, 128, "bf16", d=2048, seed=47)
     a = _run(wl, pw)
