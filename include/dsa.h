@@ -141,7 +141,10 @@ typedef struct {
  * layout is [256-byte status area][indexer group region and published-key
  * slots, a fixed size per device][attention partial slots of tokens shared
  * by several SM pairs, a fixed size per device]; one buffer sized with both
- * serves all three entry points, for any mix of shapes.
+ * serves all three entry points, for any mix of shapes.  With an FP8 latent
+ * cache (at->kv_dtype) a staging region follows: the selected rows of up to
+ * 64 tokens as bf16 plus their per-token batch (sized for ix->K, or for
+ * K = 2048 when ix is NULL); its contents are scratch.
  * The workspace must be 256-byte aligned and ZERO-FILLED before its first
  * use.  After that the library keeps it consistent by itself (a call that
  * completes without a device error leaves its histograms zero and its
