@@ -14,9 +14,10 @@
 //
 // Orientation: D^T[n, t] = sum_c W[n, c] * x[t, c].  The weight rows are the
 // MMA's M side (128 per tile, TMEM lanes), the tokens its N side (BN per tile,
-// TMEM columns), so that each epilogue thread owns one output row: an MXFP8
-// group (32 consecutive rows of one head) is one warp, and the key's RMS norm
-// is a reduction over the warps holding the key rows.
+// TMEM columns), so that each epilogue thread owns one output row (two warps
+// per TMEM lane quarter, each taking half of the token columns): an MXFP8 group
+// (32 consecutive rows of one head) is one warp, and the key's RMS norm is a
+// reduction over the warps holding the key rows.
 //
 // Work units are (row tile, token tile, K split).  With one split the unit's
 // CTA runs the epilogue from TMEM.  With S splits (few tiles, e.g. decode)
@@ -66,18 +67,18 @@ struct PrologMisc {
     int last;
     int pad_;
     uint64_t wait_ns;
-    float red_ss[2][4][8];       // key sum of squares per (warp, token column), double-buffered by sub-chunk
-    float red_am[2][4][8];       // key amax per (warp, token column) for the per-64 fp8 scale
+    float red_ss[2][2][4][8];    // key sum of squares per (column half, sub-chunk parity, lane quarter, column)
+    float red_am[2][2][4][8];    // key amax, the same indexing, for the per-64 fp8 scale
     int64_t row[256];            // key-cache row of each token column (-1: none)
 };
 
 template <int BN>
 struct PrologCfg {
     static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "token tile");
-    static constexpr int THREADS = 192;             // 4 epilogue warps, TMA producer, MMA issuer
-    static constexpr int EPI_THREADS = 128;
-    static constexpr int PRODUCER_WARP = 4;
-    static constexpr int MMA_WARP = 5;
+    static constexpr int THREADS = 320;             // 8 epilogue warps, TMA producer, MMA issuer
+    static constexpr int EPI_THREADS = 256;         // two warps per TMEM lane quarter, each half the columns
+    static constexpr int PRODUCER_WARP = 8;
+    static constexpr int MMA_WARP = 9;
     static constexpr int A_BYTES = 128 * 128;       // 128 weight rows x 64 bf16, 128-byte swizzle
     static constexpr int B_BYTES = BN * 128;        // BN tokens x 64 bf16
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -297,7 +298,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
             mbar_wait(&m->drain, 0, &no_abort, wlim);
         }
     } else {
-        // ---------------------------------------------------------------- epilogue (warps 0-3)
+        // ---------------------------------------------------------------- epilogue (warps 0-7)
         const int et = threadIdx.x;
         const int key_fp8_groups = p.k_scale_f32 != nullptr;
         int lu = 0;
@@ -306,7 +307,10 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
             prolog_unit(p, u, tile, mt, nt, ks, ns, kb0, kb1);
             const int buf = lu & 1;
             const int row0 = mt * 128;
-            const int base = row0 + warp * 32;          // first output row of this warp
+            const int q4 = warp & 3;                     // TMEM lane quarter = the warp's 32 rows
+            const int half = warp >> 2;                  // which half of the token columns
+            const int cb = half * (BN / 2), ce = cb + BN / 2;
+            const int base = row0 + q4 * 32;             // first output row of this warp
             const int n = base + lane;                   // this thread's output row
             const bool has_k = row0 < p.HD + p.D_I && row0 + 128 > p.HD;
             const bool kw = base >= p.HD && base < p.HD + p.D_I;   // this warp holds key rows
@@ -328,14 +332,14 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + buf * BN;
-            const int r_in = warp * 32 + lane;
+            const uint32_t tb = tmem_base + ((uint32_t)(q4 * 32) << 16) + buf * BN;
+            const int r_in = q4 * 32 + lane;
             bool fin = true;
             if (ns > 1) {
                 // this split's partial tile, [BN columns][128 rows] fp32
                 float* mine = p.partials + ((int64_t)ks * p.MT * p.NT + tile) * (BN * 128) + r_in;
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 8) {
+                for (int c0 = cb; c0 < ce; c0 += 8) {
                     uint32_t r[8];
                     tmem_ld8(tb + c0, r);
                     tmem_wait_ld();
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                     break;
                 }
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 8) {
+                for (int c0 = cb; c0 < ce; c0 += 8) {
                     uint32_t r[8];
                     tmem_ld8(tb + c0, r);
                     tmem_wait_ld();
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                 const int kw0 = (p.HD - row0) / 32;      // first warp holding key rows (has_k)
                 const float g = kw ? __ldg(p.gamma + (base - p.HD) + lane) : 0.0f;
 #pragma unroll 1
-                for (int c0 = 0, cc = 0; c0 < BN; c0 += 8, ++cc) {
+                for (int c0 = cb, cc = 0; c0 < ce; c0 += 8, ++cc) {
                     uint32_t r[8];
                     tmem_ld8(tb + c0, r);
                     tmem_wait_ld();
@@ -457,7 +461,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
                                 const float s2 = warp_sum(v[j] * v[j]);
-                                if (lane == 0) m->red_ss[rb][warp][j] = s2;
+                                if (lane == 0) m->red_ss[half][rb][q4][j] = s2;
                             }
                         }
                         named_bar_sync(4, Cfg::EPI_THREADS);
@@ -469,7 +473,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                                 float ss = 0.0f;
 #pragma unroll
                                 for (int w = 0; w < 4; ++w)
-                                    if (w < p.D_I / 32) ss += m->red_ss[rb][kw0 + w][lane];
+                                    if (w < p.D_I / 32) ss += m->red_ss[half][rb][kw0 + w][lane];
                                 fac = rsqrtf(ss / (float)p.D_I + p.eps);
                             }
 #pragma unroll
@@ -480,7 +484,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
 #pragma unroll
                                 for (int j = 0; j < 8; ++j) {
                                     const float a = warp_max(fabsf(v[j]));
-                                    if (lane == 0) m->red_am[rb][warp][j] = a;
+                                    if (lane == 0) m->red_am[half][rb][q4][j] = a;
                                 }
                             }
                             named_bar_sync(5, Cfg::EPI_THREADS);
@@ -522,7 +526,7 @@ __global__ void __launch_bounds__(PrologCfg<BN>::THREADS, 1)
                             const bool first = ((base - p.HD) & 63) == 0;
                             float scl = 1.0f;
                             if (lane < 8) {
-                                const float a = fmaxf(m->red_am[rb][w0][lane], m->red_am[rb][w0 + 1][lane]);
+                                const float a = fmaxf(m->red_am[half][rb][w0][lane], m->red_am[half][rb][w0 + 1][lane]);
                                 scl = a > 0.0f ? a / 448.0f : 1.0f;
                             }
 #pragma unroll
